@@ -1,0 +1,103 @@
+"""Pins for the oracle's 4-bit group quantizers: closed-form blocks, the
+special cases of the scale rule, and the rounding-error bound that every
+element must meet."""
+import numpy as np
+
+from oracle import formats as F
+from oracle import svdquant as S
+
+
+def _block(vals, n=16):
+    v = np.zeros((1, n), np.float32)
+    v[0, :len(vals)] = vals
+    return v
+
+
+# --------------------------------------------------------------------- NVFP4 closed forms
+def test_nvfp4_closed_form_block():
+    # s_t = 1, amax 12 -> block scale 12 / 6 = 2 (E4M3 0x40), d = 2, inv = 0.5
+    q, s = S.quantize_nvfp4(_block([12, -12, 6, 3, 1, 0.5, -1, 0, 2.5, -5.5]), 1.0)
+    assert s.tolist() == [[0x40]]
+    # v * 0.5 = 6, -6, 3, 1.5, 0.5, 0.25(tie->0), -0.5, 0, 1.25(tie->1.0), -2.75(->-3)
+    assert q[0, :10].tolist() == [0x7, 0xF, 0x5, 0x3, 0x1, 0x0, 0x9, 0x0, 0x2, 0xD]
+
+
+def test_nvfp4_tensor_scale_enters_block_scale():
+    s_t = np.float32(0.125)                 # power of two: every step exact
+    q, s = S.quantize_nvfp4(_block([3.0, -1.5]), s_t)
+    # a / (6 s_t) = 3 / 0.75 = 4 -> E4M3 0x48 ; d = 4 * 0.125 = 0.5 ; inv = 2
+    assert s.tolist() == [[0x48]]
+    assert q[0, :2].tolist() == [0x7, 0xD]  # 6, -3
+
+
+def test_nvfp4_scale_saturates_at_448():
+    q, s = S.quantize_nvfp4(_block([3000.0, -1.0]), 1.0)
+    assert s.tolist() == [[0x7E]]            # 500 -> 448
+    assert q[0, 0] == 0x7                    # 3000/448 = 6.7 -> saturates to 6
+
+
+def test_nvfp4_zero_and_underflow_blocks_give_signed_zero_codes():
+    q, s = S.quantize_nvfp4(np.zeros((1, 16), np.float32), 1.0)
+    assert s.tolist() == [[0]] and np.all(q == 0)
+    tiny = _block([1e-6, -1e-6, -0.0])       # a / 6 = 1.7e-7 < 2^-10: scale rounds to 0
+    q, s = S.quantize_nvfp4(tiny, 1.0)
+    assert s.tolist() == [[0]]
+    assert q[0, :3].tolist() == [0x0, 0x8, 0x8]
+
+
+def test_nvfp4_error_bound_every_element():
+    """|dequant - v| <= half the E2M1 step at |v inv| (times d), unless the
+    code saturated; and the block scale is the nearest E4M3 value."""
+    rng = np.random.default_rng(5)
+    V = (rng.standard_normal((64, 256)) * np.exp(rng.uniform(-3, 3, (64, 1)))).astype(np.float32)
+    s_t = S.tensor_scale(V)
+    q, s = S.quantize_nvfp4(V, s_t)
+    sb = F.e4m3_decode(s).astype(np.float32)
+    d = (sb * s_t).astype(np.float32)
+    a = np.abs(V).reshape(64, 16, 16).max(axis=2)
+    target = (a / np.float32(6.0 * s_t)).astype(np.float64)
+    # scale: within half an E4M3 step of a / (6 s_t)
+    e = np.maximum(np.floor(np.log2(np.maximum(target, 2.0 ** -6))), -6)
+    assert np.all(np.abs(sb - target) <= 0.5 * 2.0 ** (e - 3) * (1 + 1e-9))
+    deq = F.e2m1_decode(q).reshape(64, 16, 16) * d[:, :, None]
+    x = (np.abs(V.reshape(64, 16, 16)) / d[:, :, None])
+    step = np.where(x < 2, 0.5, np.where(x < 4, 1.0, 2.0))
+    err = np.abs(deq - V.reshape(64, 16, 16))
+    ok = (err <= 0.5 * step * d[:, :, None] * (1 + 1e-6)) | (x > 6)
+    assert ok.all()
+
+
+def test_nvfp4_groups_run_along_k_per_row():
+    rng = np.random.default_rng(1)
+    V = rng.standard_normal((4, 64)).astype(np.float32)
+    _, s0 = S.quantize_nvfp4(V, 0.01)
+    V2 = V.copy()
+    V2[2, 37] = 50.0
+    _, s1 = S.quantize_nvfp4(V2, 0.01)
+    diff = np.argwhere(s0 != s1)
+    assert diff.tolist() == [[2, 37 // 16]]
+
+
+# --------------------------------------------------------------------- INT4
+def test_int4_closed_form_block():
+    v = np.zeros((1, 64), np.float32)
+    v[0, :6] = [7, -7, 3.5, 2.5, -0.5, 0.4]
+    q, s = S.quantize_int4(v)
+    assert s.dtype == np.float16 and float(s[0, 0]) == 1.0
+    assert q[0, :6].tolist() == [7, -7, 4, 2, 0, 0]
+
+
+def test_int4_error_bound_every_element():
+    rng = np.random.default_rng(9)
+    V = (rng.standard_normal((32, 256)) * np.exp(rng.uniform(-4, 4, (32, 1)))).astype(np.float32)
+    q, s = S.quantize_int4(V)
+    d = s.astype(np.float64)
+    deq = q.reshape(32, 4, 64) * d[:, :, None]
+    err = np.abs(deq - V.reshape(32, 4, 64))
+    # |v inv| can exceed 7 only by the fp16 rounding of a/7 (relative 2^-11)
+    assert np.all(err <= d[:, :, None] * (0.5 + 7 * 2.0 ** -10))
+
+
+def test_int4_zero_block():
+    q, s = S.quantize_int4(np.zeros((2, 128), np.float32))
+    assert np.all(q == 0) and np.all(s == 0)
