@@ -1,0 +1,407 @@
+"""Benchmark of the SVDQuant W4A4 linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload: the FLUX-like fused QKV projection, NVFP4, M = 4608 tokens (4096
+image + 512 text), K = 3072, N = 9216, rank 32, synthetic seeded inputs with
+the outlier recipe of workloads.py.  A step is one pass of the whole layer
+(kernel 1: quantize + low-rank down; kernel 2: block-scaled FP4 GEMM + fused
+low-rank up + bias) over the batch.  Metric: effective TFLOP/s = 2 M N K per
+step time (low-rank flops not counted), also reported as us/layer and as the
+fraction of the FP4 tensor peak.
+
+Timing: W untimed warm-up steps, then exactly K steps between a barrier and
+a device synchronize on both sides, timed with CUDA events on the launching
+stream; the slowest rank's time counts.  Each step uses the next of three
+rotating X / Y buffer sets (together larger than the 126 MB L2), so
+activations and outputs come from HBM.  Under torchrun every rank runs its
+own batch (weak scaling; no collective on the data path).
+
+--impl reference times the CPU oracle (float64 numpy) on the host cores on a
+bounded sample of the same workload, as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = dict(name="nvfp4_qkv_M4608_K3072_N9216_r32", fmt="nvfp4", M=4608, K=3072, N=9216, rank=32)
+METRIC = "SVDQuant W4A4 linear effective TFLOPS & % of FP4 tensor peak; µs/layer"
+UNIT = "TFLOP/s"
+FP4_PER_BF16 = 4.0          # nominal dense FP4 : BF16 tensor throughput (9 : 2.25 PFLOP/s)
+FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ------------------------------------------------------------------ helpers
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return dict(bf16=float(d["bf16_tflops"]), bf16_sustained=float(d.get("bf16_tflops_sustained", 0)) or None,
+                    hbm=float(d["hbm_gbs"]), source="measured")
+    except Exception:
+        return dict(bf16=FALLBACK_BF16_TFLOPS, bf16_sustained=None, hbm=FALLBACK_HBM_GBS, source="fallback")
+
+
+def file_sha(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic(profile_name, kernel_src):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the kernel source as it is now; else None."""
+    path = os.path.join(ROOT, "profiles", profile_name)
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    for line in open(path):
+        if ":" in line and line.strip().startswith(("dram_bytes_per_launch", "kernel_sha256", "units_scale")):
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("kernel_sha256") != file_sha(kernel_src):
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index, period_s=0.002):
+        self.ok = False
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self.period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            pass
+        self._stop = threading.Event()
+
+    def _sample(self):
+        self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+        self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+            try:
+                self._sample()
+            except Exception:
+                pass
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"]}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Largest value of x over all ranks (plumbing only: one float)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(flops_per_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job throughput in TFLOP/s: every rank did `steps` steps."""
+    return flops_per_step * steps * world / (max_ms * 1e-3) / 1e12
+
+
+# ------------------------------------------------------------------ the CPU oracle (baseline / reference arm)
+def oracle_setup():
+    import workloads
+    from oracle import svdquant as S
+    L = workloads.qkv()
+    pw = S.calibrate_and_prepare("nvfp4", L.X, L.W, L.bias, L.rank)
+    return L, pw
+
+
+def oracle_step(L, pw, rows, cols):
+    """Oracle forward on rows [0, rows) and output columns [0, cols) of the
+    workload: a slice of the prepared weights, no change to the oracle."""
+    import dataclasses
+    from oracle import svdquant as S
+    sub = dataclasses.replace(pw, N=cols, qR=pw.qR[:cols], sR=pw.sR[:cols], L2=pw.L2[:, :cols], bias=pw.bias[:cols])
+    return S.forward(sub, L.X[:rows])
+
+
+def oracle_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max(int(i.get("num_threads", 1)) for i in info) if info else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(L, pw, rows=1152, reps=3):
+    ts = []
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        oracle_step(L, pw, rows, L.N)
+        ts.append(time.perf_counter() - t0)
+    t = statistics.median(ts)
+    return {"value": round(2.0 * rows * L.N * L.K / t / 1e12, 6), "unit": UNIT, "cores": oracle_threads(),
+            "kind": "oracle",
+            "sample": "float64 numpy oracle forward (activation quantize, dequantized FP4 GEMM, low-rank "
+                      "down/up, bias) on rows 0..%d of the M=4608 QKV workload, all 9216 outputs; median of %d"
+                      % (rows - 1, reps),
+            "seconds_per_sample": round(t, 3)}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    L, pw = oracle_setup()
+    # size the per-step sample so that warm-up + steps take about two minutes
+    rows, cols = 64, 512
+    t0 = time.perf_counter()
+    oracle_step(L, pw, rows, cols)
+    t1 = time.perf_counter() - t0
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    scale = max(budget / max(t1, 1e-6), 1e-3)
+    cols = int(min(L.N, max(16, cols * scale)) // 16 * 16)
+    for _ in range(args.warmup):
+        oracle_step(L, pw, rows, cols)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(L, pw, rows, cols)
+    el = time.perf_counter() - t0
+    value = 2.0 * rows * cols * L.K * args.steps / el / 1e12
+    out = {"metric": METRIC, "value": round(value, 6), "unit": UNIT, "impl": "reference", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 4),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic (seeded, FLUX-shaped, outlier channels)",
+           "config": {"workload": WORKLOAD["name"], "M": L.M, "K": L.K, "N": L.N, "rank": L.rank,
+                      "format": "nvfp4", "sample_rows": rows, "sample_cols": cols},
+           "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "kind": "oracle", "cores": oracle_threads(),
+                            "sample": "oracle forward on rows 0..%d x output columns 0..%d per step"
+                                      % (rows - 1, cols - 1)},
+           "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+def gpu_factors(B, Wt, X, rank, torch):
+    """Offline quantizer step on the GPU: smoothing factors and activation
+    scale with the library's calibration kernel, then the SVD of W^ with
+    torch.linalg.svd (cuSOLVER), folded like the library expects."""
+    M, K = X.shape
+    N = Wt.shape[0]
+    lam = torch.empty(K, dtype=torch.float32, device="cuda")
+    act = torch.empty(1, dtype=torch.float32, device="cuda")
+    ws = torch.empty(B.svdq_calibrate_workspace_bytes(K), dtype=torch.uint8, device="cuda")
+    B.svdq_calibrate(M, K, N, X, Wt, 0.5, lam, act, ws)
+    What = (lam[:, None].double() * Wt.t().double()).float()
+    U, Sv, Vh = torch.linalg.svd(What, full_matrices=False)
+    L1f = ((U[:, :rank].double() * Sv[:rank].double()) / lam[:, None].double()).to(torch.bfloat16).contiguous()
+    L2 = Vh[:rank].to(torch.bfloat16).contiguous()
+    torch.cuda.synchronize()
+    return lam, float(act.item()), L1f, L2
+
+
+def run_ours(args, world, rank, local):
+    import numpy as np
+    import torch
+    import workloads
+    from rank_gemm_b200 import build as _b
+    if rank == 0:
+        _b.build()
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", init_method="env://", world_size=world, rank=rank,
+                                timeout=__import__("datetime").timedelta(seconds=120))
+        dist.barrier()
+    from rank_gemm_b200 import binding as B
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    Lw = workloads.qkv()
+    M, K, N, r = Lw.M, Lw.K, Lw.N, Lw.rank
+    X0 = torch.from_numpy(Lw.X).to(torch.bfloat16).to(dev)
+    Wt = torch.from_numpy(np.ascontiguousarray(Lw.W.T)).to(torch.bfloat16).to(dev)
+    bias = torch.from_numpy(Lw.bias).to(torch.bfloat16).to(dev)
+    lam, act, L1f, L2 = gpu_factors(B, Wt, X0, r, torch)
+    h = B.svdq_prepare_weights("nvfp4", K, N, r, Wt, lam, L1f, L2, bias, None, None, 0, act)
+
+    sets = 3
+    Xs = [X0] + [X0.clone() for _ in range(sets - 1)]
+    Ys = [torch.empty(M, N, dtype=torch.bfloat16, device=dev) for _ in range(sets)]
+    qb, sb, lb = B.svdq_act_buffer_sizes(h, M)
+    acts = [(torch.empty(qb, dtype=torch.uint8, device=dev), torch.empty(sb, dtype=torch.uint8, device=dev),
+             torch.empty(lb, dtype=torch.uint8, device=dev)) for _ in range(sets)]
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        qX, sX, LR = acts[i % sets]
+        B.svdq_quantize_act_lowrank_down(h, M, Xs[i % sets], qX, sX, LR, stream)
+        ev_mid[i].record(stream)
+        B.svdq_w4a4_gemm_lowrank_up(h, M, qX, sX, LR, B.SVDQ_EPI_NONE, Ys[i % sets], stream)
+
+    K_steps, W_steps = args.steps, args.warmup
+    ev_mid = [torch.cuda.Event(enable_timing=True) for _ in range(max(K_steps, W_steps))]
+    for i in range(W_steps):
+        step(i)
+    torch.cuda.synchronize()
+    assert B.svdq_poll_device_error(stream) == 0
+
+    ev_beg = [torch.cuda.Event(enable_timing=True) for _ in range(K_steps)]
+    ev_end = [torch.cuda.Event(enable_timing=True) for _ in range(K_steps)]
+    t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t_start.record(stream)
+        for i in range(K_steps):
+            ev_beg[i].record(stream)
+            step(i)
+            ev_end[i].record(stream)
+        t_stop.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    total_ms = t_start.elapsed_time(t_stop)
+    status = B.svdq_poll_device_error(stream)
+    max_ms = max_over_ranks(total_ms, world, dev)
+    k1_ms = statistics.mean(ev_beg[i].elapsed_time(ev_mid[i]) for i in range(K_steps))
+    k2_ms = statistics.mean(ev_mid[i].elapsed_time(ev_end[i]) for i in range(K_steps))
+
+    flops = 2.0 * M * N * K
+    value = weak_scaling_value(flops, K_steps, world, max_ms)
+    peaks = measured_peaks()
+    fp4_peak = peaks["bf16"] * FP4_PER_BF16
+    k2_tflops = flops / (k2_ms * 1e-3) / 1e12
+    bytes_k1 = M * K * 2 + K * 4 + r * K * 2 + qb + sb + lb
+    bytes_k2 = qb + sb + lb + (N * K // 2) + (N * K // 16) + N * 64 * 2 + N * 4 + M * N * 2
+    traffic = profiled_traffic("gemm_nvfp4_qkv.md", os.path.join(ROOT, "rank_gemm_b200", "csrc", "gemm_nvfp4.cu"))
+
+    # end to end through the public call with host buffers
+    e2e_steps = min(K_steps, 50)
+    Xh = torch.empty(M, K, dtype=torch.bfloat16, pin_memory=True)
+    Xh.copy_(X0.cpu())
+    Yh = torch.empty(M, N, dtype=torch.bfloat16, pin_memory=True)
+    ws = torch.empty(B.svdq_linear_workspace_bytes(h, M), dtype=torch.uint8, device=dev)
+    Xd, Yd = Xs[0], Ys[0]
+    for _ in range(3):
+        Xd.copy_(Xh, non_blocking=True)
+        B.svdq_linear(h, M, Xd, B.SVDQ_EPI_NONE, Yd, ws, None, stream)
+        Yh.copy_(Yd, non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        Xd.copy_(Xh, non_blocking=True)
+        B.svdq_linear(h, M, Xd, B.SVDQ_EPI_NONE, Yd, ws, None, stream)
+        Yh.copy_(Yd, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / e2e_steps
+    e2e_value = flops * world / (e2e_ms * 1e-3) / 1e12
+
+    out = None
+    if rank == 0:
+        out = {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": K_steps,
+               "warmup": W_steps, "ms_per_step": round(max_ms / K_steps, 5), "us_per_layer": round(max_ms / K_steps * 1e3, 2),
+               "fp4_peak_frac": round(value / world / fp4_peak, 4), "higher_is_better": True, "scaling": "weak",
+               "vs_baseline": None, "dtype": "nvfp4",
+               "data": "synthetic (seeded, FLUX-shaped, 0.5% outlier channels x20 / x5), random-init weights",
+               "config": {"workload": WORKLOAD["name"], "M": M, "K": K, "N": N, "rank": r, "format": "nvfp4",
+                          "group": 16, "parallelism": "replicas x%d (each rank its own batch)" % world,
+                          "l2": "3 rotating X/Y/workspace sets (%.0f MB) > 126 MB L2"
+                                % (sets * (M * K * 2 + M * N * 2 + qb + sb + lb) / 1e6)},
+               "roofline": {"kernel": "gemm_nvfp4 (kernel 2)", "bound": "tensor", "achieved": round(k2_tflops, 2),
+                            "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(k2_tflops / fp4_peak, 4),
+                            "peak_source": "%s bf16 %.1f TFLOP/s x %.0f (nominal FP4:BF16)"
+                                           % (peaks["source"], peaks["bf16"], FP4_PER_BF16),
+                            "traffic": traffic, "algorithmic_bytes": bytes_k2, "us": round(k2_ms * 1e3, 2)},
+               "roofline_k1": {"kernel": "quant_down (kernel 1)", "bound": "hbm",
+                               "achieved": round(bytes_k1 / (k1_ms * 1e-3) / 1e9, 1), "peak": peaks["hbm"],
+                               "unit": "GB/s", "frac": round(bytes_k1 / (k1_ms * 1e-3) / 1e9 / peaks["hbm"], 4),
+                               "algorithmic_bytes": bytes_k1, "us": round(k1_ms * 1e3, 2)},
+               "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": M * K * 2,
+                       "d2h_bytes_per_step": M * N * 2, "ms_per_step": round(e2e_ms, 4)},
+               "gpu_launches": 2 * K_steps,
+               "device_status": status,
+               "clocks": clocks.summary()}
+    B.svdq_free_weights(h)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            L, pw = oracle_setup()
+            out["cpu_baseline"] = cpu_baseline(L, pw)
+        print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+    else:
+        run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

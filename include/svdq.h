@@ -1,0 +1,257 @@
+/*
+ * svdq.h -- C ABI of the SVDQuant W4A4 linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer (SVDQuant overview figure, Stages 2 and 3, "svdq-int4-flux.1-dev"
+ * model card; abstract of "SVDQuant: Absorbing Outliers by Low-Rank Components
+ * for 4-Bit Diffusion Models"):
+ *
+ *     Y = X^ L1 L2  +  Q(X^) Q(R)  +  b,      X^ = X diag(lambda)^-1,
+ *     W^ = diag(lambda) W ~= L1 L2 + R   (rank-r SVD split, R quantized to 4 bits)
+ *
+ * computed as two fused kernels ("Nunchaku engine design" figure (b) of the
+ * same model card: the down projection shares its input with the quantize
+ * kernel, the up projection shares its output with the 4-bit GEMM):
+ *
+ *     kernel 1  svdq_quantize_act_lowrank_down : X -> (qX, sX, LR = X L1f)
+ *     kernel 2  svdq_w4a4_gemm_lowrank_up      : (qX, sX, LR) -> Y
+ *
+ * Conventions shared by every call
+ *   - Shapes: M tokens (rows of X and Y), K input features, N output features.
+ *     The math weight is W (K x N); the API takes it in nn.Linear order
+ *     W_t[N][K] (row n = output feature n), because the layer replaces an
+ *     nn.Linear (Diffusers blog, "Introducing Nunchaku Lite").
+ *   - Requirements: K % 64 == 0, N % 16 == 0, M >= 0 (M == 0 is a no-op),
+ *     rank + lora_rank a multiple of 16 in [16, 256].
+ *   - "dev" pointers are device memory of the current CUDA device; "host"
+ *     pointers are host memory.  Every device pointer must be 16-byte aligned.
+ *   - The caller owns X, Y, qX, sX, LR and any workspace; their sizes come from
+ *     the query calls.  The library owns the buffers behind an svdq_weights
+ *     handle and frees them in svdq_free_weights.
+ *   - Launches are asynchronous on `stream` (0 = legacy default stream).
+ *     Argument, shape and alignment errors are returned before anything is
+ *     launched.  A kernel that detects a problem while running (a wait that
+ *     exceeded its time limit, a failed bounds check) records it in a device
+ *     error word; svdq_poll_device_error() reports it.
+ *   - Every call returns SVDQ_ERR_UNSUPPORTED_DEVICE unless the current
+ *     device has compute capability 10.0, instead of producing wrong output
+ *     (Diffusers blog, "Hardware support": unsupported GPUs are rejected at
+ *     load time with a clear error).  There is no CPU fallback.
+ *   - No call aborts the process or throws across the ABI.
+ *
+ * Library-defined layouts (svdq_weights_view reports them):
+ *   K_pad = K rounded up to a multiple of 256, r_tot = rank + lora_rank,
+ *   r_pad = r_tot rounded up to a multiple of 64.
+ *   qX    uint8 [M][K_pad/2]: two 4-bit codes per byte, even k in the low
+ *         nibble; columns k >= K hold code 0.
+ *   sX    NVFP4: E4M3 block scales (one per 16 k) in tcgen05 scale-factor
+ *         atoms: atom (i, j) for rows 128i..128i+127 and k in [64j, 64j+64)
+ *         is 512 contiguous bytes at ((i * K_pad/64) + j) * 512; inside it
+ *         the scale of row r and 16-group g (0..3) sits at byte
+ *         (r % 32) * 16 + ((r % 128) / 32) * 4 + g.  Rows >= M hold 0.
+ *         INT4: binary16 block scales (one per 64 k), row-major
+ *         [M_pad128][K_pad/64]; rows >= M and columns >= K/64 hold 0.
+ *   LR    bf16 [M][r_pad]: X L1f for the r_tot low-rank columns, zeros after.
+ */
+#ifndef SVDQ_H_
+#define SVDQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SVDQ_OK = 0,
+  SVDQ_ERR_INVALID_ARG = 1,        /* null pointer, unknown enum, bad scalar */
+  SVDQ_ERR_SHAPE = 2,              /* dimension outside the requirements above */
+  SVDQ_ERR_ALIGNMENT = 3,          /* a device pointer is not 16-byte aligned */
+  SVDQ_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not compute capability 10.0 */
+  SVDQ_ERR_WORKSPACE = 5,          /* workspace missing or smaller than required */
+  SVDQ_ERR_CUDA = 6,               /* a CUDA runtime or driver call failed */
+  SVDQ_ERR_TIMEOUT = 7,            /* a device-side wait exceeded its time limit */
+  SVDQ_ERR_DEVICE_FAULT = 8,       /* a device-side bounds or consistency check failed */
+  SVDQ_ERR_NO_MEMORY = 9           /* device allocation for a weight handle failed */
+} svdq_status;
+
+typedef enum { SVDQ_NVFP4 = 0, SVDQ_INT4 = 1 } svdq_format;
+
+typedef enum { SVDQ_EPI_NONE = 0, SVDQ_EPI_GELU_TANH = 1 } svdq_epilogue;
+
+/* Opaque, library-owned prepared weights of one layer. */
+typedef struct svdq_weights svdq_weights;
+
+/* Read-only view of a handle (device pointers stay owned by the handle). */
+typedef struct {
+  int fmt;                 /* svdq_format */
+  int K, N, rank, lora_rank, r_tot;
+  int K_pad, N_pad, r_pad; /* N_pad = N rounded up to a multiple of 256 */
+  const void* qR;          /* dev uint8 [N_pad][K_pad/2], packed like qX (rows = output features) */
+  const void* sR;          /* dev: NVFP4 E4M3 atoms like sX over N_pad rows; INT4 binary16 [N_pad][K_pad/64] */
+  const void* L1t;         /* dev bf16 [r_tot][K]: (lambda^-1-folded L1 | LoRA A), transposed */
+  const void* L2a;         /* dev bf16 [N_pad][r_pad]: (L2 ; LoRA B) transposed, divided by alpha */
+  const void* bias;        /* dev float32 [N_pad] (zeros if no bias was given) */
+  const float* lambda_inv; /* dev float32 [K]: correctly rounded 1/lambda */
+  float s_tR;              /* NVFP4 weight tensor scale (1 for INT4) */
+  float s_tX;              /* NVFP4 static activation tensor scale (1 for INT4) */
+  float alpha;             /* s_tX * s_tR in float32 */
+} svdq_weights_info;
+
+/* ------------------------------------------------------------------------
+ * Offline calibration (SVDQuant overview figure, Stage 2: outliers migrate
+ * from the activation to the weight).
+ *
+ * lambda_k = max_m|X[m,k]|^alpha / max_n|W[k,n]|^(1-alpha), in float64,
+ * rounded once to float32 (1 where either maximum is 0); then
+ * act_scale = max|fl32(X[m,k] * fl32(1/lambda_k))| / 2688 (the static NVFP4
+ * activation tensor scale; 1 if that maximum is 0).
+ *   X          dev bf16 [M][K]    calibration activation
+ *   W_t        dev bf16 [N][K]    weight in nn.Linear order
+ *   alpha      migration strength in [0, 1]
+ *   lambda_out dev float32 [K]    written
+ *   act_scale_out dev float32 [1] written
+ *   workspace  dev, at least svdq_calibrate_workspace_bytes(K) bytes, 16-aligned
+ * Errors: INVALID_ARG (null, alpha outside [0,1]), SHAPE, ALIGNMENT,
+ *         WORKSPACE, UNSUPPORTED_DEVICE, CUDA.
+ * ------------------------------------------------------------------------ */
+size_t svdq_calibrate_workspace_bytes(int K);
+svdq_status svdq_calibrate(int M, int K, int N, const void* X, const void* W_t, float alpha,
+                           float* lambda_out, float* act_scale_out, void* workspace,
+                           size_t ws_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Offline weight preparation (Stage 3 of the overview figure: W^ splits into
+ * a 16-bit rank-r branch and a 4-bit residual; abstract: LoRAs join the
+ * low-rank branch without re-quantizing the residual).
+ *
+ * Given the folded low-rank factors L1f = bf16(diag(lambda)^-1 U_r S_r)
+ * (K x rank) and L2 = bf16(V_r^T) (rank x N) from a truncated SVD of
+ * W^ = diag(lambda) W, computes on the device
+ *     R[k,n] = fp32(lambda_k W[k,n] - lambda_k sum_{i<rank} L1f[k,i] L2[i,n])
+ * (float64, i ascending, no fused multiply-add), the NVFP4 tensor scale
+ * s_tR = max|R| / 2688, the 4-bit codes and block scales of R per output
+ * column (groups of 16 along K for NVFP4, 64 for INT4), and the layouts the
+ * kernels consume.  A LoRA (A: K x lora_rank, B: lora_rank x N) is appended
+ * to the factors: L1' = [L1f | A], L2' = [L2 ; B]; R does not change.
+ *   fmt        SVDQ_NVFP4 or SVDQ_INT4
+ *   W_t        dev bf16 [N][K]
+ *   lambda     dev float32 [K]    smoothing factors (see svdq_calibrate)
+ *   L1f        dev bf16 [K][rank] row-major
+ *   L2         dev bf16 [rank][N] row-major
+ *   bias       dev bf16 [N] or NULL (no bias)
+ *   lora_A     dev bf16 [K][lora_rank] or NULL (then lora_rank must be 0)
+ *   lora_B     dev bf16 [lora_rank][N] or NULL
+ *   act_scale  NVFP4 static activation tensor scale s_tX (> 0, finite);
+ *              ignored for INT4
+ *   out        host: receives the new handle (NULL on error)
+ * The call synchronizes `stream` before returning.  Errors: INVALID_ARG,
+ * SHAPE, ALIGNMENT, UNSUPPORTED_DEVICE, NO_MEMORY, CUDA; nothing is leaked.
+ * ------------------------------------------------------------------------ */
+svdq_status svdq_prepare_weights(svdq_format fmt, int K, int N, int rank, const void* W_t,
+                                 const float* lambda, const void* L1f, const void* L2,
+                                 const void* bias, const void* lora_A, const void* lora_B,
+                                 int lora_rank, float act_scale, cudaStream_t stream,
+                                 svdq_weights** out);
+
+/* Frees the handle and its device buffers (synchronizes the device first).
+ * NULL is accepted and ignored. */
+svdq_status svdq_free_weights(svdq_weights* w);
+
+/* Fills *info with the handle's layout and device pointers. */
+svdq_status svdq_weights_view(const svdq_weights* w, svdq_weights_info* info);
+
+/* Sizes in bytes of the caller-owned intermediates for M rows (any pointer
+ * may be NULL to skip it). */
+svdq_status svdq_act_buffer_sizes(const svdq_weights* w, int M, size_t* qx_bytes,
+                                  size_t* sx_bytes, size_t* lr_bytes);
+
+/* ------------------------------------------------------------------------
+ * Kernel 1 -- quantize + low-rank down projection, fused ("Nunchaku engine
+ * design" figure (b): both read the same input, so X is read from HBM once).
+ *   x^ = fl32(x * lambda_inv_k); per row and 16- (NVFP4) or 64- (INT4)
+ *   group: amax -> block scale -> 4-bit codes, exactly as svdq_prepare_weights
+ *   quantizes R, with the handle's s_tX as the NVFP4 tensor scale;
+ *   LR = bf16(X L1') with float32 accumulation.
+ *   X   dev bf16 [M][K]
+ *   qX, sX, LR  dev, sizes from svdq_act_buffer_sizes, layouts above
+ * Errors: INVALID_ARG, SHAPE, ALIGNMENT, UNSUPPORTED_DEVICE, CUDA.
+ * ------------------------------------------------------------------------ */
+svdq_status svdq_quantize_act_lowrank_down(const svdq_weights* w, int M, const void* X,
+                                           void* qX, void* sX, void* LR, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Kernel 2 -- 4-bit GEMM + low-rank up projection, fused (figure (b): both
+ * write the same output, so the 16-bit branch adds no HBM round trip).
+ *   y[m,n] = alpha * ( sum_k dq(qX)[m,k] dq(qR)[n,k] + sum_i LR[m,i] L2a[n,i] ) + b[n]
+ *   (NVFP4: block-scaled tensor-core MMA with E4M3 scales per 16; INT4:
+ *   int8 MMA per 64-group, rescaled by sX[m,g] sR[n,g]); optional GELU (tanh
+ *   form); Y = bf16(y).
+ *   qX, sX, LR  dev, as written by kernel 1 (or by an equivalent producer)
+ *   Y   dev bf16 [M][N] row-major
+ * Errors: INVALID_ARG, SHAPE, ALIGNMENT, UNSUPPORTED_DEVICE, CUDA.
+ * ------------------------------------------------------------------------ */
+svdq_status svdq_w4a4_gemm_lowrank_up(const svdq_weights* w, int M, const void* qX,
+                                      const void* sX, const void* LR, svdq_epilogue epi,
+                                      void* Y, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * The whole layer: kernel 1 then kernel 2 on `stream`, with qX, sX and LR
+ * placed in the caller's workspace.
+ *   X  dev bf16 [M][K];  Y  dev bf16 [M][N]
+ *   workspace  dev, at least svdq_linear_workspace_bytes(w, M) bytes
+ * Errors: as kernels 1 and 2, plus WORKSPACE.
+ * ------------------------------------------------------------------------ */
+size_t svdq_linear_workspace_bytes(const svdq_weights* w, int M);
+svdq_status svdq_linear(const svdq_weights* w, int M, const void* X, svdq_epilogue epi, void* Y,
+                        void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Unfused baseline ("Nunchaku engine design" figure (a): run naively, the
+ * rank-32 branch costs an extra 16-bit read of X in the down projection and
+ * an extra 16-bit write of Y in the up projection, 57% latency overhead).
+ * These exist to measure that overhead against the fused path; they compute
+ * the same codes, scales and LR as kernel 1.
+ *   svdq_quantize_act     X -> qX, sX           (no low-rank work)
+ *   svdq_lowrank_down     X -> LR               (reads X again)
+ *   svdq_w4a4_gemm        qX, sX -> Y = bf16(alpha acc + b)   (no low-rank, no GELU)
+ *   svdq_lowrank_up       Y <- bf16(epi(Y + alpha LR L2a))    (read-modify-write of Y)
+ *   svdq_linear_unfused   the four above in order; same workspace as svdq_linear
+ * ------------------------------------------------------------------------ */
+svdq_status svdq_quantize_act(const svdq_weights* w, int M, const void* X, void* qX, void* sX,
+                              cudaStream_t stream);
+svdq_status svdq_lowrank_down(const svdq_weights* w, int M, const void* X, void* LR,
+                              cudaStream_t stream);
+svdq_status svdq_w4a4_gemm(const svdq_weights* w, int M, const void* qX, const void* sX,
+                           void* Y, cudaStream_t stream);
+svdq_status svdq_lowrank_up(const svdq_weights* w, int M, const void* LR, svdq_epilogue epi,
+                            void* Y, cudaStream_t stream);
+svdq_status svdq_linear_unfused(const svdq_weights* w, int M, const void* X, svdq_epilogue epi,
+                                void* Y, void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Diagnostics.
+ * svdq_poll_device_error: synchronizes `stream`, then reads and clears the
+ *   current device's error word.  Returns SVDQ_OK, SVDQ_ERR_TIMEOUT (a wait
+ *   ran out; the kernel that hit it skipped the rest of its work and
+ *   returned), SVDQ_ERR_DEVICE_FAULT, or SVDQ_ERR_CUDA (the stream itself
+ *   reported an error).
+ * svdq_selftest_wait_timeout: launches one CTA that waits on a barrier
+ *   nothing will complete, with a wait limit of `limit_us` microseconds;
+ *   the bounded wait must give up, set the error word and return, leaving
+ *   the context usable.  Used to test the timeout path without a fault.
+ * svdq_status_string: static English text for a status (never NULL).
+ * ------------------------------------------------------------------------ */
+svdq_status svdq_poll_device_error(cudaStream_t stream);
+svdq_status svdq_selftest_wait_timeout(unsigned limit_us, cudaStream_t stream);
+const char* svdq_status_string(svdq_status s);
+
+/* Test hook: pretend the device has compute capability major.minor for the
+ * capability check (major < 0 restores the real value). */
+void svdq_debug_override_cc(int major, int minor);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SVDQ_H_ */

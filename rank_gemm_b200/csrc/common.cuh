@@ -1,0 +1,324 @@
+// common.cuh -- device building blocks for the SVDQuant W4A4 kernels (sm_100a).
+//
+// Inline-PTX wrappers for mbarriers, TMA (cp.async.bulk[.tensor]) and the
+// 5th-generation tensor core (tcgen05: TMEM allocation, MMA, smem->TMEM copy,
+// TMEM loads), bounded waits that report a timeout instead of hanging, and
+// the 4-bit group quantizer shared by the activation kernel and the weight
+// preparation (so activations and the residual follow one rounding rule).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace svdq {
+
+// ----------------------------------------------------------------- error word
+// Bits OR-ed into the per-device error word (see api.cu).
+constexpr unsigned ERR_TIMEOUT = 1u;
+constexpr unsigned ERR_BOUNDS = 2u;
+
+struct DeviceErr {
+  unsigned* word;          // device error word
+  unsigned long long limit_ns;  // wait limit for every bounded wait
+};
+
+__device__ __forceinline__ void raise_error(const DeviceErr& e, unsigned bits) {
+  atomicOr(e.word, bits);
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// ----------------------------------------------------------------- addresses
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ----------------------------------------------------------------- mbarrier
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for the phase with the given parity to complete.  Gives up after
+// err.limit_ns (or as soon as another thread of the CTA has given up, seen
+// through *abort), records ERR_TIMEOUT and returns false.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+                                          const DeviceErr& err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > err.limit_ns) {
+      *abort = 1;
+      __threadfence_block();
+      raise_error(err, ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// ----------------------------------------------------------------- TMA
+__device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
+}
+
+// 2-D tiled load of the box at (x = inner coordinate, y = row) into smem.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+// Contiguous bulk copy global -> smem (both 16-byte aligned, bytes % 16 == 0).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// ----------------------------------------------------------------- tcgen05
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Arrives once on `bar` when every tcgen05 operation this thread issued
+// before has completed.
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+
+// Shared-memory matrix descriptor (tcgen05 "matrix descriptor"):
+//   bits  0-13 start address >> 4, 16-29 leading byte offset >> 4,
+//   32-45 stride byte offset >> 4, 46-47 version (1 on sm_100),
+//   49-51 base offset, 52 leading-offset mode, 61-63 swizzle mode
+//   (0 none, 2 = 128-byte swizzle).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo,
+                                              uint32_t swizzle) {
+  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | ((uint64_t)swizzle << 61);
+}
+
+// K-major operand tile with 128-byte rows in the 128-byte swizzle layout
+// written by TMA (8-row groups 1024 bytes apart).
+__device__ __forceinline__ uint64_t desc_k_sw128(uint32_t addr) {
+  return smem_desc(addr, 16, 1024, 2);
+}
+
+// Instruction descriptor, kind::f16 with bf16 A/B, fp32 accumulate, K-major A and B.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+// Instruction descriptor, kind::mxf4nvf4 block-scaled: E2M1 A/B, UE4M3 scales
+// (16-element blocks), K-major A and B, dense K = 64.
+__host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
+  return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | (0u << 23) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], "
+      "p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Copies a 512-byte scale-factor atom (32 rows x 16 bytes, contiguous in smem)
+// to 4 TMEM columns starting at `taddr`, replicated into all four 32-lane
+// sub-partitions.
+__device__ __forceinline__ void tmem_cp_sf_atom(uint32_t taddr, uint32_t smem_addr) {
+  const uint64_t d = smem_desc(smem_addr, 0, 128, 0);
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d)
+               : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns -> 32 registers per thread.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ----------------------------------------------------------------- conversions
+// Eight non-negative floats -> eight E2M1 magnitude codes in one word
+// (element j in bits 4j..4j+3), round to nearest even, saturate to 6.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(float x0, float x1, float x2, float x3, float x4,
+                                               float x5, float x6, float x7) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(x0), "f"(x1), "f"(x2), "f"(x3), "f"(x4), "f"(x5), "f"(x6), "f"(x7));
+  return r;
+}
+
+// Non-negative float -> E4M3 byte, round to nearest even, saturate to 448.
+__device__ __forceinline__ uint32_t cvt_e4m3(float x) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
+  return r & 0xFFu;
+}
+
+__device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
+  // E4M3 -> f32 exactly: bias 7, 3 mantissa bits, subnormals at 2^-9 steps.
+  const uint32_t e = (code >> 3) & 15u, m = code & 7u;
+  float v = e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : (float)m * 0.001953125f;
+  return (code & 0x80u) ? -v : v;
+}
+
+// ----------------------------------------------------------------- 4-bit group quantizers
+// NVFP4, one 16-element group: a = max|v|; sb = E4M3(a / six_st) with six_st
+// = fl32(6 s_t); d = fl32(f32(sb) s_t); inv = fl32(1/d) (0 if d == 0);
+// code_j = E2M1(fl32(v_j inv)), sign kept.  Returns the 16 codes packed in 8
+// bytes (element 2j in the low nibble of byte j) and the scale byte.
+__device__ __forceinline__ void quant_nvfp4_16(const float (&v)[16], float s_t, float six_st,
+                                               uint2& codes, uint32_t& scale) {
+  float a = 0.f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) a = fmaxf(a, fabsf(v[j]));
+  const uint32_t sb = cvt_e4m3(__fdiv_rn(a, six_st));
+  const float d = __fmul_rn(e4m3_to_f32(sb), s_t);
+  const float inv = (d == 0.f) ? 0.f : __frcp_rn(d);
+  uint32_t w[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float x[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) x[j] = __fmul_rn(v[8 * h + j], inv);
+    // magnitude from the converter, sign from the input: a negative value
+    // that rounds to zero keeps its sign (code 0x8)
+    uint32_t c = cvt_e2m1x8(fabsf(x[0]), fabsf(x[1]), fabsf(x[2]), fabsf(x[3]), fabsf(x[4]),
+                            fabsf(x[5]), fabsf(x[6]), fabsf(x[7]));
+#pragma unroll
+    for (int j = 0; j < 8; ++j) c |= (__float_as_uint(x[j]) >> 31) << (4 * j + 3);
+    w[h] = c;
+  }
+  codes = make_uint2(w[0], w[1]);
+  scale = sb;
+}
+
+// INT4, one 64-element group held as 4 x 16 values by 4 cooperating lanes
+// (lanes l, l^1, l^2, l^3 of one quad): sb = fp16(fl32(a / 7)),
+// d = f32(sb), inv = fl32(1/d) (0 if d == 0), code = clamp(rint(fl32(v inv)), -8, 7).
+// Each lane returns its 16 codes as 8 bytes (two's-complement nibbles).
+__device__ __forceinline__ void quant_int4_16of64(const float (&v)[16], uint2& codes,
+                                                  __half& scale) {
+  float a = 0.f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) a = fmaxf(a, fabsf(v[j]));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+  const __half sb = __float2half_rn(__fdiv_rn(a, 7.0f));
+  const float d = __half2float(sb);
+  const float inv = (d == 0.f) ? 0.f : __frcp_rn(d);
+  uint32_t w[2] = {0u, 0u};
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    int q = __float2int_rn(__fmul_rn(v[j], inv));
+    q = max(-8, min(7, q));
+    w[j >> 3] |= ((uint32_t)q & 0xFu) << ((j & 7) * 4);
+  }
+  codes = make_uint2(w[0], w[1]);
+  scale = sb;
+}
+
+// Byte offset of (row, 16-group) inside the tcgen05 scale-factor layout:
+// 512-byte atoms of 128 rows x 4 groups, ordered (row block, 64-k block).
+__host__ __device__ __forceinline__ size_t sf_atom_offset(int row, int g16, int kpad) {
+  const int rb = row >> 7, kb = g16 >> 2;
+  return ((size_t)rb * (kpad >> 6) + kb) * 512 + (size_t)(row & 31) * 16 + ((row & 127) >> 5) * 4 +
+         (g16 & 3);
+}
+
+__host__ __device__ constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+}  // namespace svdq

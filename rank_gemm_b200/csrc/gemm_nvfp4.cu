@@ -1,0 +1,254 @@
+// gemm_nvfp4.cu -- kernel 2 for NVFP4: the 4-bit GEMM fused with the low-rank
+// up projection ("Nunchaku engine design" figure (b), "svdq-int4-flux.1-dev"
+// model card: Up Projection and 4-Bit Compute share their output, so the
+// 16-bit branch is accumulated into the same output tile and Y is written
+// once).
+//
+// Persistent, warp-specialized, one 128 x 256 output tile per CTA at a time:
+//   warp 0      TMA producer: per 256-wide k-tile, the [128 x 128 B] tile of qX,
+//               the [256 x 128 B] tile of qR (both 128-byte swizzled) and the
+//               2 + 4 KB of E4M3 scale atoms (plain bulk copies); then, per
+//               64-wide chunk of the low-rank dimension, the [128 x 64] bf16 tile
+//               of LR and the [256 x 64] bf16 tile of L2/alpha, into the same
+//               ring slots (a bf16 tile of 64 columns has the byte shape of an
+//               FP4 tile of 256 columns).
+//   warp 1      TMEM owner and single-thread MMA issuer: tcgen05.cp moves the
+//               scale atoms to TMEM, tcgen05.mma.kind::mxf4nvf4 (block16,
+//               E4M3 scales) accumulates Q(X^) Q(R) in a 128 x 256 fp32 TMEM
+//               tile, then tcgen05.mma.kind::f16 adds LR (L2/alpha) into the
+//               same tile; tcgen05.commit releases ring slots and hands the
+//               finished tile to the epilogue.
+//   warps 2-5   epilogue: tcgen05.ld 32 columns at a time, y = alpha acc + b,
+//               optional GELU, bf16, 16-byte stores of each row segment.
+// All waits are bounded (see mbar_wait); TMEM is freed on every exit path.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace svdq {
+
+namespace {
+
+constexpr int BLOCK_M = 128, BLOCK_N = 256, STAGES = 4;
+constexpr int A_BYTES = BLOCK_M * 128;          // 16 KB
+constexpr int B_BYTES = BLOCK_N * 128;          // 32 KB
+constexpr int SFA_BYTES = 4 * 512;              // 4 k-blocks of 64 x 128 rows
+constexpr int SFB_BYTES = 2 * 4 * 512;          // 2 row halves x 4 k-blocks
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;   // 54 KB
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t ACC_COL = 0, SFA_COL = 256, SFB_COL = 272;
+constexpr uint32_t IDESC_F4 = idesc_nvf4(BLOCK_M, BLOCK_N);
+constexpr uint32_t IDESC_BF = idesc_bf16_f32(BLOCK_M, BLOCK_N);
+
+struct Ctl {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tfull, tempty;
+  uint32_t tmem_base;
+  int abort;
+};
+
+constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 + sizeof(Ctl);
+
+__device__ __forceinline__ float gelu_tanh(float y) {
+  const float u = 0.7978845608028654f * (y + 0.044715f * y * y * y);
+  return 0.5f * y * (1.f + tanhf(u));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                      const __grid_constant__ CUtensorMap tmLR, const __grid_constant__ CUtensorMap tmL2,
+                      K2Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Ctl* ctl = reinterpret_cast<Ctl*>(base + STAGES * STAGE_BYTES);
+  volatile int* abort_flag = &ctl->abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    if (p.nl) {
+      tma_prefetch_desc(&tmLR);
+      tma_prefetch_desc(&tmL2);
+    }
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&ctl->full[s]), 1);
+      mbar_init(smem_u32(&ctl->empty[s]), 1);
+    }
+    mbar_init(smem_u32(&ctl->tfull), 1);
+    mbar_init(smem_u32(&ctl->tempty), 4);
+    ctl->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&ctl->tmem_base), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+
+  const int num_tiles = p.num_m_blocks * p.num_n_blocks;
+  const int kiters = p.nk + p.nl;
+  const size_t kb_per_row = (size_t)(p.K_pad / 64);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        const int mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
+        for (int it = 0; it < kiters; ++it) {
+          if (!mbar_wait(smem_u32(&ctl->empty[stage]), phase ^ 1, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          const uint32_t st = smem_u32(base + stage * STAGE_BYTES);
+          const uint32_t bar = smem_u32(&ctl->full[stage]);
+          if (it < p.nk) {
+            mbar_arrive_expect_tx(bar, STAGE_BYTES);
+            tma_load_2d(st, &tmA, it * 128, mb * BLOCK_M, bar);
+            tma_load_2d(st + A_BYTES, &tmB, it * 128, nb * BLOCK_N, bar);
+            bulk_load(st + A_BYTES + B_BYTES, p.sX + ((size_t)mb * kb_per_row + it * 4) * 512,
+                      SFA_BYTES, bar);
+            bulk_load(st + A_BYTES + B_BYTES + SFA_BYTES,
+                      p.sR + ((size_t)(2 * nb) * kb_per_row + it * 4) * 512, SFB_BYTES / 2, bar);
+            bulk_load(st + A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES / 2,
+                      p.sR + ((size_t)(2 * nb + 1) * kb_per_row + it * 4) * 512, SFB_BYTES / 2, bar);
+          } else {
+            const int c = it - p.nk;
+            mbar_arrive_expect_tx(bar, A_BYTES + B_BYTES);
+            tma_load_2d(st, &tmLR, c * 64, mb * BLOCK_M, bar);
+            tma_load_2d(st + A_BYTES, &tmL2, c * 64, nb * BLOCK_N, bar);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        if (!mbar_wait(smem_u32(&ctl->tempty), acc_phase ^ 1, abort_flag, p.err)) break;
+        tc_fence_after();
+        for (int it = 0; it < kiters; ++it) {
+          if (!mbar_wait(smem_u32(&ctl->full[stage]), phase, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a = smem_u32(base + stage * STAGE_BYTES);
+          const uint32_t b = a + A_BYTES;
+          if (it < p.nk) {
+            const uint32_t sfa = b + B_BYTES, sfb = sfa + SFA_BYTES;
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb) tmem_cp_sf_atom(tmem + SFA_COL + 4 * kb, sfa + kb * 512);
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb) {
+              tmem_cp_sf_atom(tmem + SFB_COL + 8 * kb, sfb + kb * 512);
+              tmem_cp_sf_atom(tmem + SFB_COL + 8 * kb + 4, sfb + SFB_BYTES / 2 + kb * 512);
+            }
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb)
+              mma_nvf4(tmem + ACC_COL, desc_k_sw128(a + 32 * kb), desc_k_sw128(b + 32 * kb), IDESC_F4,
+                       tmem + SFA_COL + 4 * kb, tmem + SFB_COL + 8 * kb, (it | kb) != 0);
+          } else {
+            const int c = it - p.nk;
+            const int steps = min(4, (p.r_tot - 64 * c) / 16);
+            for (int j = 0; j < steps; ++j)
+              mma_bf16(tmem + ACC_COL, desc_k_sw128(a + 32 * j), desc_k_sw128(b + 32 * j), IDESC_BF, 1);
+          }
+          tc_commit(smem_u32(&ctl->empty[stage]));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        tc_commit(smem_u32(&ctl->tfull));
+        acc_phase ^= 1;
+      }
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int sub = warp & 3;                 // TMEM lanes 32 sub .. 32 sub + 31
+    const int row = sub * 32 + lane;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const int mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
+      if (!mbar_wait(smem_u32(&ctl->tfull), acc_phase, abort_flag, p.err)) break;
+      tc_fence_after();
+      const int m = mb * BLOCK_M + row;
+      for (int c = 0; c < BLOCK_N / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem + ((uint32_t)(sub * 32) << 16) + ACC_COL + c * 32, r);
+        tmem_wait_ld();
+        const int n0 = nb * BLOCK_N + c * 32;
+        if (m < p.M) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int n = n0 + 8 * q;
+            if (n < p.N) {
+              const float4 b0 = __ldg(reinterpret_cast<const float4*>(p.bias + n));
+              const float4 b1 = __ldg(reinterpret_cast<const float4*>(p.bias + n + 4));
+              const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+              float y[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                y[e] = fmaf(p.alpha, __uint_as_float(r[8 * q + e]), bb[e]);
+                if (p.epi == 1) y[e] = gelu_tanh(y[e]);
+              }
+              uint4 o;
+              o.x = pack_bf16x2(y[0], y[1]);
+              o.y = pack_bf16x2(y[2], y[3]);
+              o.z = pack_bf16x2(y[4], y[5]);
+              o.w = pack_bf16x2(y[6], y[7]);
+              *reinterpret_cast<uint4*>(p.Y + (size_t)m * p.N + n) = o;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&ctl->tempty));
+      acc_phase ^= 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+cudaError_t launch_gemm_nvfp4(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmLR,
+                              const CUtensorMap& tmL2, K2Params p, int num_sms, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const int tiles = p.num_m_blocks * p.num_n_blocks;
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  gemm_nvfp4_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmLR, tmL2, p);
+  return cudaGetLastError();
+}
+
+}  // namespace svdq

@@ -1,0 +1,104 @@
+// kernels.h -- launch interfaces between the host API (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace svdq {
+
+// ---------------------------------------------------------------- kernel 1
+struct K1Params {
+  int M, K, K_pad, r_tot, r_pad;
+  int fmt;                 // 0 NVFP4, 1 INT4
+  int do_quant, do_lr;     // fused: both; unfused baseline: one of them
+  int stages;              // set by the launcher
+  const float* inv_lambda; // [K]
+  float s_t, six_st;       // NVFP4 activation tensor scale and fl32(6 s_t)
+  uint8_t* qX;             // [M][K_pad/2]
+  uint8_t* sX;             // scale layout (see svdq.h)
+  __nv_bfloat16* LR;       // [M][r_pad]
+  DeviceErr err;
+};
+cudaError_t launch_quant_down(const CUtensorMap& tmX, const CUtensorMap& tmL1, K1Params p,
+                              cudaStream_t stream);
+
+// ---------------------------------------------------------------- kernel 2
+struct K2Params {
+  int M, N, K_pad, r_tot, r_pad, N_pad;
+  int num_m_blocks, num_n_blocks;
+  int nk;                  // K_pad / 256 4-bit k-tiles
+  int nl;                  // r_pad / 64 low-rank k-tiles (0: plain W4A4 GEMM)
+  const uint8_t* sX;       // activation scales
+  const uint8_t* sR;       // weight scales
+  const float* bias;       // [N_pad]
+  float alpha;             // s_tX * s_tR
+  int epi;                 // 0 none, 1 GELU (tanh form)
+  __nv_bfloat16* Y;        // [M][N]
+  DeviceErr err;
+};
+cudaError_t launch_gemm_nvfp4(const CUtensorMap& tmA, const CUtensorMap& tmB,
+                              const CUtensorMap& tmLR, const CUtensorMap& tmL2, K2Params p,
+                              int num_sms, cudaStream_t stream);
+
+struct K2I8Params {
+  int M, N, K_pad, r_tot, r_pad, N_pad;
+  int num_m_blocks, num_n_blocks;
+  int nk;                  // K_pad / 128 int8 k-tiles (two 64-groups each)
+  int nl;
+  const __half* sX;        // [M_pad128][K_pad/64]
+  const __half* sR;        // [N_pad][K_pad/64]
+  const float* bias;
+  int epi;
+  __nv_bfloat16* Y;
+  DeviceErr err;
+};
+cudaError_t launch_gemm_int4(const uint8_t* qX, const uint8_t* qR, const CUtensorMap& tmLR,
+                             const CUtensorMap& tmL2, K2I8Params p, int num_sms,
+                             cudaStream_t stream);
+
+// ---------------------------------------------------------------- unfused up projection
+struct UpParams {
+  int M, N, r_tot, r_pad;
+  const __nv_bfloat16* LR;   // [M][r_pad]
+  const __nv_bfloat16* L2a;  // [N_pad][r_pad]
+  float alpha;
+  int epi;
+  __nv_bfloat16* Y;          // [M][N], read-modify-write
+};
+cudaError_t launch_lowrank_up(UpParams p, cudaStream_t stream);
+
+// ---------------------------------------------------------------- preparation / calibration
+cudaError_t launch_calibrate(int M, int K, int N, const __nv_bfloat16* X, const __nv_bfloat16* Wt,
+                             float alpha, float* lambda_out, float* act_scale_out, unsigned* ws,
+                             cudaStream_t stream);
+
+struct PrepParams {
+  int fmt, K, N, K_pad, N_pad, rank, lora_rank, r_tot, r_pad;
+  const __nv_bfloat16* Wt;     // [N][K]
+  const float* lambda;         // [K]
+  const __nv_bfloat16* L1f;    // [K][rank]
+  const __nv_bfloat16* L2;     // [rank][N]
+  const __nv_bfloat16* bias;   // [N] or null
+  const __nv_bfloat16* loraA;  // [K][lora_rank] or null
+  const __nv_bfloat16* loraB;  // [lora_rank][N] or null
+  float* R;                    // scratch [N][K]
+  unsigned* amax_bits;         // scratch, 1 word
+  uint8_t* qR;                 // [N_pad][K_pad/2]
+  uint8_t* sR;                 // scales
+  __nv_bfloat16* L1t;          // [r_tot][K]
+  __nv_bfloat16* L2a;          // [N_pad][r_pad]
+  float* bias_f;               // [N_pad]
+  float* lambda_inv;           // [K]
+};
+cudaError_t launch_prepare_residual(const PrepParams& p, cudaStream_t stream);
+cudaError_t launch_prepare_quantize(const PrepParams& p, float s_tR, float alpha,
+                                    cudaStream_t stream);
+
+cudaError_t launch_selftest_timeout(DeviceErr err, cudaStream_t stream);
+
+}  // namespace svdq

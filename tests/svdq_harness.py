@@ -1,0 +1,191 @@
+"""Test-side harness: runs the CUDA path through the C ABI and maps its
+library-defined layouts back to the oracle's canonical arrays.
+
+The index functions here are written from the layout description in
+include/svdq.h (the tcgen05 scale-factor atom: 512 bytes per 128 rows x 4
+groups, byte (r % 32) * 16 + ((r % 128) / 32) * 4 + g), independently of
+the CUDA sources.  Inputs always come from workloads.py and the oracle;
+nothing computed by the GPU is ever fed back into the oracle.
+"""
+from __future__ import annotations
+
+import os
+
+import numpy as np
+import torch
+
+from oracle import formats as F
+from oracle import svdquant as S
+
+
+def rup(x, m):
+    return (x + m - 1) // m * m
+
+
+# ------------------------------------------------------------------ layout decoders
+def sf_atoms_to_canonical(raw: np.ndarray, rows: int, K: int, K_pad: int) -> np.ndarray:
+    """E4M3 scale atoms -> (rows, K/16) uint8."""
+    r = np.arange(rows)[:, None]
+    g = np.arange(K // 16)[None, :]
+    off = ((r // 128) * (K_pad // 64) + g // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + g % 4
+    return raw.reshape(-1)[off]
+
+
+def unpack_codes(raw: np.ndarray, rows: int, K: int, K_pad: int, fmt: str) -> np.ndarray:
+    b = raw.reshape(-1)[: rows * (K_pad // 2)].reshape(rows, K_pad // 2)
+    c = F.unpack_nibbles(b)[:, :K]
+    return c if fmt == "nvfp4" else F.int4_from_nibble(c)
+
+
+def int4_scales(raw: np.ndarray, rows: int, K: int, K_pad: int) -> np.ndarray:
+    h = raw.reshape(-1).view(np.float16)
+    return h[: rows * (K_pad // 64)].reshape(rows, K_pad // 64)[:, : K // 64]
+
+
+def to_np(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().numpy()
+
+
+def bf16_np(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def dev_bf16(a) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(np.asarray(a, np.float32))).to(torch.bfloat16).cuda()
+
+
+def dev_f32(a) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(np.asarray(a, np.float32))).cuda()
+
+
+_cudart = None
+
+
+def _libcudart():
+    """The CUDA runtime library torch already loaded in this process."""
+    global _cudart
+    if _cudart is None:
+        import ctypes
+        torch.cuda.init()
+        path = None
+        with open("/proc/self/maps") as f:
+            for line in f:
+                if "libcudart.so" in line:
+                    path = line.split()[-1]
+                    break
+        if path is None:
+            import nvidia.cuda_runtime as cr
+            path = os.path.join(os.path.dirname(cr.__file__), "lib", "libcudart.so.12")
+        _cudart = ctypes.CDLL(path)
+        _cudart.cudaMemcpy.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int]
+        _cudart.cudaMemcpy.restype = ctypes.c_int
+    return _cudart
+
+
+def read_device(ptr: int, nbytes: int) -> np.ndarray:
+    """Copy nbytes at a device address owned by the library into numpy."""
+    out = np.empty(nbytes, np.uint8)
+    torch.cuda.synchronize()
+    rc = _libcudart().cudaMemcpy(out.ctypes.data, ptr, nbytes, 2)   # device -> host
+    assert rc == 0, rc
+    return out
+
+
+# ------------------------------------------------------------------ tolerance
+def y_check(Y_gpu: np.ndarray, Y_o: np.ndarray, rel: float = 1e-2):
+    """max|dY| <= rel * rms(Y_o); an element above that must still be within
+    one bf16 ulp of Y_o (both sides round to bf16 at a tie boundary)."""
+    rms = float(np.sqrt(np.mean(Y_o ** 2)))
+    diff = np.abs(Y_gpu - Y_o)
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(Y_o), 1e-30))) - 7)
+    bad = (diff > rel * rms) & (diff > ulp * (1 + 1e-9))
+    return dict(max_abs=float(diff.max()), rms=rms, max_rel_rms=float(diff.max() / rms),
+                n_over=int(np.sum(diff > rel * rms)), n_bad=int(bad.sum()))
+
+
+def assert_y(Y_gpu, Y_o, rel=1e-2):
+    r = y_check(Y_gpu, Y_o, rel)
+    assert r["n_bad"] == 0, r
+    return r
+
+
+# ------------------------------------------------------------------ the layer on the GPU
+class GpuLayer:
+    """Prepared weights on the GPU plus the oracle's view of the same layer."""
+
+    def __init__(self, fmt, X_cal, W, bias, rank, lora_A=None, lora_B=None, factors=None, act=None):
+        from rank_gemm_b200 import binding as B
+        self.B = B
+        self.fmt = fmt
+        W = np.asarray(W, np.float32)
+        self.K, self.N = W.shape
+        if factors is None:
+            lam = S.smoothing_factors(X_cal, W)
+            L1f, L2, _ = S.svd_factors(W, lam, rank)
+        else:
+            lam, L1f, L2 = factors
+        if act is None:
+            act = S.act_tensor_scale(X_cal, S.inverse_lambda(lam)) if fmt == "nvfp4" else np.float32(1.0)
+        self.pw = S.prepare(fmt, W, lam, L1f, L2, bias, act, lora_A, lora_B)
+        self.rank = L1f.shape[1]
+        self.lora_rank = 0 if lora_A is None else lora_A.shape[1]
+        self.r_tot = self.rank + self.lora_rank
+        self.lam, self.act = lam, act
+        self.d_W = dev_bf16(W.T)
+        self.d_lam = dev_f32(lam)
+        self.d_L1f = dev_bf16(L1f)
+        self.d_L2 = dev_bf16(L2)
+        self.d_bias = dev_bf16(bias)
+        self.d_A = dev_bf16(lora_A) if lora_A is not None else None
+        self.d_B = dev_bf16(lora_B) if lora_B is not None else None
+        self.h = B.svdq_prepare_weights(fmt, self.K, self.N, self.rank, self.d_W, self.d_lam, self.d_L1f,
+                                        self.d_L2, self.d_bias, self.d_A, self.d_B, self.lora_rank, float(act))
+        self.info = B.svdq_weights_view(self.h)
+
+    def close(self):
+        if self.h:
+            self.B.svdq_free_weights(self.h)
+            self.h = None
+
+    # -------------------------------------------------------------- weight-side outputs
+    def weight_codes(self):
+        i = self.info
+        qraw = read_device(i.qR, i.N_pad * i.K_pad // 2)
+        qR = unpack_codes(qraw, self.N, self.K, i.K_pad, self.fmt)
+        if self.fmt == "nvfp4":
+            sraw = read_device(i.sR, i.N_pad * i.K_pad // 16)
+            sR = sf_atoms_to_canonical(sraw, self.N, self.K, i.K_pad)
+        else:
+            sraw = read_device(i.sR, i.N_pad * (i.K_pad // 64) * 2)
+            sR = int4_scales(sraw, self.N, self.K, i.K_pad)
+        return qR, sR, np.float32(i.s_tR)
+
+    # -------------------------------------------------------------- activation-side
+    def buffers(self, M):
+        qb, sb, lb = self.B.svdq_act_buffer_sizes(self.h, M)
+        f = lambda n: torch.empty(max(n, 16), dtype=torch.uint8, device="cuda").fill_(0xA5)
+        return f(qb), f(sb), f(lb)
+
+    def kernel1(self, Xd, M):
+        qX, sX, LR = self.buffers(M)
+        self.B.svdq_quantize_act_lowrank_down(self.h, M, Xd, qX, sX, LR)
+        torch.cuda.synchronize()
+        return qX, sX, LR
+
+    def decode_act(self, qX, sX, LR, M):
+        i = self.info
+        q = unpack_codes(to_np(qX), M, self.K, i.K_pad, self.fmt)
+        if self.fmt == "nvfp4":
+            s = sf_atoms_to_canonical(to_np(sX), M, self.K, i.K_pad)
+        else:
+            s = int4_scales(to_np(sX), M, self.K, i.K_pad)
+        lr = to_np(LR)[: M * i.r_pad * 2].view(np.uint16).reshape(M, i.r_pad)
+        return q, s, F.bf16_from_bits(lr[:, : self.r_tot]), F.bf16_from_bits(lr[:, self.r_tot:])
+
+    def linear(self, Xd, M, gelu=False, unfused=False):
+        Y = torch.empty(M, self.N, dtype=torch.bfloat16, device="cuda")
+        ws = torch.empty(max(self.B.svdq_linear_workspace_bytes(self.h, M), 16), dtype=torch.uint8, device="cuda")
+        epi = self.B.SVDQ_EPI_GELU_TANH if gelu else self.B.SVDQ_EPI_NONE
+        (self.B.svdq_linear_unfused if unfused else self.B.svdq_linear)(self.h, M, Xd, epi, Y, ws)
+        torch.cuda.synchronize()
+        return Y
