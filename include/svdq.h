@@ -96,7 +96,7 @@ typedef struct {
   const float* lambda_inv; /* dev float32 [K]: correctly rounded 1/lambda */
   float s_tR;              /* NVFP4 weight tensor scale (1 for INT4) */
   float s_tX;              /* NVFP4 static activation tensor scale (1 for INT4) */
-  float alpha;             /* s_tX * s_tR in float32 */
+  float alpha;             /* 2^k = s_tX * s_tR up to one float32 rounding (1 for INT4) */
 } svdq_weights_info;
 
 /* ------------------------------------------------------------------------
@@ -131,7 +131,10 @@ svdq_status svdq_calibrate(int M, int K, int N, const void* X, const void* W_t, 
  * W^ = diag(lambda) W, computes on the device
  *     R[k,n] = fp32(lambda_k W[k,n] - lambda_k sum_{i<rank} L1f[k,i] L2[i,n])
  * (float64, i ascending, no fused multiply-add), the NVFP4 tensor scale
- * s_tR = max|R| / 2688, the 4-bit codes and block scales of R per output
+ * s_tR = fl32(2^k / act_scale) with k the smallest integer such that
+ * 2^k >= act_scale max|R| / 2688 (so s_tR >= max|R| / 2688 and the product
+ * alpha = act_scale s_tR is the power of two 2^k, which lets L2 / alpha be
+ * stored exactly in bf16), the 4-bit codes and block scales of R per output
  * column (groups of 16 along K for NVFP4, 64 for INT4), and the layouts the
  * kernels consume.  A LoRA (A: K x lora_rank, B: lora_rank x N) is appended
  * to the factors: L1' = [L1f | A], L2' = [L2 ; B]; R does not change.

@@ -33,8 +33,12 @@ Readings where the pages are silent (each one is a choice of this build):
     The rounded factors are used, so low-rank + residual rebuild W^.
   * Groups run along K (the contraction), per activation row and per weight
     output column.
-  * NVFP4: tensor scale s_t = fp32(amax / 2688) (2688 = 6 * 448), 1 if the
-    amax is 0.  Per block of 16: a = max|v|, sb = E4M3(a / fp32(6 s_t)),
+  * NVFP4 tensor scales: the activation's s_tX is a static calibration,
+    fp32(amax(|X^|) / 2688) (2688 = 6 * 448; 1 if the amax is 0); the
+    residual's is s_tR = fl32(2^k / s_tX) with k the smallest integer such
+    that 2^k >= s_tX amax(|R|) / 2688, so s_tR >= amax(|R|) / 2688 and
+    s_tX s_tR is a power of two (see weight_tensor_scale).
+    Per block of 16: a = max|v|, sb = E4M3(a / fp32(6 s_t)),
     d = fp32(f32(sb) s_t), inv = fp32(1/d) (0 if d = 0),
     code = E2M1(fp32(v inv)).  The activation tensor scale is static (an
     offline calibration: amax of X^ / 2688).
@@ -141,6 +145,22 @@ def tensor_scale(V) -> np.float32:
     return np.float32(1.0) if a == 0 else np.float32(a / NVFP4_TENSOR_DIVISOR)
 
 
+def weight_tensor_scale(R, s_tX):
+    """NVFP4 tensor scale of the residual, paired with the activation's.
+
+    k is the smallest integer with 2^k >= s_tX amax(|R|) / 2688 (float64;
+    amax 0 counts as 2688), and s_tR = fl32(2^k / s_tX).  Then s_tR is at
+    least amax / 2688 up to one float32 rounding, so no block scale needs
+    more than E4M3's 448, and the product alpha = s_tX s_tR that the 4-bit
+    product is multiplied by is 2^k up to that rounding: the 16-bit branch
+    can carry 1/alpha exactly.  Returns (s_tR, k)."""
+    a = float(np.max(np.abs(np.asarray(R, np.float32)))) if np.size(R) else 0.0
+    x = (a if a > 0 else 2688.0) * float(np.float32(s_tX)) / 2688.0
+    m, e = np.frexp(x)
+    k = int(e - 1) if m == 0.5 else int(e)
+    return np.float32(np.float32(np.ldexp(1.0, k)) / np.float32(s_tX)), k
+
+
 # ============================================================ 4-bit group quantization
 def quantize_nvfp4(V, s_t):
     """Rows of V (rows, K) in groups of 16 along K.
@@ -224,6 +244,7 @@ class PreparedWeights:
     s_tX: np.float32         # NVFP4 static activation tensor scale (1 for INT4)
     bias: np.ndarray         # (N,) bf16 values
     sigma: Optional[np.ndarray] = None
+    alpha_log2: int = 0      # log2 of the power of two that s_tX s_tR rounds to
 
 
 def prepare(fmt: str, W, lam, L1f, L2, bias, act_scale=None, lora_A=None, lora_B=None,
@@ -236,12 +257,13 @@ def prepare(fmt: str, W, lam, L1f, L2, bias, act_scale=None, lora_A=None, lora_B
     lam = np.asarray(lam, np.float32)
     R = residual(W, lam, L1f, L2)
     if fmt == "nvfp4":
-        s_tR = tensor_scale(R)
-        qR, sR = quantize_nvfp4(R.T.copy(), s_tR)
         s_tX = np.float32(act_scale)
+        s_tR, alpha_log2 = weight_tensor_scale(R, s_tX)
+        qR, sR = quantize_nvfp4(R.T.copy(), s_tR)
     elif fmt == "int4":
         s_tR = np.float32(1.0)
         s_tX = np.float32(1.0)
+        alpha_log2 = 0
         qR, sR = quantize_int4(R.T.copy())
     else:
         raise ValueError(fmt)
@@ -252,7 +274,8 @@ def prepare(fmt: str, W, lam, L1f, L2, bias, act_scale=None, lora_A=None, lora_B
         L2_all = np.concatenate([L2_all, np.asarray(lora_B, np.float64)], axis=0)
     return PreparedWeights(fmt=fmt, K=K, N=N, rank=np.asarray(L1f).shape[1], lam=lam,
                            inv_lam=inverse_lambda(lam), L1f=L1f_all, L2=L2_all, R=R, qR=qR, sR=sR,
-                           s_tR=s_tR, s_tX=s_tX, bias=np.asarray(bias, np.float64), sigma=sigma)
+                           s_tR=s_tR, s_tX=s_tX, bias=np.asarray(bias, np.float64), sigma=sigma,
+                           alpha_log2=alpha_log2)
 
 
 def quantize_activation(pw: PreparedWeights, X):

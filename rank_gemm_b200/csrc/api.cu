@@ -368,13 +368,21 @@ svdq_status svdq_prepare_weights(svdq_format fmt, int K, int N, int rank, const 
     float a;
     std::memcpy(&a, &amax_host, 4);
     if (fmt == SVDQ_NVFP4) {
-      w->s_tR = (a == 0.f) ? 1.f : a / 2688.0f;
+      // k: the smallest integer with 2^k >= s_tX amax(|R|) / 2688; then
+      // s_tR = fl32(2^k / s_tX), so alpha = s_tX s_tR is the power of two 2^k
+      // (to one float32 rounding) and L2 / alpha below is exact in bf16.
+      const double x = (a > 0.f ? (double)a : 2688.0) * (double)act_scale / 2688.0;
+      int e = 0;
+      const double m = std::frexp(x, &e);
+      const int k = (m == 0.5) ? e - 1 : e;
       w->s_tX = act_scale;
+      w->s_tR = std::ldexp(1.0f, k) / act_scale;
+      w->alpha = std::ldexp(1.0f, k);
     } else {
       w->s_tR = 1.f;
       w->s_tX = 1.f;
+      w->alpha = 1.f;
     }
-    w->alpha = w->s_tX * w->s_tR;
     e = launch_prepare_quantize(p, w->s_tR, w->alpha, stream);
   }
   if (e == cudaSuccess) e = cudaStreamSynchronize(stream);

@@ -63,8 +63,13 @@ def _brute_layer(fmt, X, W, bias, lam, L1f, L2, act_scale, gelu=False):
             R[n][k] = f32(float(lam[k]) * float(W[k, n]) - float(lam[k]) * s)
     if fmt == "nvfp4":
         amax = max(abs(R[n][k]) for n in range(N) for k in range(K))
-        s_tR = f32(1.0) if amax == 0 else f32(f32(amax) / f32(2688.0))
         s_tX = f32(act_scale)
+        # smallest power of two 2^k >= s_tX amax / 2688, then s_tR = 2^k / s_tX
+        target = (float(amax) if amax > 0 else 2688.0) * float(s_tX) / 2688.0
+        k = -200
+        while 2.0 ** k < target:
+            k += 1
+        s_tR = f32(f32(2.0 ** k) / s_tX)
     else:
         s_tR = s_tX = f32(1.0)
 

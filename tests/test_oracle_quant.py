@@ -101,3 +101,20 @@ def test_int4_error_bound_every_element():
 def test_int4_zero_block():
     q, s = S.quantize_int4(np.zeros((2, 128), np.float32))
     assert np.all(q == 0) and np.all(s == 0)
+
+
+def test_weight_tensor_scale_pairs_to_a_power_of_two():
+    rng = np.random.default_rng(12)
+    for trial in range(200):
+        R = (rng.standard_normal((8, 64)) * np.exp(rng.uniform(-12, 6))).astype(np.float32)
+        s_tX = np.float32(np.exp(rng.uniform(-12, 2)))
+        s_tR, k = S.weight_tensor_scale(R, s_tX)
+        amax = float(np.max(np.abs(R)))
+        # 2^k is the smallest power of two >= s_tX amax / 2688
+        assert 2.0 ** k >= s_tX * amax / 2688 and 2.0 ** (k - 1) < s_tX * amax / 2688
+        # s_tX s_tR = 2^k within one float32 rounding
+        assert abs(float(s_tX) * float(s_tR) / 2.0 ** k - 1) <= 2.0 ** -24
+        # no block scale beyond E4M3's range is needed, and the largest is at least 224
+        _, sc = S.quantize_nvfp4(R, s_tR)
+        top = F.e4m3_decode(sc).max()
+        assert 224 <= top <= 448
