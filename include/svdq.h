@@ -48,8 +48,10 @@
  *         is 512 contiguous bytes at ((i * K_pad/64) + j) * 512; inside it
  *         the scale of row r and 16-group g (0..3) sits at byte
  *         (r % 32) * 16 + ((r % 128) / 32) * 4 + g.  Rows >= M hold 0.
- *         INT4: binary16 block scales (one per 64 k), row-major
- *         [M_pad128][K_pad/64]; rows >= M and columns >= K/64 hold 0.
+ *         INT4: binary16 block scales (one per 64 k) in 512-byte chunks of
+ *         128 rows x 2 groups: the scale of row r and 64-group g sits at
+ *         element (((r / 128) * (K_pad/128) + g / 2) * 2 + g % 2) * 128 + r % 128;
+ *         rows >= M and groups >= K/64 hold 0.
  *   LR    bf16 [M][r_pad]: X L1f for the r_tot low-rank columns, zeros after.
  */
 #ifndef SVDQ_H_
@@ -89,7 +91,7 @@ typedef struct {
   int K, N, rank, lora_rank, r_tot;
   int K_pad, N_pad, r_pad; /* N_pad = N rounded up to a multiple of 256 */
   const void* qR;          /* dev uint8 [N_pad][K_pad/2], packed like qX (rows = output features) */
-  const void* sR;          /* dev: NVFP4 E4M3 atoms like sX over N_pad rows; INT4 binary16 [N_pad][K_pad/64] */
+  const void* sR;          /* dev: scales of R laid out like sX, over N_pad rows */
   const void* L1t;         /* dev bf16 [r_tot][K]: (lambda^-1-folded L1 | LoRA A), transposed */
   const void* L2a;         /* dev bf16 [N_pad][r_pad]: (L2 ; LoRA B) transposed, divided by alpha */
   const void* bias;        /* dev float32 [N_pad] (zeros if no bias was given) */

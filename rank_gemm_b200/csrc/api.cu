@@ -34,6 +34,7 @@ struct svdq_weights {
   float* lambda_inv;
   float s_tR, s_tX, alpha;
   CUtensorMap tm_qR, tm_L2a, tm_L1t;
+  CUtensorMap tm_qR_i4, tm_L2a_i4;   // INT4 kernel: packed 64-byte rows / 32-column low-rank chunks
 };
 
 namespace {
@@ -116,16 +117,17 @@ svdq_status current_device(DevState** out) {
 
 DeviceErr dev_err(const DevState* d) { return DeviceErr{d->err_word, wait_limit_ns()}; }
 
-// 2-D tensor map, row-major [rows][inner] with a 128-byte-swizzled box.
+// 2-D tensor map, row-major [rows][inner]; boxes land in shared memory with
+// the given swizzle (128-byte by default).
 bool tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t inner, uint64_t rows,
-             uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows) {
+             uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows,
+             CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   cuuint64_t dims[2] = {inner, rows};
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t es[2] = {1, 1};
-  return g_encode(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return g_encode(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 size_t qx_bytes(const svdq_weights* w, int M) { return (size_t)M * (w->K_pad / 2); }
@@ -183,10 +185,11 @@ svdq_status run_k2(const svdq_weights* w, int M, const void* qX, const void* sX,
   if (s != SVDQ_OK) return s;
   CUtensorMap tmLR;
   std::memset(&tmLR, 0, sizeof(tmLR));
-  if (lowrank &&
-      !tmap_2d(&tmLR, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, LR, w->r_pad, M, (uint64_t)w->r_pad * 2, 64, 128))
+  const bool nv = w->fmt == SVDQ_NVFP4;
+  if (lowrank && !tmap_2d(&tmLR, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, LR, w->r_pad, M, (uint64_t)w->r_pad * 2,
+                          nv ? 64 : 32, 128, nv ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
     return SVDQ_ERR_CUDA;
-  if (w->fmt == SVDQ_NVFP4) {
+  if (nv) {
     CUtensorMap tmA;
     if (!tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, qX, w->K_pad / 2, M, w->K_pad / 2, 128, 128))
       return SVDQ_ERR_CUDA;
@@ -210,6 +213,10 @@ svdq_status run_k2(const svdq_weights* w, int M, const void* qX, const void* sX,
     p.err = dev_err(d);
     return from_cuda(launch_gemm_nvfp4(tmA, w->tm_qR, tmLR, w->tm_L2a, p, d->num_sms, stream));
   }
+  CUtensorMap tmXp;
+  if (!tmap_2d(&tmXp, CU_TENSOR_MAP_DATA_TYPE_UINT8, qX, w->K_pad / 2, M, w->K_pad / 2, 64, 128,
+               CU_TENSOR_MAP_SWIZZLE_NONE))
+    return SVDQ_ERR_CUDA;
   K2I8Params p;
   p.M = M;
   p.N = w->N;
@@ -220,15 +227,14 @@ svdq_status run_k2(const svdq_weights* w, int M, const void* qX, const void* sX,
   p.num_m_blocks = (M + 127) / 128;
   p.num_n_blocks = w->N_pad / 256;
   p.nk = w->K_pad / 128;
-  p.nl = lowrank ? w->r_pad / 64 : 0;
+  p.nl = lowrank ? (w->r_tot + 31) / 32 : 0;
   p.sX = static_cast<const __half*>(sX);
   p.sR = reinterpret_cast<const __half*>(w->sR);
   p.bias = w->bias_f;
   p.epi = (int)epi;
   p.Y = static_cast<__nv_bfloat16*>(Y);
   p.err = dev_err(d);
-  return from_cuda(launch_gemm_int4(static_cast<const uint8_t*>(qX), w->qR, tmLR, w->tm_L2a, p, d->num_sms,
-                                    stream));
+  return from_cuda(launch_gemm_int4(tmXp, w->tm_qR_i4, tmLR, w->tm_L2a_i4, p, d->num_sms, stream));
 }
 
 void free_buffers(svdq_weights* w) {
@@ -394,7 +400,11 @@ svdq_status svdq_prepare_weights(svdq_format fmt, int K, int N, int rank, const 
               tmap_2d(&w->tm_L2a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->L2a, w->r_pad, w->N_pad,
                       (uint64_t)w->r_pad * 2, 64, 256) &&
               tmap_2d(&w->tm_L1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->L1t, K, r_tot, (uint64_t)K * 2, 64,
-                      r_tot);
+                      r_tot) &&
+              tmap_2d(&w->tm_qR_i4, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->qR, w->K_pad / 2, w->N_pad, w->K_pad / 2,
+                      64, 128, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+              tmap_2d(&w->tm_L2a_i4, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->L2a, w->r_pad, w->N_pad,
+                      (uint64_t)w->r_pad * 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B);
   if (!maps) {
     free_buffers(w);
     delete w;

@@ -319,6 +319,13 @@ __host__ __device__ __forceinline__ size_t sf_atom_offset(int row, int g16, int 
          (g16 & 3);
 }
 
+// Element offset of (row, 64-group) in the INT4 binary16 scale layout:
+// 512-byte chunks of 128 rows x 2 groups (one 128-wide k-tile), ordered
+// (row block, k-tile), group-major inside a chunk.
+__host__ __device__ __forceinline__ size_t int4_scale_offset(int row, int g64, int kpad) {
+  return (((size_t)(row >> 7) * (kpad >> 7) + (g64 >> 1)) * 2 + (g64 & 1)) * 128 + (row & 127);
+}
+
 __host__ __device__ constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
 }  // namespace svdq

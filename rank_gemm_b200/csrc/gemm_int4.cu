@@ -1,12 +1,396 @@
-// gemm_int4.cu -- kernel 2 for INT4 (placeholder until the int8 tensor-core path lands).
+// gemm_int4.cu -- kernel 2 for INT4: the 4-bit GEMM fused with the low-rank up
+// projection ("Nunchaku engine design" figure (b), "svdq-int4-flux.1-dev" model
+// card), on the int8 tensor-core path.
+//
+// INT4 block scales are binary16 per 64 elements, which no block-scaled MMA
+// kind can take, so each 64-group is its own integer product:
+//     y[m,n] = sum_g sX[m,g] sR[n,g] (sum_{k in g} qX[m,k] qR[n,k]) + LR[m,:] L2[n,:] + b[n]
+// The int4 codes are unpacked to int8 in shared memory, every group runs as
+// two tcgen05.mma.kind::i8 (K = 32) into a fresh int32 TMEM tile, and CUDA
+// cores apply sX sR and accumulate in fp32 registers.  That per-group rescale
+// (about three ALU operations per output element per group) bounds this kernel,
+// not the int8 tensor core.
+//
+// One 128 x 128 output tile per CTA at a time, persistent over tiles:
+//   warp 0       TMA producer: packed int4 tiles of qX and qR (128 rows x 64 B
+//                per 128-wide k-tile) into a staging ring, then the low-rank
+//                chunks (LR and L2, 32 columns, 64-byte swizzle).
+//   warps 1-4    unpack: staging int4 -> int8 operand tiles (128-byte swizzle)
+//                in the MMA ring.
+//   warp 5       TMEM owner and MMA issuer (kind::i8 per group into one of two
+//                TMEM buffers; the low-rank chunks as kind::f16 straight from
+//                the staging ring into one more buffer use).
+//   warps 6-13   rescale + epilogue: 2 warps per TMEM sub-partition, 64 columns
+//                each; fp32 accumulators in registers; bias, GELU, bf16 store.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace svdq {
 
-cudaError_t launch_gemm_int4(const uint8_t*, const uint8_t*, const CUtensorMap&, const CUtensorMap&, K2I8Params,
-                             int, cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace {
+
+constexpr int BM = 128, BN = 128;
+constexpr int ST = 6;                    // staging ring (packed int4 / low-rank chunks)
+constexpr int MS = 3;                    // MMA ring (unpacked int8 tiles)
+constexpr int STG_HALF = 8192;           // packed [128 x 64 B] or bf16 [128 x 32]
+constexpr int STG_BYTES = 2 * STG_HALF;
+constexpr int OP_BYTES = 16384;          // int8 [128 x 128 B]
+constexpr int MMA_BYTES = 2 * OP_BYTES;
+constexpr int WARPS = 14, THREADS = WARPS * 32;
+constexpr int W_UNPACK = 1, W_MMA = 5, W_RESCALE = 6;
+constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t IDESC_I8 = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                              ((uint32_t)(BM >> 4) << 24);
+constexpr uint32_t IDESC_BF = idesc_bf16_f32(BM, BN);
+
+struct Ctl {
+  uint64_t sfull[ST], sempty[ST], mfull[MS], mempty[MS], dfull[2], dempty[2];
+  uint32_t unpack_done[ST];
+  uint32_t tmem_base;
+  int abort;
+};
+constexpr size_t SMEM_BYTES = (size_t)ST * STG_BYTES + (size_t)MS * MMA_BYTES + 1024 + sizeof(Ctl);
+
+__device__ __forceinline__ void mma_i8(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+// K-major bf16 tile with 64-byte rows in the 64-byte swizzle (8-row groups 512 B apart).
+__device__ __forceinline__ uint64_t desc_k_sw64(uint32_t addr) { return smem_desc(addr, 16, 512, 4); }
+
+// Sign-extends the four 4-bit values held in the low nibbles of the bytes of x.
+__device__ __forceinline__ uint32_t sext4x4(uint32_t x) {
+  return ((x ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
+}
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+// 16 packed bytes (32 int4, element 2j in the low nibble of byte j) -> 32 int8.
+__device__ __forceinline__ void unpack32(const uint4 p, uint4& o0, uint4& o1) {
+  const uint32_t w[4] = {p.x, p.y, p.z, p.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t lo = sext4x4(w[i] & 0x0F0F0F0Fu), hi = sext4x4((w[i] >> 4) & 0x0F0F0F0Fu);
+    o[2 * i] = prmt(lo, hi, 0x5140u);
+    o[2 * i + 1] = prmt(lo, hi, 0x7362u);
+  }
+  o0 = make_uint4(o[0], o[1], o[2], o[3]);
+  o1 = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+__device__ __forceinline__ float gelu_tanh(float y) {
+  const float u = 0.7978845608028654f * (y + 0.044715f * y * y * y);
+  return 0.5f * y * (1.f + tanhf(u));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_int4_kernel(const __grid_constant__ CUtensorMap tmXp, const __grid_constant__ CUtensorMap tmRp,
+                     const __grid_constant__ CUtensorMap tmLR, const __grid_constant__ CUtensorMap tmL2,
+                     K2I8Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stg = base;                              // ST x 16 KB
+  uint8_t* mring = base + ST * STG_BYTES;           // MS x 32 KB
+  Ctl* ctl = reinterpret_cast<Ctl*>(mring + MS * MMA_BYTES);
+  volatile int* abort_flag = &ctl->abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tmXp);
+    tma_prefetch_desc(&tmRp);
+    if (p.nl) {
+      tma_prefetch_desc(&tmLR);
+      tma_prefetch_desc(&tmL2);
+    }
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(smem_u32(&ctl->sfull[s]), 1);
+      mbar_init(smem_u32(&ctl->sempty[s]), 1);
+      ctl->unpack_done[s] = 0;
+    }
+    for (int s = 0; s < MS; ++s) {
+      mbar_init(smem_u32(&ctl->mfull[s]), 4);
+      mbar_init(smem_u32(&ctl->mempty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&ctl->dfull[b]), 1);
+      mbar_init(smem_u32(&ctl->dempty[b]), 8);
+    }
+    ctl->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == W_MMA) {
+    tmem_alloc(smem_u32(&ctl->tmem_base), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+
+  const int num_tiles = p.num_m_blocks * p.num_n_blocks;
+  const int nk = p.nk, nl = p.nl;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // -------------------------------------------------------------- producer
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        const int mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
+        for (int it = 0; it < nk + nl; ++it) {
+          if (!mbar_wait(smem_u32(&ctl->sempty[s]), ph ^ 1, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          const uint32_t dst = smem_u32(stg + s * STG_BYTES), bar = smem_u32(&ctl->sfull[s]);
+          mbar_arrive_expect_tx(bar, STG_BYTES);
+          if (it < nk) {
+            tma_load_2d(dst, &tmXp, it * 64, mb * BM, bar);
+            tma_load_2d(dst + STG_HALF, &tmRp, it * 64, nb * BN, bar);
+          } else {
+            tma_load_2d(dst, &tmLR, (it - nk) * 32, mb * BM, bar);
+            tma_load_2d(dst + STG_HALF, &tmL2, (it - nk) * 32, nb * BN, bar);
+          }
+          if (++s == ST) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+      }
+    }
+  } else if (warp >= W_UNPACK && warp < W_MMA) {
+    // ---------------------------------------------------------------- unpack
+    const int ut = threadIdx.x - W_UNPACK * 32;      // 0..127
+    int s = 0, t = 0;
+    uint32_t sph = 0, mph = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+      for (int it = 0; it < nk + nl; ++it) {
+        if (it < nk) {
+          if (!mbar_wait(smem_u32(&ctl->sfull[s]), sph, abort_flag, p.err) ||
+              !mbar_wait(smem_u32(&ctl->mempty[t]), mph ^ 1, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          const uint8_t* src = stg + s * STG_BYTES;
+          uint8_t* dst = mring + t * MMA_BYTES;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {           // h = 0: A (activations), 1: B (weights)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int u = ut + 128 * j, row = u >> 2, c16 = u & 3;
+              const uint4 pk = *reinterpret_cast<const uint4*>(src + h * STG_HALF + row * 64 + c16 * 16);
+              uint4 o0, o1;
+              unpack32(pk, o0, o1);
+              uint8_t* rbase = dst + h * OP_BYTES + row * 128;
+              *reinterpret_cast<uint4*>(rbase + (((2 * c16) ^ (row & 7)) << 4)) = o0;
+              *reinterpret_cast<uint4*>(rbase + (((2 * c16 + 1) ^ (row & 7)) << 4)) = o1;
+            }
+          }
+          fence_proxy_async_smem();                // generic-proxy writes -> tensor core
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(smem_u32(&ctl->mfull[t]));
+            // the last of the four unpack warps to finish releases the staging slot
+            if (atomicAdd(&ctl->unpack_done[s], 1u) == 3u) {
+              ctl->unpack_done[s] = 0;
+              mbar_arrive(smem_u32(&ctl->sempty[s]));
+            }
+          }
+          if (++t == MS) {
+            t = 0;
+            mph ^= 1;
+          }
+        }
+        if (++s == ST) {
+          s = 0;
+          sph ^= 1;
+        }
+      }
+    }
+  } else if (warp == W_MMA) {
+    if (lane == 0) {
+      // -------------------------------------------------------------- MMA issuer
+      int s = 0, t = 0;
+      uint32_t sph = 0, mph = 0, uses = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        for (int it = 0; ok && it < nk; ++it) {
+          if (!mbar_wait(smem_u32(&ctl->mfull[t]), mph, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a = smem_u32(mring + t * MMA_BYTES), b = a + OP_BYTES;
+          for (int j = 0; j < 2; ++j, ++uses) {
+            const uint32_t buf = uses & 1, dph = (uses >> 1) & 1;
+            if (!mbar_wait(smem_u32(&ctl->dempty[buf]), dph ^ 1, abort_flag, p.err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t d = tmem + buf * BN;
+            mma_i8(d, desc_k_sw128(a + 64 * j), desc_k_sw128(b + 64 * j), IDESC_I8, 0);
+            mma_i8(d, desc_k_sw128(a + 64 * j + 32), desc_k_sw128(b + 64 * j + 32), IDESC_I8, 1);
+            tc_commit(smem_u32(&ctl->dfull[buf]));
+          }
+          if (!ok) break;
+          tc_commit(smem_u32(&ctl->mempty[t]));
+          if (++t == MS) {
+            t = 0;
+            mph ^= 1;
+          }
+          if (++s == ST) {
+            s = 0;
+            sph ^= 1;
+          }
+        }
+        if (!ok) break;
+        if (nl) {
+          const uint32_t buf = uses & 1, dph = (uses >> 1) & 1;
+          if (!mbar_wait(smem_u32(&ctl->dempty[buf]), dph ^ 1, abort_flag, p.err)) break;
+          for (int c = 0; c < nl; ++c) {
+            if (!mbar_wait(smem_u32(&ctl->sfull[s]), sph, abort_flag, p.err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a = smem_u32(stg + s * STG_BYTES), b = a + STG_HALF;
+            const int steps = min(2, (p.r_tot - 32 * c) / 16);
+            for (int j = 0; j < steps; ++j)
+              mma_bf16(tmem + buf * BN, desc_k_sw64(a + 32 * j), desc_k_sw64(b + 32 * j), IDESC_BF,
+                       (c | j) != 0);
+            tc_commit(smem_u32(&ctl->sempty[s]));
+            if (++s == ST) {
+              s = 0;
+              sph ^= 1;
+            }
+          }
+          if (!ok) break;
+          tc_commit(smem_u32(&ctl->dfull[buf]));
+          ++uses;
+        }
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- rescale + epilogue
+    const int rw = warp - W_RESCALE;                 // 0..7
+    const int sub = warp & 3, half = rw >> 2;        // TMEM sub-partition, 64-column half
+    const int row = sub * 32 + lane;
+    uint32_t uses = 0;
+    const __half* sX = p.sX;
+    const __half* sR = p.sR;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const int mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
+      const int m = mb * BM + row, n0 = nb * BN + half * 64;
+      float acc[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) acc[c] = 0.f;
+      bool ok = true;
+      const int groups = 2 * nk;
+      for (int g = 0; g < groups + (nl ? 1 : 0); ++g, ++uses) {
+        float sx = 0.f;
+        if (g < groups) sx = __half2float(sX[int4_scale_offset(m, g, p.K_pad)]);
+        const uint32_t buf = uses & 1, dph = (uses >> 1) & 1;
+        if (!mbar_wait(smem_u32(&ctl->dfull[buf]), dph, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int hc = 0; hc < 2; ++hc) {
+          uint32_t r[32];
+          tmem_ld32(tmem + ((uint32_t)(sub * 32) << 16) + buf * BN + half * 64 + hc * 32, r);
+          tmem_wait_ld();
+          if (hc == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&ctl->dempty[buf]));
+          }
+          if (g < groups) {
+            // weight scales of these 32 columns: 64 contiguous bytes, the same for the whole warp
+            const uint4* sp = reinterpret_cast<const uint4*>(sR + int4_scale_offset(n0 + hc * 32, g, p.K_pad));
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint4 v = __ldg(sp + i);
+              const __half2* h2 = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 srf = __half22float2(h2[e]);
+                const int c = 8 * i + 2 * e;
+                // exact int32 -> float for |d| < 2^22 (here |d| <= 64 * 8 * 8)
+                const float d0 = __int_as_float(0x4B400000 + (int)r[c]) - 12582912.0f;
+                const float d1 = __int_as_float(0x4B400000 + (int)r[c + 1]) - 12582912.0f;
+                acc[hc * 32 + c] = fmaf(sx * srf.x, d0, acc[hc * 32 + c]);
+                acc[hc * 32 + c + 1] = fmaf(sx * srf.y, d1, acc[hc * 32 + c + 1]);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) acc[hc * 32 + c] += __uint_as_float(r[c]);
+          }
+        }
+      }
+      if (!ok) break;
+      if (m < p.M) {
+#pragma unroll
+        for (int c8 = 0; c8 < 64; c8 += 8) {
+          const int n = n0 + c8;
+          if (n < p.N) {
+            const float4 b0 = __ldg(reinterpret_cast<const float4*>(p.bias + n));
+            const float4 b1 = __ldg(reinterpret_cast<const float4*>(p.bias + n + 4));
+            const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            float y[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              y[e] = acc[c8 + e] + bb[e];
+              if (p.epi == 1) y[e] = gelu_tanh(y[e]);
+            }
+            uint4 o;
+            o.x = pack_bf16x2(y[0], y[1]);
+            o.y = pack_bf16x2(y[2], y[3]);
+            o.z = pack_bf16x2(y[4], y[5]);
+            o.w = pack_bf16x2(y[6], y[7]);
+            *reinterpret_cast<uint4*>(p.Y + (size_t)m * p.N + n) = o;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == W_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+cudaError_t launch_gemm_int4(const CUtensorMap& tmXp, const CUtensorMap& tmRp, const CUtensorMap& tmLR,
+                             const CUtensorMap& tmL2, K2I8Params p, int num_sms, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const int tiles = p.num_m_blocks * p.num_n_blocks;
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  gemm_int4_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tmXp, tmRp, tmLR, tmL2, p);
+  return cudaGetLastError();
 }
 
 }  // namespace svdq

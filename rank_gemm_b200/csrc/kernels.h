@@ -49,7 +49,7 @@ struct K2I8Params {
   int M, N, K_pad, r_tot, r_pad, N_pad;
   int num_m_blocks, num_n_blocks;
   int nk;                  // K_pad / 128 int8 k-tiles (two 64-groups each)
-  int nl;
+  int nl;                  // ceil(r_tot / 32) low-rank chunks (0: plain W4A4 GEMM)
   const __half* sX;        // [M_pad128][K_pad/64]
   const __half* sR;        // [N_pad][K_pad/64]
   const float* bias;
@@ -57,9 +57,8 @@ struct K2I8Params {
   __nv_bfloat16* Y;
   DeviceErr err;
 };
-cudaError_t launch_gemm_int4(const uint8_t* qX, const uint8_t* qR, const CUtensorMap& tmLR,
-                             const CUtensorMap& tmL2, K2I8Params p, int num_sms,
-                             cudaStream_t stream);
+cudaError_t launch_gemm_int4(const CUtensorMap& tmXp, const CUtensorMap& tmRp, const CUtensorMap& tmLR,
+                             const CUtensorMap& tmL2, K2I8Params p, int num_sms, cudaStream_t stream);
 
 // ---------------------------------------------------------------- unfused up projection
 struct UpParams {

@@ -73,7 +73,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (p.fmt == 0)
         p.sX[sf_atom_offset(r, g, p.K_pad)] = 0;
       else if ((g & 3) == 0)
-        reinterpret_cast<__half*>(p.sX)[(size_t)r * (p.K_pad / 64) + g / 4] = __float2half(0.f);
+        reinterpret_cast<__half*>(p.sX)[int4_scale_offset(r, g / 4, p.K_pad)] = __float2half(0.f);
     }
     return;
   }
@@ -176,8 +176,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       } else {
         __half sc;
         quant_int4_16of64(v, codes, sc);
-        if ((qg & 3) == 0)
-          reinterpret_cast<__half*>(p.sX)[(size_t)m * (p.K_pad / 64) + k0 / 64] = sc;
+        if ((qg & 3) == 0) reinterpret_cast<__half*>(p.sX)[int4_scale_offset(m, k0 / 64, p.K_pad)] = sc;
       }
       if (m < p.M) *reinterpret_cast<uint2*>(p.qX + (size_t)m * qx_row_bytes + k0 / 2) = codes;
     }

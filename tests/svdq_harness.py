@@ -38,8 +38,12 @@ def unpack_codes(raw: np.ndarray, rows: int, K: int, K_pad: int, fmt: str) -> np
 
 
 def int4_scales(raw: np.ndarray, rows: int, K: int, K_pad: int) -> np.ndarray:
+    """binary16 scale chunks (128 rows x 2 groups per 128-wide k-tile) -> (rows, K/64)."""
     h = raw.reshape(-1).view(np.float16)
-    return h[: rows * (K_pad // 64)].reshape(rows, K_pad // 64)[:, : K // 64]
+    r = np.arange(rows)[:, None]
+    g = np.arange(K // 64)[None, :]
+    off = (((r // 128) * (K_pad // 128) + g // 2) * 2 + g % 2) * 128 + r % 128
+    return h[off]
 
 
 def to_np(t: torch.Tensor) -> np.ndarray:
