@@ -216,3 +216,31 @@ def test_capability_check_rejects_other_devices(B):
     finally:
         B.svdq_debug_override_cc(-1, 0)
         g.close()
+
+
+# ------------------------------------------------------------------ INT4 (int8 tensor-core path)
+def test_int4_small_parity(B):
+    L = workloads.draw_layer("int4", "int4", 200, 512, 384, 32, seed=21, n_out=4)
+    print("int4:", _full_check(L))
+
+
+def test_int4_ragged_gelu_lora(B):
+    L = workloads.draw_layer("int4r", "int4", 77, 320, 272, 16, seed=22, n_out=3, gelu=True, lora_rank=16)
+    print("int4 ragged:", _full_check(L, gelu=True, lora=True))
+
+
+def test_int4_unfused_and_plain(B):
+    L = workloads.draw_layer("int4u", "int4", 130, 768, 256, 32, seed=23, n_out=4)
+    g = GpuLayer(L.fmt, L.X, L.W, L.bias, L.rank)
+    try:
+        Xd = dev_bf16(L.X)
+        Y_o = S.forward(g.pw, L.X)["Y"]
+        assert_y(bf16_np(g.linear(Xd, L.M, unfused=True)), Y_o)
+        qX, sX, LR = g.kernel1(Xd, L.M)
+        Yp = torch.empty(L.M, L.N, dtype=torch.bfloat16, device="cuda")
+        B.svdq_w4a4_gemm(g.h, L.M, qX, sX, Yp)
+        torch.cuda.synchronize()
+        oq, osc = S.quantize_activation(g.pw, L.X)
+        assert_y(bf16_np(Yp), S.epilogue(S.main_product(g.pw, oq, osc), g.pw.bias, False))
+    finally:
+        g.close()
