@@ -213,6 +213,38 @@ svdq_status svdq_linear(const svdq_weights* w, int M, const void* X, svdq_epilog
                         void* workspace, size_t ws_bytes, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * svdq_linear without a workspace argument (no counterpart in the paper: it
+ * is an integration convenience, not part of the method).
+ *
+ * Some callers cannot allocate device memory at the point where they run
+ * the layer: cudaMalloc may synchronize the whole device and take
+ * milliseconds, which a latency-critical serving loop cannot afford, and a
+ * plug-in hosted by an application that owns all device memory through its
+ * own allocator is often given no allocator at all.  This entry point keeps
+ * the intermediates qX, sX and LR in a scratch array that is part of the
+ * library image (SVDQ_NOALLOC_SCRATCH_BYTES per GPU, held by every GPU that
+ * loads the library until the process exits).  It calls no cudaMalloc,
+ * cudaFree or allocating library routine; the caller still passes X and Y.
+ *   - Sizes: svdq_linear_workspace_bytes(w, M) must not exceed
+ *     SVDQ_NOALLOC_SCRATCH_BYTES (32 MiB: at rank 32 about 1.9 KB per row
+ *     for K = 3072, so M up to about 18,000, and about 4,700 rows for
+ *     K = 12288); a larger request returns SVDQ_ERR_WORKSPACE before
+ *     anything is launched.
+ *   - The first call on each device looks up the scratch array's device
+ *     address for that device (a runtime query, no allocation), so that
+ *     first call should come before any stream capture.
+ *   - All calls on a device share the one array and it keeps the previous
+ *     call's contents; nothing in it needs clearing, because kernel 1
+ *     rewrites every byte kernel 2 reads.  Calls whose kernels overlap on
+ *     the GPU (different streams, no ordering between them) race on the
+ *     array: order them, e.g. issue them on one stream.
+ * Errors: as svdq_linear, plus WORKSPACE when M is too large.
+ * ------------------------------------------------------------------------ */
+#define SVDQ_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+svdq_status svdq_linear_noalloc(const svdq_weights* w, int M, const void* X, svdq_epilogue epi, void* Y,
+                                cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * Unfused baseline ("Nunchaku engine design" figure (a): run naively, the
  * rank-32 branch costs an extra 16-bit read of X in the down projection and
  * an extra 16-bit write of Y in the up projection, 57% latency overhead).

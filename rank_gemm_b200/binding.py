@@ -68,6 +68,7 @@ _SIGS = {
     "svdq_w4a4_gemm": (_i, [_vp, _i, _vp, _vp, _vp, _vp]),
     "svdq_lowrank_up": (_i, [_vp, _i, _vp, _i, _vp, _vp]),
     "svdq_linear_unfused": (_i, [_vp, _i, _vp, _i, _vp, _vp, _sz, _vp]),
+    "svdq_linear_noalloc": (_i, [_vp, _i, _vp, _i, _vp, _vp]),
     "svdq_poll_device_error": (_i, [_vp]),
     "svdq_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
     "svdq_debug_override_cc": (None, [_i, _i]),
@@ -182,6 +183,16 @@ def svdq_linear_unfused(w, M, X, epi, Y, workspace, ws_bytes=None, stream=None):
     ws_bytes = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
     _check(lib.svdq_linear_unfused(w, M, _ptr(X), epi, _ptr(Y), _ptr(workspace), ws_bytes, _stream(stream)),
            "svdq_linear_unfused")
+
+
+def svdq_linear_noalloc(w, M, X, epi, Y, stream=None):
+    """svdq_linear with the intermediates in the library's own scratch array
+    (no workspace, no allocation); see include/svdq.h for its size limit and
+    the rule that calls overlapping on the GPU race."""
+    _check(lib.svdq_linear_noalloc(w, M, _ptr(X), epi, _ptr(Y), _stream(stream)), "svdq_linear_noalloc")
+
+
+SVDQ_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 def svdq_poll_device_error(stream=None) -> int:
