@@ -327,6 +327,40 @@ def run_ours(args, world, rank, local):
     bytes_k2 = qb + sb + lb + (N * K // 2) + (N * K // 16) + N * 64 * 2 + N * 4 + M * N * 2
     traffic = profiled_traffic("gemm_nvfp4_qkv.md", os.path.join(ROOT, "rank_gemm_b200", "csrc", "gemm_nvfp4.cu"))
 
+    # low-rank overhead (the "Nunchaku engine design" figure's comparison):
+    # plain W4A4 path (quantize + GEMM, no low-rank branch), the fused layer,
+    # and the naive four-launch path, each timed over the same steps
+    def timed(fn, n):
+        for i in range(3):
+            fn(i)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for i in range(n):
+            fn(i)
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    def plain(i):
+        qX, sX, LR = acts[i % sets]
+        B.svdq_quantize_act(h, M, Xs[i % sets], qX, sX, stream)
+        B.svdq_w4a4_gemm(h, M, qX, sX, Ys[i % sets], stream)
+
+    def unfused(i):
+        qX, sX, LR = acts[i % sets]
+        B.svdq_quantize_act(h, M, Xs[i % sets], qX, sX, stream)
+        B.svdq_lowrank_down(h, M, Xs[i % sets], LR, stream)
+        B.svdq_w4a4_gemm(h, M, qX, sX, Ys[i % sets], stream)
+        B.svdq_lowrank_up(h, M, LR, B.SVDQ_EPI_NONE, Ys[i % sets], stream)
+
+    n_ov = min(K_steps, 100)
+    t_plain = timed(plain, n_ov)
+    t_fused = timed(lambda i: (B.svdq_quantize_act_lowrank_down(h, M, Xs[i % sets], *acts[i % sets], stream),
+                               B.svdq_w4a4_gemm_lowrank_up(h, M, *acts[i % sets], B.SVDQ_EPI_NONE,
+                                                           Ys[i % sets], stream)), n_ov)
+    t_unfused = timed(unfused, n_ov)
+
     # end to end through the public call with host buffers
     e2e_steps = min(K_steps, 50)
     Xh = torch.empty(M, K, dtype=torch.bfloat16, pin_memory=True)
@@ -372,6 +406,10 @@ def run_ours(args, world, rank, local):
                                "algorithmic_bytes": bytes_k1, "us": round(k1_ms * 1e3, 2)},
                "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": M * K * 2,
                        "d2h_bytes_per_step": M * N * 2, "ms_per_step": round(e2e_ms, 4)},
+               "lowrank_overhead": {"plain_w4a4_us": round(t_plain * 1e3, 2), "fused_us": round(t_fused * 1e3, 2),
+                                    "unfused_us": round(t_unfused * 1e3, 2),
+                                    "fused_over_plain": round(t_fused / t_plain - 1, 4),
+                                    "unfused_over_plain": round(t_unfused / t_plain - 1, 4)},
                "gpu_launches": 2 * K_steps,
                "device_status": status,
                "clocks": clocks.summary()}

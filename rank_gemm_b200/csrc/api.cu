@@ -32,8 +32,9 @@ struct svdq_weights {
   __nv_bfloat16* L2a;
   float* bias_f;
   float* lambda_inv;
+  float* lambda_inv_k1;
   float s_tR, s_tX, alpha;
-  CUtensorMap tm_qR, tm_L2a, tm_L1t;
+  CUtensorMap tm_qR, tm_L2a;
   CUtensorMap tm_qR_i4, tm_L2a_i4;   // INT4 kernel: packed 64-byte rows / 32-column low-rank chunks
 };
 
@@ -157,7 +158,8 @@ K1Params k1_params(const svdq_weights* w, const DevState* d, int M, void* qX, vo
   p.do_quant = do_quant;
   p.do_lr = do_lr;
   p.stages = 0;
-  p.inv_lambda = w->lambda_inv;
+  p.inv_lambda = w->lambda_inv_k1;
+  p.L1t = w->L1t;
   p.s_t = w->s_tX;
   p.six_st = 6.0f * w->s_tX;   // one IEEE float32 multiply on the host
   p.qX = static_cast<uint8_t*>(qX);
@@ -175,7 +177,7 @@ svdq_status run_k1(const svdq_weights* w, int M, const void* X, void* qX, void* 
   CUtensorMap tmX;
   if (!tmap_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, w->K, M, (uint64_t)w->K * 2, 64, 32))
     return SVDQ_ERR_CUDA;
-  return from_cuda(launch_quant_down(tmX, w->tm_L1t, k1_params(w, d, M, qX, sX, LR, do_quant, do_lr), stream));
+  return from_cuda(launch_quant_down(tmX, k1_params(w, d, M, qX, sX, LR, do_quant, do_lr), stream));
 }
 
 svdq_status run_k2(const svdq_weights* w, int M, const void* qX, const void* sX, const void* LR,
@@ -225,7 +227,7 @@ svdq_status run_k2(const svdq_weights* w, int M, const void* qX, const void* sX,
   p.r_pad = w->r_pad;
   p.N_pad = w->N_pad;
   p.num_m_blocks = (M + 127) / 128;
-  p.num_n_blocks = w->N_pad / 256;
+  p.num_n_blocks = w->N_pad / 128;   // the INT4 kernel's tiles are 128 wide
   p.nk = w->K_pad / 128;
   p.nl = lowrank ? (w->r_tot + 31) / 32 : 0;
   p.sX = static_cast<const __half*>(sX);
@@ -244,6 +246,7 @@ void free_buffers(svdq_weights* w) {
   cudaFree(w->L2a);
   cudaFree(w->bias_f);
   cudaFree(w->lambda_inv);
+  cudaFree(w->lambda_inv_k1);
 }
 
 }  // namespace
@@ -327,10 +330,11 @@ svdq_status svdq_prepare_weights(svdq_format fmt, int K, int N, int rank, const 
   float* R = nullptr;
   unsigned* amax = nullptr;
   bool ok = cudaMalloc(&w->qR, qr_b) == cudaSuccess && cudaMalloc(&w->sR, sr_b) == cudaSuccess &&
-            cudaMalloc(&w->L1t, (size_t)r_tot * K * 2) == cudaSuccess &&
+            cudaMalloc(&w->L1t, (size_t)r_tot * w->K_pad * 2) == cudaSuccess &&
             cudaMalloc(&w->L2a, (size_t)w->N_pad * w->r_pad * 2) == cudaSuccess &&
             cudaMalloc(&w->bias_f, (size_t)w->N_pad * 4) == cudaSuccess &&
             cudaMalloc(&w->lambda_inv, (size_t)K * 4) == cudaSuccess &&
+            cudaMalloc(&w->lambda_inv_k1, (size_t)w->K_pad * 4) == cudaSuccess &&
             cudaMalloc(&R, (size_t)N * K * 4) == cudaSuccess && cudaMalloc(&amax, 256) == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
@@ -365,6 +369,7 @@ svdq_status svdq_prepare_weights(svdq_format fmt, int K, int N, int rank, const 
   p.L2a = w->L2a;
   p.bias_f = w->bias_f;
   p.lambda_inv = w->lambda_inv;
+  p.lambda_inv_k1 = w->lambda_inv_k1;
 
   unsigned amax_host = 0;
   cudaError_t e = launch_prepare_residual(p, stream);
@@ -399,8 +404,6 @@ svdq_status svdq_prepare_weights(svdq_format fmt, int K, int N, int rank, const 
                       128, 256) &&
               tmap_2d(&w->tm_L2a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->L2a, w->r_pad, w->N_pad,
                       (uint64_t)w->r_pad * 2, 64, 256) &&
-              tmap_2d(&w->tm_L1t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->L1t, K, r_tot, (uint64_t)K * 2, 64,
-                      r_tot) &&
               tmap_2d(&w->tm_qR_i4, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->qR, w->K_pad / 2, w->N_pad, w->K_pad / 2,
                       64, 128, CU_TENSOR_MAP_SWIZZLE_NONE) &&
               tmap_2d(&w->tm_L2a_i4, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->L2a, w->r_pad, w->N_pad,

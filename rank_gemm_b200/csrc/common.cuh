@@ -225,8 +225,8 @@ __device__ __forceinline__ void tmem_wait_ld() {
 }
 
 // ----------------------------------------------------------------- conversions
-// Eight non-negative floats -> eight E2M1 magnitude codes in one word
-// (element j in bits 4j..4j+3), round to nearest even, saturate to 6.
+// Eight floats -> eight E2M1 codes in one word (element j in bits 4j..4j+3),
+// round to nearest even, saturate to +-6, sign kept.
 __device__ __forceinline__ uint32_t cvt_e2m1x8(float x0, float x1, float x2, float x3, float x4,
                                                float x5, float x6, float x7) {
   uint32_t r;
@@ -255,6 +255,34 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
   return (code & 0x80u) ? -v : v;
 }
 
+// ----------------------------------------------------------------- packed float32 helpers
+// Two IEEE float32 multiplies (round to nearest even) in one instruction.
+__device__ __forceinline__ void mul2_rn(float a0, float a1, float b0, float b1, float& r0, float& r1) {
+  uint64_t a, b, r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(b) : "f"(b0), "f"(b1));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r0), "=f"(r1) : "l"(r));
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// max |v_j| over 16 values
+__device__ __forceinline__ float absmax16(const float (&v)[16]) {
+  float a = max3f(fabsf(v[0]), fabsf(v[1]), fabsf(v[2]));
+  a = max3f(a, fabsf(v[3]), fabsf(v[4]));
+  a = max3f(a, fabsf(v[5]), fabsf(v[6]));
+  a = max3f(a, fabsf(v[7]), fabsf(v[8]));
+  a = max3f(a, fabsf(v[9]), fabsf(v[10]));
+  a = max3f(a, fabsf(v[11]), fabsf(v[12]));
+  a = max3f(a, fabsf(v[13]), fabsf(v[14]));
+  return fmaxf(a, fabsf(v[15]));
+}
+
 // ----------------------------------------------------------------- 4-bit group quantizers
 // NVFP4, one 16-element group: a = max|v|; sb = E4M3(a / six_st) with six_st
 // = fl32(6 s_t); d = fl32(f32(sb) s_t); inv = fl32(1/d) (0 if d == 0);
@@ -262,9 +290,7 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
 // bytes (element 2j in the low nibble of byte j) and the scale byte.
 __device__ __forceinline__ void quant_nvfp4_16(const float (&v)[16], float s_t, float six_st,
                                                uint2& codes, uint32_t& scale) {
-  float a = 0.f;
-#pragma unroll
-  for (int j = 0; j < 16; ++j) a = fmaxf(a, fabsf(v[j]));
+  const float a = absmax16(v);
   const uint32_t sb = cvt_e4m3(__fdiv_rn(a, six_st));
   const float d = __fmul_rn(e4m3_to_f32(sb), s_t);
   const float inv = (d == 0.f) ? 0.f : __frcp_rn(d);
@@ -273,14 +299,37 @@ __device__ __forceinline__ void quant_nvfp4_16(const float (&v)[16], float s_t, 
   for (int h = 0; h < 2; ++h) {
     float x[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) x[j] = __fmul_rn(v[8 * h + j], inv);
-    // magnitude from the converter, sign from the input: a negative value
-    // that rounds to zero keeps its sign (code 0x8)
-    uint32_t c = cvt_e2m1x8(fabsf(x[0]), fabsf(x[1]), fabsf(x[2]), fabsf(x[3]), fabsf(x[4]),
-                            fabsf(x[5]), fabsf(x[6]), fabsf(x[7]));
+    for (int j = 0; j < 8; j += 2) mul2_rn(v[8 * h + j], v[8 * h + j + 1], inv, inv, x[j], x[j + 1]);
+    // the converter keeps the sign of a negative value that rounds to zero
+    // (code 0x8), the same rule as the definition; the exhaustive bf16 sweep
+    // in the GPU tests checks it
+    w[h] = cvt_e2m1x8(x[0], x[1], x[2], x[3], x[4], x[5], x[6], x[7]);
+  }
+  codes = make_uint2(w[0], w[1]);
+  scale = sb;
+}
+
+// The same NVFP4 group quantizer with the per-code reciprocal taken from a
+// table: inv_tab[c] = fl32(1 / fl32(f32(E4M3 c) s_t)) (0 where that product
+// is 0), built once with exactly the operations above, so the codes are
+// bit-identical to quant_nvfp4_16.
+__device__ __forceinline__ float nvfp4_inv_entry(uint32_t code, float s_t) {
+  const float d = __fmul_rn(e4m3_to_f32(code), s_t);
+  return (d == 0.f) ? 0.f : __frcp_rn(d);
+}
+
+__device__ __forceinline__ void quant_nvfp4_16_tab(const float (&v)[16], float six_st, const float* inv_tab,
+                                                   uint2& codes, uint32_t& scale) {
+  const float a = absmax16(v);
+  const uint32_t sb = cvt_e4m3(__fdiv_rn(a, six_st));
+  const float inv = inv_tab[sb];
+  uint32_t w[2];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) c |= (__float_as_uint(x[j]) >> 31) << (4 * j + 3);
-    w[h] = c;
+  for (int h = 0; h < 2; ++h) {
+    float x[8];
+#pragma unroll
+    for (int j = 0; j < 8; j += 2) mul2_rn(v[8 * h + j], v[8 * h + j + 1], inv, inv, x[j], x[j + 1]);
+    w[h] = cvt_e2m1x8(x[0], x[1], x[2], x[3], x[4], x[5], x[6], x[7]);
   }
   codes = make_uint2(w[0], w[1]);
   scale = sb;
@@ -292,9 +341,7 @@ __device__ __forceinline__ void quant_nvfp4_16(const float (&v)[16], float s_t, 
 // Each lane returns its 16 codes as 8 bytes (two's-complement nibbles).
 __device__ __forceinline__ void quant_int4_16of64(const float (&v)[16], uint2& codes,
                                                   __half& scale) {
-  float a = 0.f;
-#pragma unroll
-  for (int j = 0; j < 16; ++j) a = fmaxf(a, fabsf(v[j]));
+  float a = absmax16(v);
   a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
   a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
   const __half sb = __float2half_rn(__fdiv_rn(a, 7.0f));

@@ -18,8 +18,10 @@
 //               tile, then tcgen05.mma.kind::f16 adds LR (L2/alpha) into the
 //               same tile; tcgen05.commit releases ring slots and hands the
 //               finished tile to the epilogue.
-//   warps 2-5   epilogue: tcgen05.ld 32 columns at a time, y = alpha acc + b,
-//               optional GELU, bf16, 16-byte stores of each row segment.
+//   warps 2-9   epilogue: two warps per TMEM sub-partition, 128 columns each;
+//               the whole 128 x 256 tile is loaded to registers and the TMEM
+//               accumulator released before y = alpha acc + b, optional GELU,
+//               bf16 and the 16-byte stores, which overlap the next tile's MMAs.
 // All waits are bounded (see mbar_wait); TMEM is freed on every exit path.
 #include "common.cuh"
 #include "kernels.h"
@@ -34,7 +36,8 @@ constexpr int B_BYTES = BLOCK_N * 128;          // 32 KB
 constexpr int SFA_BYTES = 4 * 512;              // 4 k-blocks of 64 x 128 rows
 constexpr int SFB_BYTES = 2 * 4 * 512;          // 2 row halves x 4 k-blocks
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;   // 54 KB
-constexpr int THREADS = 192;
+constexpr int THREADS = 320;              // producer, MMA, 8 epilogue warps
+constexpr int EPI_WARPS = 8;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0, SFA_COL = 256, SFB_COL = 272;
 constexpr uint32_t IDESC_F4 = idesc_nvf4(BLOCK_M, BLOCK_N);
@@ -48,7 +51,19 @@ struct Ctl {
   int abort;
 };
 
-constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 + sizeof(Ctl);
+constexpr int BIAS_BYTES = EPI_WARPS * 128 * 4;   // warp-private bias slices
+constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + BIAS_BYTES + 1024 + sizeof(Ctl);
+
+// Tile order: groups of 8 row blocks, column blocks within a group, so the
+// CTAs running at the same time share each activation tile among ~8 and each
+// weight tile among ~18 readers instead of reading one weight tile all at once.
+__device__ __forceinline__ void tile_coords(int tile, int nmb, int nnb, int& mb, int& nb) {
+  constexpr int GM = 8;
+  const int grp = tile / (GM * nnb), rr = tile % (GM * nnb);
+  const int gs = min(GM, nmb - grp * GM);
+  mb = grp * GM + rr % gs;
+  nb = rr / gs;
+}
 
 __device__ __forceinline__ float gelu_tanh(float y) {
   const float u = 0.7978845608028654f * (y + 0.044715f * y * y * y);
@@ -68,7 +83,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                       K2Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Ctl* ctl = reinterpret_cast<Ctl*>(base + STAGES * STAGE_BYTES);
+  float* bias_s = reinterpret_cast<float*>(base + STAGES * STAGE_BYTES);
+  Ctl* ctl = reinterpret_cast<Ctl*>(base + STAGES * STAGE_BYTES + BIAS_BYTES);
   volatile int* abort_flag = &ctl->abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -84,7 +100,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(smem_u32(&ctl->empty[s]), 1);
     }
     mbar_init(smem_u32(&ctl->tfull), 1);
-    mbar_init(smem_u32(&ctl->tempty), 4);
+    mbar_init(smem_u32(&ctl->tempty), EPI_WARPS);
     ctl->abort = 0;
     fence_barrier_init();
   }
@@ -108,7 +124,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t phase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-        const int mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
+        int mb, nb;
+        tile_coords(tile, p.num_m_blocks, p.num_n_blocks, mb, nb);
         for (int it = 0; it < kiters; ++it) {
           if (!mbar_wait(smem_u32(&ctl->empty[stage]), phase ^ 1, abort_flag, p.err)) {
             ok = false;
@@ -188,47 +205,62 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // -------------------------------------------------------------- epilogue
-    const int sub = warp & 3;                 // TMEM lanes 32 sub .. 32 sub + 31
+    // Warp e = warp - 2 drains TMEM lanes 32 (warp % 4) .. +31 (its sub-partition),
+    // columns [128 (e / 4), +128): all four 32-column loads are issued before one
+    // wait, the accumulator is released at once, and the bias / GELU / bf16 /
+    // store work then overlaps the MMAs of the next tile.
+    const int e = warp - 2, sub = warp & 3, ch = e >> 2;
     const int row = sub * 32 + lane;
+    float* bslice = bias_s + e * 128;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      const int mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
+      int mb, nb;
+      tile_coords(tile, p.num_m_blocks, p.num_n_blocks, mb, nb);
+      const int n0 = nb * BLOCK_N + ch * 128;
+      // this warp's 128 bias values, staged before the accumulator is ready
+      const float4 bv = __ldg(reinterpret_cast<const float4*>(p.bias + n0) + lane);
+      __syncwarp();
+      reinterpret_cast<float4*>(bslice)[lane] = bv;
+      __syncwarp();
       if (!mbar_wait(smem_u32(&ctl->tfull), acc_phase, abort_flag, p.err)) break;
       tc_fence_after();
+      uint32_t r[4][32];
+      const uint32_t taddr = tmem + ((uint32_t)(sub * 32) << 16) + ACC_COL + ch * 128;
+      tmem_ld32(taddr, r[0]);
+      tmem_ld32(taddr + 32, r[1]);
+      tmem_ld32(taddr + 64, r[2]);
+      tmem_ld32(taddr + 96, r[3]);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&ctl->tempty));
+      acc_phase ^= 1;
       const int m = mb * BLOCK_M + row;
-      for (int c = 0; c < BLOCK_N / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem + ((uint32_t)(sub * 32) << 16) + ACC_COL + c * 32, r);
-        tmem_wait_ld();
-        const int n0 = nb * BLOCK_N + c * 32;
-        if (m < p.M) {
+      if (m < p.M) {
+        __nv_bfloat16* yrow = p.Y + (size_t)m * p.N;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const int n = n0 + 8 * q;
+            const int col = c * 32 + q * 8;
+            const int n = n0 + col;
             if (n < p.N) {
-              const float4 b0 = __ldg(reinterpret_cast<const float4*>(p.bias + n));
-              const float4 b1 = __ldg(reinterpret_cast<const float4*>(p.bias + n + 4));
-              const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
               float y[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                y[e] = fmaf(p.alpha, __uint_as_float(r[8 * q + e]), bb[e]);
-                if (p.epi == 1) y[e] = gelu_tanh(y[e]);
+              for (int j = 0; j < 8; ++j) {
+                y[j] = fmaf(p.alpha, __uint_as_float(r[c][q * 8 + j]), bslice[col + j]);
+                if (p.epi == 1) y[j] = gelu_tanh(y[j]);
               }
               uint4 o;
               o.x = pack_bf16x2(y[0], y[1]);
               o.y = pack_bf16x2(y[2], y[3]);
               o.z = pack_bf16x2(y[4], y[5]);
               o.w = pack_bf16x2(y[6], y[7]);
-              *reinterpret_cast<uint4*>(p.Y + (size_t)m * p.N + n) = o;
+              *reinterpret_cast<uint4*>(yrow + n) = o;
             }
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&ctl->tempty));
-      acc_phase ^= 1;
     }
   }
 

@@ -17,15 +17,15 @@ struct K1Params {
   int fmt;                 // 0 NVFP4, 1 INT4
   int do_quant, do_lr;     // fused: both; unfused baseline: one of them
   int stages;              // set by the launcher
-  const float* inv_lambda; // [K]
+  const float* inv_lambda; // [K_pad], permuted per stage (see prepare.cu)
+  const __nv_bfloat16* L1t; // L1f^T in the staged layout (one contiguous tile per stage)
   float s_t, six_st;       // NVFP4 activation tensor scale and fl32(6 s_t)
   uint8_t* qX;             // [M][K_pad/2]
   uint8_t* sX;             // scale layout (see svdq.h)
   __nv_bfloat16* LR;       // [M][r_pad]
   DeviceErr err;
 };
-cudaError_t launch_quant_down(const CUtensorMap& tmX, const CUtensorMap& tmL1, K1Params p,
-                              cudaStream_t stream);
+cudaError_t launch_quant_down(const CUtensorMap& tmX, K1Params p, cudaStream_t stream);
 
 // ---------------------------------------------------------------- kernel 2
 struct K2Params {
@@ -89,10 +89,11 @@ struct PrepParams {
   unsigned* amax_bits;         // scratch, 1 word
   uint8_t* qR;                 // [N_pad][K_pad/2]
   uint8_t* sR;                 // scales
-  __nv_bfloat16* L1t;          // [r_tot][K]
+  __nv_bfloat16* L1t;          // [K_pad/256][4][r_tot][64], 128-byte swizzled
   __nv_bfloat16* L2a;          // [N_pad][r_pad]
   float* bias_f;               // [N_pad]
   float* lambda_inv;           // [K]
+  float* lambda_inv_k1;        // [K_pad], permuted per 256-wide stage for kernel 1
 };
 cudaError_t launch_prepare_residual(const PrepParams& p, cudaStream_t stream);
 cudaError_t launch_prepare_quantize(const PrepParams& p, float s_tR, float alpha,

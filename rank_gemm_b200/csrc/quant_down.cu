@@ -3,18 +3,27 @@
 // model card: the Quantize and Down Projection kernels read the same input,
 // so they are fused and X is read from HBM once).
 //
-// One CTA owns 32 rows of X and walks all of K in 128-column stages.  TMA
-// stages each [32 x 128] bf16 tile of X (and the matching [r_tot x 128] tile
-// of L1f^T) into shared memory through a multi-stage mbarrier ring.  From the
-// same staged tile:
-//   * every thread quantizes one 16-element group of one row (x^ = x / lambda,
-//     amax, block scale, 4-bit codes) and writes packed codes and scales in
-//     the layout kernel 2's tensor-core MMA consumes;
-//   * every warp runs bf16 mma.sync tiles of LR = X L1f with fp32 accumulators
-//     that stay in registers across the whole K loop (no atomics, no second
-//     pass), then writes LR in bf16 once at the end.
-// The kernel is HBM-bound: per row it reads 2K bytes of X and writes about
-// K/2 + K/16 bytes of codes and scales plus 2 r_pad bytes of LR.
+// One CTA owns 32 rows of X and walks all of K in 256-column stages.  A
+// producer warp keeps a TMA ring of stages in flight; a stage holds the
+// [32 x 256] bf16 tile of X (four 128-byte-swizzled boxes), the matching
+// [r_tot x 256] tile of L1f^T (stored pre-swizzled, one contiguous bulk copy)
+// and the 256 values of 1/lambda.  Each CTA walks
+// the stages starting at its own offset, so the CTAs of a wave read different
+// L1f^T tiles and different X columns at any moment.  From the same staged
+// tile:
+//   * 16 quantizer warps: every thread one 16-element group of one row
+//     (x^ = x / lambda, amax, block scale, 4-bit codes), written packed with
+//     scales in the layout kernel 2's tensor-core MMA consumes;
+//   * one thread issues the down projection on the 5th-generation tensor core
+//     as the transposed product LR^T = L1f^T X^T: A = the L1f^T tile (128 rows
+//     per MMA, rows past r_tot are ignored), B = the staged X tile itself
+//     (N = 32 rows), fp32 accumulation in a 32-column TMEM tile across all of
+//     K; four warps read it out at the end and store LR in bf16.
+// Stages are released through an mbarrier (the 16 quantizer warps plus the
+// MMA commit) instead of a CTA-wide sync, so warps drift apart and overlap
+// their load, math and store phases.  The kernel is HBM-bound: per row it
+// reads 2K bytes of X and writes about K/2 + K/16 bytes of codes and scales
+// plus 2 r_pad bytes of LR.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -22,28 +31,20 @@ namespace svdq {
 
 namespace {
 
-constexpr int BM = 32;         // rows per CTA
-constexpr int BK = 128;        // K columns per stage (two 64-column TMA boxes)
-constexpr int THREADS = 256;
+constexpr int BM = 32;                       // rows per CTA (= MMA N)
+constexpr int BK = 256;                      // K columns per stage (four 64-column TMA boxes)
+constexpr int QWARPS = 16;                   // quantizer warps
+constexpr int THREADS = 32 * (QWARPS + 2);   // + producer warp + MMA warp
+constexpr int X_BOX = BM * 128;              // one [32 x 64] bf16 box
+constexpr int X_BYTES = 4 * X_BOX;           // 16 KB
+constexpr int IL_BYTES = BK * 4;             // 1/lambda for the stage
+constexpr int W_PROD = 0, W_MMA = 1, W_Q0 = 2;
+constexpr int CHAINS = 1;                     // LR accumulators (interleaved k16 steps)
 
-__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                            uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldmatrix_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
-               : "=r"(r0), "=r"(r1)
-               : "r"(addr));
-}
-__device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                          uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 u;
+  asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w) : "r"(addr));
+  return u;
 }
 
 // Address of the 16-byte chunk holding columns [8c, 8c+8) of row `row` in a
@@ -52,13 +53,29 @@ __device__ __forceinline__ uint32_t sw128_chunk(uint32_t box_base, int row, int 
   return box_base + row * 128 + ((c ^ (row & 7)) << 4);
 }
 
-constexpr int MAX_PAIRS_PER_WARP = 8;   // r_tot <= 256 -> 2 * 32 (m, n) tiles over 8 warps
+struct Layout {
+  int stages, l_box, x_ring, il_ring, l_ring, bar_off;
+};
+
+// Shared memory: X ring | 1/lambda ring | L1f^T boxes (compact) + a tail so
+// an M = 128 MMA reading past the last box stays inside the allocation |
+// barriers.
+__host__ __device__ inline Layout make_layout(int stages, int r_tot, bool do_lr) {
+  Layout L;
+  L.stages = stages;
+  L.l_box = do_lr ? r_tot * 128 : 0;
+  L.x_ring = 0;
+  L.il_ring = stages * X_BYTES;
+  L.l_ring = L.il_ring + stages * IL_BYTES;
+  const int tail = do_lr ? (r_tot > 128 ? 32768 : 16384) : 0;
+  L.bar_off = L.l_ring + stages * 4 * L.l_box + tail;
+  return L;
+}
 
 }  // namespace
 
 __global__ void __launch_bounds__(THREADS, 1)
-    quant_down_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmL1,
-                      K1Params p) {
+    quant_down_kernel(const __grid_constant__ CUtensorMap tmX, K1Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int m0 = blockIdx.x * BM;
@@ -79,100 +96,129 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int x_bytes = BM * BK * 2;                        // 8 KB
-  const int l_bytes = p.do_lr ? p.r_tot * BK * 2 : 0;    // r_tot x 128 bf16
-  const int stage_bytes = x_bytes + l_bytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(base + p.stages * stage_bytes);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(full + p.stages);
+  const Layout L = make_layout(p.stages, p.r_tot, p.do_lr != 0);
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + L.bar_off);
+  uint64_t* empty = full + p.stages;
+  uint64_t* dfull = empty + p.stages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(dfull + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* inv_tab = reinterpret_cast<float*>(tmem_slot + 4);        // 128 entries, NVFP4 only
+  // LR accumulates in CHAINS independent TMEM tiles (k16 step j goes to chain
+  // j % CHAINS) so consecutive MMAs do not wait on each other's result; per
+  // 128-row half of L1f^T: CHAINS x 32 columns
+  const int halves = p.r_tot > 128 ? 2 : 1;
+  const uint32_t tmem_cols = (uint32_t)(halves * CHAINS * BM);
 
   const int nk = p.K_pad / BK;
+  const int k_first = blockIdx.x % nk;                   // this CTA's first stage
   if (tid == 0) {
     tma_prefetch_desc(&tmX);
-    if (p.do_lr) tma_prefetch_desc(&tmL1);
-    for (int s = 0; s < p.stages; ++s) mbar_init(smem_u32(&full[s]), 1);
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), (p.do_quant ? QWARPS : 0) + (p.do_lr ? 1 : 0));
+    }
+    mbar_init(smem_u32(dfull), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
+  if (p.fmt == 0 && tid < 128) inv_tab[tid] = nvfp4_inv_entry((uint32_t)tid, p.s_t);
+  if (p.do_lr && warp == W_MMA) {
+    tmem_alloc(smem_u32(tmem_slot), tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = p.do_lr ? *tmem_slot : 0u;
 
-  auto issue = [&](int kt) {
-    const int s = kt % p.stages;
-    const uint32_t st = smem_u32(base + s * stage_bytes);
-    const uint32_t bar = smem_u32(&full[s]);
-    mbar_arrive_expect_tx(bar, stage_bytes);
-    tma_load_2d(st, &tmX, kt * BK, m0, bar);
-    tma_load_2d(st + x_bytes / 2, &tmX, kt * BK + 64, m0, bar);
-    if (p.do_lr) {
-      tma_load_2d(st + x_bytes, &tmL1, kt * BK, 0, bar);
-      tma_load_2d(st + x_bytes + l_bytes / 2, &tmL1, kt * BK + 64, 0, bar);
-    }
-  };
-  if (tid == 0)
-    for (int kt = 0; kt < min(nk, p.stages); ++kt) issue(kt);
-
-  // LR accumulators: warp w owns (m-tile w & 1) x (n-tiles (w >> 1) + 4 i).
-  const int mt = warp & 1;
-  const int n_tiles = p.r_tot / 8;
-  float acc[MAX_PAIRS_PER_WARP][4];
+  if (warp == W_PROD) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      for (int it = 0; it < nk; ++it) {
+        const int s = it % p.stages;
+        if (!mbar_wait(smem_u32(&empty[s]), ((it / p.stages) & 1) ^ 1, abort_flag, p.err)) break;
+        const int kt = (k_first + it) % nk;
+        const uint32_t bar = smem_u32(&full[s]);
+        mbar_arrive_expect_tx(bar, X_BYTES + 4 * L.l_box + IL_BYTES);
+        const uint32_t xs = smem_u32(base + L.x_ring + s * X_BYTES);
 #pragma unroll
-  for (int i = 0; i < MAX_PAIRS_PER_WARP; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-
-  // quantization role: row qr, 16-column group qg of the stage
-  const int qr = tid >> 3, qg = tid & 7;
-  const int m = m0 + qr;
-  const size_t qx_row_bytes = (size_t)(p.K_pad / 2);
-
-  bool ok = true;
-  for (int kt = 0; kt < nk; ++kt) {
-    const int s = kt % p.stages;
-    if (!mbar_wait(smem_u32(&full[s]), (kt / p.stages) & 1, abort_flag, p.err)) {
-      ok = false;
-      break;
-    }
-    const uint32_t st = smem_u32(base + s * stage_bytes);
-
-    if (p.do_quant) {
-      const int k0 = kt * BK + qg * 16;
-      const uint32_t box = st + (qg >> 2) * (x_bytes / 2);
-      const int c0 = (qg & 3) * 2;
-      uint4 u0, u1;
-      asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
-                   : "=r"(u0.x), "=r"(u0.y), "=r"(u0.z), "=r"(u0.w)
-                   : "r"(sw128_chunk(box, qr, c0)));
-      asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
-                   : "=r"(u1.x), "=r"(u1.y), "=r"(u1.z), "=r"(u1.w)
-                   : "r"(sw128_chunk(box, qr, c0 + 1)));
-      const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-      float v[16];
-      if (k0 < p.K) {
-        const float4* il = reinterpret_cast<const float4*>(p.inv_lambda + k0);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4 f = __ldg(il + q);
-          const float fl[4] = {f.x, f.y, f.z, f.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int j = 4 * q + e;
-            const uint32_t bits = (j & 1) ? (w[j >> 1] & 0xFFFF0000u) : (w[j >> 1] << 16);
-            v[j] = __fmul_rn(__uint_as_float(bits), fl[e]);
-          }
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = 0.f;
+        for (int b = 0; b < 4; ++b) tma_load_2d(xs + b * X_BOX, &tmX, kt * BK + 64 * b, m0, bar);
+        if (p.do_lr)   // the stage's L1f^T tile is stored contiguous and pre-swizzled: one bulk copy
+          bulk_load(smem_u32(base + L.l_ring + s * 4 * L.l_box), p.L1t + (size_t)kt * p.r_tot * BK, 4 * L.l_box, bar);
+        bulk_load(smem_u32(base + L.il_ring + s * IL_BYTES), p.inv_lambda + kt * BK, IL_BYTES, bar);
       }
+    }
+  } else if (warp == W_MMA) {
+    // ---------------------------------------------------------------- tensor-core down projection
+    if (p.do_lr && lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, BM);
+      uint32_t started = 0;                          // bit c: chain c has its first product
+      bool ok = true;
+      for (int it = 0; it < nk; ++it) {
+        const int s = it % p.stages;
+        if (!mbar_wait(smem_u32(&full[s]), (it / p.stages) & 1, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int kt = (k_first + it) % nk;
+        const int kvalid = p.K - kt * BK;              // multiple of 64 (may be <= 0 in the pad)
+        const uint32_t xs = smem_u32(base + L.x_ring + s * X_BYTES);
+        const uint32_t ls = smem_u32(base + L.l_ring + s * 4 * L.l_box);
+        for (int j = 0; j < BK / 16; ++j) {
+          if (j * 16 >= kvalid) break;
+          const int box = j >> 2, koff = (j & 3) * 32, c = j % CHAINS;
+          const uint64_t bdesc = desc_k_sw128(xs + box * X_BOX + koff);
+          for (int h = 0; h < halves; ++h)
+            mma_bf16(tmem + (h * CHAINS + c) * BM, desc_k_sw128(ls + box * L.l_box + h * 16384 + koff), bdesc,
+                     idesc, (started >> c) & 1u);
+          started |= 1u << c;
+        }
+        tc_commit(smem_u32(&empty[s]));
+      }
+      if (ok) tc_commit(smem_u32(dfull));
+    }
+  } else if (p.do_quant) {
+    // ---------------------------------------------------------------- quantizers
+    // row qr, 16-column group qg of the stage
+    const int ct = tid - 32 * W_Q0;
+    const int qr = ct >> 4, qg = ct & 15;
+    const int m = m0 + qr;
+    const size_t qx_row_bytes = (size_t)(p.K_pad / 2);
+    for (int it = 0; it < nk; ++it) {
+      const int s = it % p.stages;
+      if (!mbar_wait(smem_u32(&full[s]), (it / p.stages) & 1, abort_flag, p.err)) break;
+      const int kt = (k_first + it) % nk;
+      const int k0 = kt * BK + qg * 16;
+      const uint32_t box = smem_u32(base + L.x_ring + s * X_BYTES) + (qg >> 2) * X_BOX;
+      const int c0 = (qg & 3) * 2;
+      const uint4 u0 = lds128(sw128_chunk(box, qr, c0));
+      const uint4 u1 = lds128(sw128_chunk(box, qr, c0 + 1));
+      const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+      // 1/lambda of this group: chunk q at position 16 q + qg of the permuted
+      // stage copy (zeros past K, where TMA also filled x with zeros)
+      const uint32_t ila = smem_u32(base + L.il_ring + s * IL_BYTES) + qg * 16;
+      float il[16];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 f = lds128(ila + 256 * q);
+        il[4 * q] = __uint_as_float(f.x);
+        il[4 * q + 1] = __uint_as_float(f.y);
+        il[4 * q + 2] = __uint_as_float(f.z);
+        il[4 * q + 3] = __uint_as_float(f.w);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&empty[s]));   // shared-memory reads of stage s are done
+      float v[16];
+#pragma unroll
+      for (int j = 0; j < 16; j += 2)   // bf16 pair -> two floats, times 1/lambda
+        mul2_rn(__uint_as_float(w[j >> 1] << 16), __uint_as_float(w[j >> 1] & 0xFFFF0000u), il[j], il[j + 1],
+                v[j], v[j + 1]);
       uint2 codes;
       if (p.fmt == 0) {
         uint32_t sc;
-        quant_nvfp4_16(v, p.s_t, p.six_st, codes, sc);
-        // four consecutive groups (one 64-k block) of a row -> one 32-bit store
-        const uint32_t s1 = __shfl_down_sync(0xffffffffu, sc, 1);
-        const uint32_t s2 = __shfl_down_sync(0xffffffffu, sc, 2);
-        const uint32_t s3 = __shfl_down_sync(0xffffffffu, sc, 3);
-        if ((qg & 3) == 0) {
-          const uint32_t word = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
-          *reinterpret_cast<uint32_t*>(p.sX + sf_atom_offset(m, k0 / 16, p.K_pad)) = word;
-        }
+        quant_nvfp4_16_tab(v, p.six_st, inv_tab, codes, sc);
+        p.sX[sf_atom_offset(m, k0 / 16, p.K_pad)] = (uint8_t)sc;
       } else {
         __half sc;
         quant_int4_16of64(v, codes, sc);
@@ -180,55 +226,35 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (m < p.M) *reinterpret_cast<uint2*>(p.qX + (size_t)m * qx_row_bytes + k0 / 2) = codes;
     }
-
-    if (p.do_lr) {
-      const int kvalid = min(BK, p.K - kt * BK);   // multiple of 64 (may be <= 0 in the pad)
-      const uint32_t lbase = st + x_bytes;
-#pragma unroll 2
-      for (int j = 0; j < BK / 16; ++j) {
-        if (j * 16 >= kvalid) break;
-        const int half = j >> 2;                       // which 64-column box
-        const int cj = (j & 3) * 2;                    // 16-byte chunk index of this k16 step
-        uint32_t a0, a1, a2, a3;
-        {
-          const int row = mt * 16 + (lane & 15);
-          ldmatrix_x4(sw128_chunk(st + half * (x_bytes / 2), row, cj + (lane >> 4)), a0, a1, a2, a3);
-        }
-#pragma unroll
-        for (int i = 0; i < MAX_PAIRS_PER_WARP; ++i) {
-          const int nt = (warp >> 1) + 4 * i;
-          if (nt < n_tiles) {
-            const int n = nt * 8 + (lane & 7);
-            uint32_t b0, b1;
-            ldmatrix_x2(sw128_chunk(lbase + half * (l_bytes / 2), n, cj + ((lane >> 3) & 1)), b0, b1);
-            mma_16816(acc[i], a0, a1, a2, a3, b0, b1);
-          }
-        }
-      }
-    }
-
-    __syncthreads();                                   // stage s fully consumed
-    if (tid == 0 && kt + p.stages < nk) issue(kt + p.stages);
   }
 
-  if (!ok) return;
-
-  if (p.do_lr) {
-    const int g = lane >> 2, t4 = lane & 3;
+  if (p.do_lr && warp >= W_Q0 && warp < W_Q0 + 4) {
+    // ---------------------------------------------------------------- LR read-out
+    // TMEM lane = rank index r (row of LR^T), column = row n of this CTA's X tile
+    if (mbar_wait(smem_u32(dfull), 0, abort_flag, p.err)) {
+      tc_fence_after();
+      const int sub = warp & 3;
+      for (int h = 0; h < halves; ++h) {
+        float acc[BM];
 #pragma unroll
-    for (int i = 0; i < MAX_PAIRS_PER_WARP; ++i) {
-      const int nt = (warp >> 1) + 4 * i;
-      if (nt < n_tiles) {
-        const int col = nt * 8 + 2 * t4;
-        const int r0 = m0 + mt * 16 + g, r1 = r0 + 8;
-        if (r0 < p.M)
-          *reinterpret_cast<__nv_bfloat162*>(p.LR + (size_t)r0 * p.r_pad + col) =
-              __floats2bfloat162_rn(acc[i][0], acc[i][1]);
-        if (r1 < p.M)
-          *reinterpret_cast<__nv_bfloat162*>(p.LR + (size_t)r1 * p.r_pad + col) =
-              __floats2bfloat162_rn(acc[i][2], acc[i][3]);
+        for (int n = 0; n < BM; ++n) acc[n] = 0.f;
+        for (int c = 0; c < CHAINS; ++c) {               // fixed order: chain 0, 1, 2, 3
+          uint32_t d[32];
+          tmem_ld32(tmem + ((uint32_t)(sub * 32) << 16) + (h * CHAINS + c) * BM, d);
+          tmem_wait_ld();
+#pragma unroll
+          for (int n = 0; n < BM; ++n) acc[n] += __uint_as_float(d[n]);
+        }
+        const int r = 128 * h + 32 * sub + lane;
+        if (r < p.r_tot) {
+#pragma unroll
+          for (int n = 0; n < BM; ++n)
+            if (m0 + n < p.M) p.LR[(size_t)(m0 + n) * p.r_pad + r] = __float2bfloat16_rn(acc[n]);
+        }
       }
     }
+  }
+  if (p.do_lr) {
     // zero padding columns [r_tot, r_pad)
     const int padc = p.r_pad - p.r_tot;
     for (int i = tid; i < BM * padc; i += THREADS) {
@@ -236,26 +262,36 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (r < p.M) p.LR[(size_t)r * p.r_pad + c] = __float2bfloat16(0.f);
     }
   }
+
+  // Every thread reaches this point, also after a timeout (the loops above
+  // leave early when the abort flag is set); TMEM is freed on every path.
+  tc_fence_before();
+  __syncthreads();
+  if (p.do_lr && warp == W_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, tmem_cols);
+  }
 }
 
 size_t quant_down_smem_bytes(int r_tot, bool do_lr, int* stages_out, int nk) {
-  const int stage_bytes = BM * BK * 2 + (do_lr ? r_tot * BK * 2 : 0);
-  int stages = (196 * 1024) / stage_bytes;
-  stages = stages < 2 ? 2 : (stages > 8 ? 8 : stages);
+  const int stage_bytes = X_BYTES + IL_BYTES + (do_lr ? 4 * r_tot * 128 : 0);
+  const int tail = do_lr ? (r_tot > 128 ? 32768 : 16384) : 0;
+  int stages = (200 * 1024 - tail) / stage_bytes;
+  stages = stages < 2 ? 2 : (stages > 6 ? 6 : stages);
   if (stages > nk) stages = nk < 1 ? 1 : nk;
   *stages_out = stages;
-  return (size_t)stages * stage_bytes + 1024 /*alignment slack*/ + 8 * stages + 64;
+  const Layout L = make_layout(stages, r_tot, do_lr);
+  return (size_t)L.bar_off + 1024 /*alignment slack*/ + 8 * (2 * stages + 1) + 16 + 128 * 4 + 64;
 }
 
-cudaError_t launch_quant_down(const CUtensorMap& tmX, const CUtensorMap& tmL1, K1Params p,
-                              cudaStream_t stream) {
+cudaError_t launch_quant_down(const CUtensorMap& tmX, K1Params p, cudaStream_t stream) {
   const int nk = p.K_pad / BK;
   const size_t smem = quant_down_smem_bytes(p.r_tot, p.do_lr != 0, &p.stages, nk);
   cudaError_t e = cudaFuncSetAttribute(quant_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
   const int grid = round_up(p.M, 128) / BM;
-  quant_down_kernel<<<grid, THREADS, smem, stream>>>(tmX, tmL1, p);
+  quant_down_kernel<<<grid, THREADS, smem, stream>>>(tmX, p);
   return cudaGetLastError();
 }
 

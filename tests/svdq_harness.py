@@ -107,6 +107,22 @@ def y_check(Y_gpu: np.ndarray, Y_o: np.ndarray, rel: float = 1e-2):
                 n_over=int(np.sum(diff > rel * rms)), n_bad=int(bad.sum()))
 
 
+def lr_check(lr_gpu, X, L1f):
+    """LR parity: |LR_gpu - LR_oracle| <= one bf16 ulp of LR_oracle plus the
+    float32 dot-product error bound 2 K u sum_k |x_k l_k| (u = 2^-24): the
+    tensor-core sum is float32 in an order of its own, and with the outlier
+    channels its partial sums can be far larger than the result."""
+    X = np.asarray(X, np.float64)
+    L1f = np.asarray(L1f, np.float64)
+    lr_o = F.bf16_round(X @ L1f)
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(lr_o), 1e-38))) - 7)
+    gamma = 2.0 * X.shape[1] * 2.0 ** -24
+    bound = ulp * (1 + 1e-9) + gamma * (np.abs(X) @ np.abs(L1f))
+    err = np.abs(np.asarray(lr_gpu, np.float64) - lr_o)
+    return dict(ok=bool(np.all(err <= bound)), n_beyond_ulp=int(np.sum(err > ulp * (1 + 1e-9))),
+                max_err_over_bound=float(np.max(err / bound)))
+
+
 def assert_y(Y_gpu, Y_o, rel=1e-2):
     r = y_check(Y_gpu, Y_o, rel)
     assert r["n_bad"] == 0, r

@@ -2,7 +2,7 @@
 benchmark times (the same entry points, grids and tile shapes).
 
 Codes, block scales and tensor scales are compared in full; LR in full (one
-bf16 ulp); Y on 193 rows spread over M (the oracle computes those rows one
+bf16 ulp plus the float32 dot-product error bound); Y on 193 rows spread over M (the oracle computes those rows one
 by one in float64) within 1e-2 rms.  Workloads:
   QKV      NVFP4, M=4608, K=3072, N=9216, rank 32
   MLP      NVFP4, fc1 3072 -> 12288 with GELU, fc2 12288 -> 3072 fed with the
@@ -18,7 +18,7 @@ import torch
 import workloads
 from oracle import formats as F
 from oracle import svdquant as S
-from svdq_harness import GpuLayer, assert_y, bf16_np, dev_bf16
+from svdq_harness import GpuLayer, assert_y, bf16_np, dev_bf16, lr_check
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -35,11 +35,6 @@ def sample_rows(M, n=192):
     return np.unique(np.concatenate([np.linspace(0, M - 1, n).astype(np.int64), [M - 1]]))
 
 
-def lr_within_ulp(lr_gpu, lr_o):
-    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(lr_o), 1e-38))) - 7)
-    return bool(np.all(np.abs(lr_gpu - lr_o) <= ulp * (1 + 1e-9)))
-
-
 def check_layer(g, X, gelu=False, check_codes=True, rows=None):
     """Codes of both sides, LR, and Y on sampled rows.  Returns (Y_gpu, stats)."""
     pw, M = g.pw, X.shape[0]
@@ -54,7 +49,8 @@ def check_layer(g, X, gelu=False, check_codes=True, rows=None):
         oq, osc = S.quantize_activation(pw, X)
         assert np.array_equal(q, oq)
         assert np.array_equal(np.asarray(s).view(np.uint8), np.asarray(osc).view(np.uint8))
-        assert lr_within_ulp(lr, S.lowrank_down(X, pw.L1f))
+        lrc = lr_check(lr, X, pw.L1f)
+        assert lrc["ok"], lrc
         assert np.all(lr_pad == 0)
         del qX, sX, LR
     Yd = g.linear(Xd, M, gelu=gelu)
@@ -96,12 +92,20 @@ def test_mlp_pair_full(B):
         try:
             _, r2 = check_layer(g2, Y1_o)
             print("MLP fc2 (oracle input):", r2)
-            # the all-GPU chain against the all-oracle chain, same tolerance
+            # The all-GPU chain against the all-oracle chain.  fc1's outputs
+            # differ by up to one bf16 ulp, which flips some of fc2's input codes
+            # at rounding boundaries (a discontinuous step), so this check bounds
+            # the relative RMS (1%) and the worst element (10% of rms) instead of
+            # the per-element layer tolerance.
             Y2d = g2.linear(Y1d, fc1.M)
             rows = sample_rows(fc1.M)
             Y2_gpu = bf16_np(Y2d[torch.from_numpy(rows).cuda()])
             Y2_o = S.forward(g2.pw, Y1_o[rows])["Y"]
-            print("MLP chain:", assert_y(Y2_gpu, Y2_o))
+            rms = float(np.sqrt(np.mean(Y2_o ** 2)))
+            d = Y2_gpu - Y2_o
+            rel_rms, rel_max = float(np.sqrt(np.mean(d ** 2))) / rms, float(np.max(np.abs(d))) / rms
+            print("MLP chain: rel_rms %.3e rel_max %.3e" % (rel_rms, rel_max))
+            assert rel_rms <= 1e-2 and rel_max <= 0.1
             # fc2 sees non-negative skewed activations (post-GELU): min > -0.2
             assert Y1_o.min() > -0.2
         finally:
