@@ -93,7 +93,7 @@ typedef struct {
   const void* qR;          /* dev uint8 [N_pad][K_pad/2], packed like qX (rows = output features) */
   const void* sR;          /* dev: scales of R laid out like sX, over N_pad rows */
   const void* L1t;         /* dev bf16 (lambda^-1-folded L1 | LoRA A)^T in kernel 1's staged layout:
-                              per 256-wide k stage, four [r_tot x 64] boxes, chunk c of row r at c ^ (r % 8) */
+                              one [r_tot x 64] box per 64-wide k block, in k order; chunk c of row r at c ^ (r % 8) */
   const void* L2a;         /* dev bf16 [N_pad][r_pad]: (L2 ; LoRA B) transposed, divided by alpha */
   const void* bias;        /* dev float32 [N_pad] (zeros if no bias was given) */
   const float* lambda_inv; /* dev float32 [K]: correctly rounded 1/lambda */

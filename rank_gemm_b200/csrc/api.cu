@@ -175,7 +175,7 @@ svdq_status run_k1(const svdq_weights* w, int M, const void* X, void* qX, void* 
   svdq_status s = check_handle_device(w, &d);
   if (s != SVDQ_OK) return s;
   CUtensorMap tmX;
-  if (!tmap_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, w->K, M, (uint64_t)w->K * 2, 64, 32))
+  if (!tmap_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, w->K, M, (uint64_t)w->K * 2, 64, K1_BOX_ROWS))
     return SVDQ_ERR_CUDA;
   return from_cuda(launch_quant_down(tmX, k1_params(w, d, M, qX, sX, LR, do_quant, do_lr), stream));
 }

@@ -17,7 +17,7 @@ struct K1Params {
   int fmt;                 // 0 NVFP4, 1 INT4
   int do_quant, do_lr;     // fused: both; unfused baseline: one of them
   int stages;              // set by the launcher
-  const float* inv_lambda; // [K_pad], permuted per stage (see prepare.cu)
+  const float* inv_lambda; // [K_pad], permuted per 64-wide stage (see prepare.cu)
   const __nv_bfloat16* L1t; // L1f^T in the staged layout (one contiguous tile per stage)
   float s_t, six_st;       // NVFP4 activation tensor scale and fl32(6 s_t)
   uint8_t* qX;             // [M][K_pad/2]
@@ -25,6 +25,9 @@ struct K1Params {
   __nv_bfloat16* LR;       // [M][r_pad]
   DeviceErr err;
 };
+// Kernel 1 stages X in [K1_BOX_ROWS x 64] bf16 TMA boxes (128-byte swizzle);
+// the host encodes tmX with exactly this box.
+constexpr int K1_BOX_ROWS = 64;
 cudaError_t launch_quant_down(const CUtensorMap& tmX, K1Params p, cudaStream_t stream);
 
 // ---------------------------------------------------------------- kernel 2

@@ -160,17 +160,16 @@ __global__ void quantize_weights_kernel(PrepParams p, float s_tR, float six_st) 
 __global__ void factors_kernel(PrepParams p, float alpha) {
   const int tid = blockIdx.x * blockDim.x + threadIdx.x;
   const int stride = gridDim.x * blockDim.x;
-  // L1t = ([L1f | A])^T in kernel 1's staged layout: per 256-wide k stage,
-  // four [r_tot x 64] bf16 boxes, each row's eight 16-byte chunks placed with
-  // the 128-byte swizzle (chunk c of row r at c ^ (r % 8)), zeros for k >= K.
+  // L1t = ([L1f | A])^T in kernel 1's staged layout: per 64-wide k stage one
+  // [r_tot x 64] bf16 box, each row's eight 16-byte chunks placed with the
+  // 128-byte swizzle (chunk c of row r at c ^ (r % 8)), zeros for k >= K.
   for (int i = tid; i < p.r_tot * p.K_pad; i += stride) {
     const int r = i / p.K_pad, k = i % p.K_pad;
     __nv_bfloat16 v = __float2bfloat16(0.f);
     if (k < p.K)
       v = (r < p.rank) ? p.L1f[(size_t)k * p.rank + r] : p.loraA[(size_t)k * p.lora_rank + (r - p.rank)];
-    const int kt = k >> 8, b = (k >> 6) & 3, c = k & 63;
-    const size_t off = (size_t)kt * p.r_tot * 256 + (size_t)b * p.r_tot * 64 + (size_t)r * 64 +
-                       ((((c >> 3) ^ (r & 7)) << 3) | (c & 7));
+    const int kb = k >> 6, c = k & 63;
+    const size_t off = (size_t)kb * p.r_tot * 64 + (size_t)r * 64 + ((((c >> 3) ^ (r & 7)) << 3) | (c & 7));
     p.L1t[off] = v;
   }
   // L2a [N_pad][r_pad] = ([L2 ; B] / alpha)^T, zero padded
@@ -187,12 +186,13 @@ __global__ void factors_kernel(PrepParams p, float alpha) {
   for (int n = tid; n < p.N_pad; n += stride)
     p.bias_f[n] = (n < p.N && p.bias) ? bf(p.bias[n]) : 0.f;
   for (int k = tid; k < p.K; k += stride) p.lambda_inv[k] = __frcp_rn(p.lambda[k]);
-  // kernel 1's copy of 1/lambda, permuted inside every 256-wide stage so that
-  // its quantizer threads (one per 16-column group g) read 16-byte chunk q of
-  // their group from position 16 q + g: conflict-free shared-memory reads
+  // kernel 1's copy of 1/lambda, permuted inside every 64-wide stage so that
+  // its quantizer threads (one per 16-column group g, four adjacent lanes per
+  // row) read 16-byte chunk q of their group from position 4 q + g:
+  // conflict-free shared-memory reads
   for (int k = tid; k < p.K_pad; k += stride) {
-    const int kt = k >> 8, g = (k >> 4) & 15, q = (k >> 2) & 3, e = k & 3;
-    p.lambda_inv_k1[(size_t)kt * 256 + (q * 16 + g) * 4 + e] = (k < p.K) ? __frcp_rn(p.lambda[k]) : 0.f;
+    const int kb = k >> 6, g = (k >> 4) & 3, q = (k >> 2) & 3, e = k & 3;
+    p.lambda_inv_k1[(size_t)kb * 64 + (q * 4 + g) * 4 + e] = (k < p.K) ? __frcp_rn(p.lambda[k]) : 0.f;
   }
 }
 

@@ -3,22 +3,26 @@
 // model card: the Quantize and Down Projection kernels read the same input,
 // so they are fused and X is read from HBM once).
 //
-// One CTA owns 32 rows of X and walks all of K in 256-column stages.  A
-// producer warp keeps a TMA ring of stages in flight; a stage holds the
-// [32 x 256] bf16 tile of X (four 128-byte-swizzled boxes), the matching
-// [r_tot x 256] tile of L1f^T (stored pre-swizzled, one contiguous bulk copy)
-// and the 256 values of 1/lambda.  Each CTA walks
-// the stages starting at its own offset, so the CTAs of a wave read different
-// L1f^T tiles and different X columns at any moment.  From the same staged
-// tile:
+// A cluster of two CTAs owns 64 rows of X; CTA c of the cluster walks the
+// c-th half of K in 128-column stages.  A producer warp keeps a TMA ring of
+// stages in flight; a stage holds the [64 x 128] bf16 tile of X (two
+// 128-byte-swizzled [64 x 64] boxes), the matching [r_tot x 128] tile of
+// L1f^T (stored pre-swizzled, one contiguous bulk copy) and the 128 values of
+// 1/lambda.
+// From the same staged tile:
 //   * 16 quantizer warps: every thread one 16-element group of one row
 //     (x^ = x / lambda, amax, block scale, 4-bit codes), written packed with
 //     scales in the layout kernel 2's tensor-core MMA consumes;
-//   * one thread issues the down projection on the 5th-generation tensor core
-//     as the transposed product LR^T = L1f^T X^T: A = the L1f^T tile (128 rows
-//     per MMA, rows past r_tot are ignored), B = the staged X tile itself
-//     (N = 32 rows), fp32 accumulation in a 32-column TMEM tile across all of
-//     K; four warps read it out at the end and store LR in bf16.
+//   * one thread issues the down projection on the 5th-generation tensor core:
+//     A = the staged X tile (M = 64 rows), B = the L1f^T tile (N = r_tot),
+//     fp32 accumulation in TMEM across the CTA's half of K.
+// At the end four warps move the partial [64 x r_tot] tile from TMEM to
+// shared memory; after a cluster barrier CTA c adds the two partials of rows
+// [32c, 32c + 32) through distributed shared memory, always in the order
+// CTA 0, 1 (so LR is the same on every run), and stores LR in bf16.
+// Why 64 rows and two CTAs: the four-way split of a 128-row tile needs
+// clusters of four, and at one CTA per SM only 33 of those are resident at
+// once on 148 SMs; clusters of two fill every SM.
 // Stages are released through an mbarrier (the 16 quantizer warps plus the
 // MMA commit) instead of a CTA-wide sync, so warps drift apart and overlap
 // their load, math and store phases.  The kernel is HBM-bound: per row it
@@ -31,20 +35,34 @@ namespace svdq {
 
 namespace {
 
-constexpr int BM = 32;                       // rows per CTA (= MMA N)
-constexpr int BK = 256;                      // K columns per stage (four 64-column TMA boxes)
-constexpr int QWARPS = 16;                   // quantizer warps
+constexpr int BM = K1_BOX_ROWS;              // rows per cluster (= MMA M = TMA box rows)
+constexpr int BK = 128;                      // K columns per stage (two 64-column swizzled boxes)
+constexpr int KSPLIT = 2;                    // CTAs per cluster, each half of K
+constexpr int QWARPS = 16;                   // quantizer warps: 64 rows x 8 groups
 constexpr int THREADS = 32 * (QWARPS + 2);   // + producer warp + MMA warp
-constexpr int X_BOX = BM * 128;              // one [32 x 64] bf16 box
-constexpr int X_BYTES = 4 * X_BOX;           // 16 KB
+constexpr int X_BOX = BM * 128;              // one [64 x 64] bf16 box, 8 KB
+constexpr int X_BYTES = 2 * X_BOX;           // 16 KB
 constexpr int IL_BYTES = BK * 4;             // 1/lambda for the stage
 constexpr int W_PROD = 0, W_MMA = 1, W_Q0 = 2;
-constexpr int CHAINS = 1;                     // LR accumulators (interleaved k16 steps)
+constexpr int MAX_STAGES = 8;
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 u;
   asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w) : "r"(addr));
   return u;
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+__device__ __forceinline__ float4 dsmem_ld_f32x4(uint32_t cluster_addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(cluster_addr)
+               : "memory");
+  return v;
 }
 
 // Address of the 16-byte chunk holding columns [8c, 8c+8) of row `row` in a
@@ -53,23 +71,33 @@ __device__ __forceinline__ uint32_t sw128_chunk(uint32_t box_base, int row, int 
   return box_base + row * 128 + ((c ^ (row & 7)) << 4);
 }
 
+// Row stride (floats) of the partial LR tile in shared memory: a multiple of
+// 4 (16-byte rows) that is 4 or 20 mod 32, so the 16-byte writes of 8
+// consecutive rows hit 8 different bank quads.
+__host__ __device__ constexpr int part_stride(int r_tot) { return r_tot + 4; }
+
 struct Layout {
-  int stages, l_box, x_ring, il_ring, l_ring, bar_off;
+  int stages, l_bytes, x_ring, l_ring, il_ring, bar_off;
 };
 
-// Shared memory: X ring | 1/lambda ring | L1f^T boxes (compact) + a tail so
-// an M = 128 MMA reading past the last box stays inside the allocation |
-// barriers.
+// Shared memory: X ring | L1f^T ring | 1/lambda ring | barriers.  The partial
+// LR tile reuses the start of the ring once every stage has been consumed.
 __host__ __device__ inline Layout make_layout(int stages, int r_tot, bool do_lr) {
   Layout L;
   L.stages = stages;
-  L.l_box = do_lr ? r_tot * 128 : 0;
+  L.l_bytes = do_lr ? 2 * r_tot * 128 : 0;  // r_tot % 16 == 0: 2 KB multiples keep the 1 KB swizzle atoms aligned
   L.x_ring = 0;
-  L.il_ring = stages * X_BYTES;
-  L.l_ring = L.il_ring + stages * IL_BYTES;
-  const int tail = do_lr ? (r_tot > 128 ? 32768 : 16384) : 0;
-  L.bar_off = L.l_ring + stages * 4 * L.l_box + tail;
+  L.l_ring = stages * X_BYTES;
+  L.il_ring = L.l_ring + stages * L.l_bytes;
+  int end = L.il_ring + stages * IL_BYTES;
+  const int part = do_lr ? BM * part_stride(r_tot) * 4 : 0;
+  if (part > end) end = part;
+  L.bar_off = round_up(end, 16);
   return L;
+}
+
+__host__ __device__ constexpr uint32_t tmem_cols_for(int r_tot) {
+  return r_tot <= 32 ? 32u : r_tot <= 64 ? 64u : r_tot <= 128 ? 128u : 256u;
 }
 
 }  // namespace
@@ -78,22 +106,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     quant_down_kernel(const __grid_constant__ CUtensorMap tmX, K1Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int m0 = blockIdx.x * BM;
-
-  // CTAs past the last activation row only clear the scale rows that pad the
-  // last 128-row scale-factor block.
-  if (m0 >= p.M) {
-    if (!p.do_quant) return;
-    const int ngroups = p.K_pad / 16;
-    for (int i = tid; i < BM * ngroups; i += THREADS) {
-      const int r = m0 + i / ngroups, g = i % ngroups;
-      if (p.fmt == 0)
-        p.sX[sf_atom_offset(r, g, p.K_pad)] = 0;
-      else if ((g & 3) == 0)
-        reinterpret_cast<__half*>(p.sX)[int4_scale_offset(r, g / 4, p.K_pad)] = __float2half(0.f);
-    }
-    return;
-  }
+  // half of K; with the low-rank branch the two CTAs of a row block form a
+  // cluster, and the cluster rank equals this index
+  const int split = blockIdx.x % KSPLIT;
+  const int m0 = (blockIdx.x / KSPLIT) * BM;
+  const int ns = p.K_pad / BK / KSPLIT;                  // stages per CTA (K_pad % 256 == 0)
+  const int kb0 = split * ns;                            // first 128-column block of this CTA
 
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const Layout L = make_layout(p.stages, p.r_tot, p.do_lr != 0);
@@ -103,14 +121,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(dfull + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* inv_tab = reinterpret_cast<float*>(tmem_slot + 4);        // 128 entries, NVFP4 only
-  // LR accumulates in CHAINS independent TMEM tiles (k16 step j goes to chain
-  // j % CHAINS) so consecutive MMAs do not wait on each other's result; per
-  // 128-row half of L1f^T: CHAINS x 32 columns
-  const int halves = p.r_tot > 128 ? 2 : 1;
-  const uint32_t tmem_cols = (uint32_t)(halves * CHAINS * BM);
+  const uint32_t tmem_cols = tmem_cols_for(p.r_tot);
 
-  const int nk = p.K_pad / BK;
-  const int k_first = blockIdx.x % nk;                   // this CTA's first stage
   if (tid == 0) {
     tma_prefetch_desc(&tmX);
     for (int s = 0; s < p.stages; ++s) {
@@ -134,45 +146,42 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == W_PROD) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
-      for (int it = 0; it < nk; ++it) {
+      for (int it = 0; it < ns; ++it) {
         const int s = it % p.stages;
         if (!mbar_wait(smem_u32(&empty[s]), ((it / p.stages) & 1) ^ 1, abort_flag, p.err)) break;
-        const int kt = (k_first + it) % nk;
+        const int kb = kb0 + it;
         const uint32_t bar = smem_u32(&full[s]);
-        mbar_arrive_expect_tx(bar, X_BYTES + 4 * L.l_box + IL_BYTES);
-        const uint32_t xs = smem_u32(base + L.x_ring + s * X_BYTES);
-#pragma unroll
-        for (int b = 0; b < 4; ++b) tma_load_2d(xs + b * X_BOX, &tmX, kt * BK + 64 * b, m0, bar);
+        mbar_arrive_expect_tx(bar, X_BYTES + L.l_bytes + IL_BYTES);
+        tma_load_2d(smem_u32(base + L.x_ring + s * X_BYTES), &tmX, kb * BK, m0, bar);
+        tma_load_2d(smem_u32(base + L.x_ring + s * X_BYTES + X_BOX), &tmX, kb * BK + 64, m0, bar);
         if (p.do_lr)   // the stage's L1f^T tile is stored contiguous and pre-swizzled: one bulk copy
-          bulk_load(smem_u32(base + L.l_ring + s * 4 * L.l_box), p.L1t + (size_t)kt * p.r_tot * BK, 4 * L.l_box, bar);
-        bulk_load(smem_u32(base + L.il_ring + s * IL_BYTES), p.inv_lambda + kt * BK, IL_BYTES, bar);
+          bulk_load(smem_u32(base + L.l_ring + s * L.l_bytes), p.L1t + (size_t)kb * p.r_tot * BK, L.l_bytes, bar);
+        bulk_load(smem_u32(base + L.il_ring + s * IL_BYTES), p.inv_lambda + kb * BK, IL_BYTES, bar);
       }
     }
   } else if (warp == W_MMA) {
     // ---------------------------------------------------------------- tensor-core down projection
     if (p.do_lr && lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, BM);
-      uint32_t started = 0;                          // bit c: chain c has its first product
+      const uint32_t idesc = idesc_bf16_f32(BM, p.r_tot);
+      uint32_t started = 0;
       bool ok = true;
-      for (int it = 0; it < nk; ++it) {
+      for (int it = 0; it < ns; ++it) {
         const int s = it % p.stages;
         if (!mbar_wait(smem_u32(&full[s]), (it / p.stages) & 1, abort_flag, p.err)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const int kt = (k_first + it) % nk;
-        const int kvalid = p.K - kt * BK;              // multiple of 64 (may be <= 0 in the pad)
+        const int kvalid = p.K - (kb0 + it) * BK;      // multiple of 64 (may be <= 0 in the pad)
         const uint32_t xs = smem_u32(base + L.x_ring + s * X_BYTES);
-        const uint32_t ls = smem_u32(base + L.l_ring + s * 4 * L.l_box);
+        const uint32_t ls = smem_u32(base + L.l_ring + s * L.l_bytes);
+#pragma unroll
         for (int j = 0; j < BK / 16; ++j) {
           if (j * 16 >= kvalid) break;
-          const int box = j >> 2, koff = (j & 3) * 32, c = j % CHAINS;
-          const uint64_t bdesc = desc_k_sw128(xs + box * X_BOX + koff);
-          for (int h = 0; h < halves; ++h)
-            mma_bf16(tmem + (h * CHAINS + c) * BM, desc_k_sw128(ls + box * L.l_box + h * 16384 + koff), bdesc,
-                     idesc, (started >> c) & 1u);
-          started |= 1u << c;
+          const int b = j >> 2, koff = (j & 3) * 32;
+          mma_bf16(tmem, desc_k_sw128(xs + b * X_BOX + koff), desc_k_sw128(ls + b * p.r_tot * 128 + koff), idesc,
+                   started);
+          started = 1u;
         }
         tc_commit(smem_u32(&empty[s]));
       }
@@ -180,28 +189,28 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (p.do_quant) {
     // ---------------------------------------------------------------- quantizers
-    // row qr, 16-column group qg of the stage
-    const int ct = tid - 32 * W_Q0;
-    const int qr = ct >> 4, qg = ct & 15;
+    // box qb, row qr, 16-column group qg of the stage: a warp covers 8 rows
+    // of one box (conflict-free swizzled reads), the four groups of a row
+    // sit in one quad of lanes
+    const int qw = warp - W_Q0;
+    const int qb = qw & 1, qr = (qw >> 1) * 8 + (lane >> 2), qg = lane & 3;
     const int m = m0 + qr;
     const size_t qx_row_bytes = (size_t)(p.K_pad / 2);
-    for (int it = 0; it < nk; ++it) {
+    for (int it = 0; it < ns; ++it) {
       const int s = it % p.stages;
       if (!mbar_wait(smem_u32(&full[s]), (it / p.stages) & 1, abort_flag, p.err)) break;
-      const int kt = (k_first + it) % nk;
-      const int k0 = kt * BK + qg * 16;
-      const uint32_t box = smem_u32(base + L.x_ring + s * X_BYTES) + (qg >> 2) * X_BOX;
-      const int c0 = (qg & 3) * 2;
-      const uint4 u0 = lds128(sw128_chunk(box, qr, c0));
-      const uint4 u1 = lds128(sw128_chunk(box, qr, c0 + 1));
+      const int kb = 2 * (kb0 + it) + qb;                // 64-column block
+      const uint32_t box = smem_u32(base + L.x_ring + s * X_BYTES + qb * X_BOX);
+      const uint4 u0 = lds128(sw128_chunk(box, qr, 2 * qg));
+      const uint4 u1 = lds128(sw128_chunk(box, qr, 2 * qg + 1));
       const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-      // 1/lambda of this group: chunk q at position 16 q + qg of the permuted
+      // 1/lambda of this group: chunk q at position 4 q + qg of the permuted
       // stage copy (zeros past K, where TMA also filled x with zeros)
-      const uint32_t ila = smem_u32(base + L.il_ring + s * IL_BYTES) + qg * 16;
+      const uint32_t ila = smem_u32(base + L.il_ring + s * IL_BYTES) + qb * 256 + qg * 16;
       float il[16];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const uint4 f = lds128(ila + 256 * q);
+        const uint4 f = lds128(ila + 64 * q);
         il[4 * q] = __uint_as_float(f.x);
         il[4 * q + 1] = __uint_as_float(f.y);
         il[4 * q + 2] = __uint_as_float(f.z);
@@ -218,49 +227,77 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (p.fmt == 0) {
         uint32_t sc;
         quant_nvfp4_16_tab(v, p.six_st, inv_tab, codes, sc);
-        p.sX[sf_atom_offset(m, k0 / 16, p.K_pad)] = (uint8_t)sc;
+        // the row's four scale bytes are adjacent in the scale atom: one word
+        uint32_t sw = sc << (8 * qg);
+        sw |= __shfl_xor_sync(0xffffffffu, sw, 1);
+        sw |= __shfl_xor_sync(0xffffffffu, sw, 2);
+        if (qg == 0) *reinterpret_cast<uint32_t*>(p.sX + sf_atom_offset(m, kb * 4, p.K_pad)) = sw;
       } else {
         __half sc;
         quant_int4_16of64(v, codes, sc);
-        if ((qg & 3) == 0) reinterpret_cast<__half*>(p.sX)[int4_scale_offset(m, k0 / 64, p.K_pad)] = sc;
+        if (qg == 0) reinterpret_cast<__half*>(p.sX)[int4_scale_offset(m, kb, p.K_pad)] = sc;
       }
-      if (m < p.M) *reinterpret_cast<uint2*>(p.qX + (size_t)m * qx_row_bytes + k0 / 2) = codes;
+      if (m < p.M) *reinterpret_cast<uint2*>(p.qX + (size_t)m * qx_row_bytes + (size_t)kb * 32 + qg * 8) = codes;
     }
   }
 
-  if (p.do_lr && warp >= W_Q0 && warp < W_Q0 + 4) {
-    // ---------------------------------------------------------------- LR read-out
-    // TMEM lane = rank index r (row of LR^T), column = row n of this CTA's X tile
-    if (mbar_wait(smem_u32(dfull), 0, abort_flag, p.err)) {
-      tc_fence_after();
-      const int sub = warp & 3;
-      for (int h = 0; h < halves; ++h) {
-        float acc[BM];
-#pragma unroll
-        for (int n = 0; n < BM; ++n) acc[n] = 0.f;
-        for (int c = 0; c < CHAINS; ++c) {               // fixed order: chain 0, 1, 2, 3
+  // All stages are consumed (or a wait gave up): the ring can hold the partial tile.
+  tc_fence_before();
+  __syncthreads();
+  if (p.do_lr) {
+    const int ps = part_stride(p.r_tot);
+    const uint32_t part = smem_u32(base);
+    if (warp >= W_Q0 && warp < W_Q0 + 4) {
+      // ---------------------------------------------------------------- TMEM -> shared partial
+      // M = 64 accumulator: row i in TMEM lane 32 (i / 16) + i % 16, column =
+      // rank index; lanes 16-31 of each sub-partition are unused
+      const int sub = warp & 3, row = 16 * sub + lane;
+      const bool has_mma = kb0 * BK < p.K;               // else this half lies in the K pad: zeros
+      if (mbar_wait(smem_u32(dfull), 0, abort_flag, p.err)) {
+        tc_fence_after();
+        for (int c0 = 0; c0 < p.r_tot; c0 += 32) {
           uint32_t d[32];
-          tmem_ld32(tmem + ((uint32_t)(sub * 32) << 16) + (h * CHAINS + c) * BM, d);
-          tmem_wait_ld();
+          if (has_mma) {
+            tmem_ld32(tmem + ((uint32_t)(sub * 32) << 16) + (uint32_t)c0, d);
+            tmem_wait_ld();
+          } else {
 #pragma unroll
-          for (int n = 0; n < BM; ++n) acc[n] += __uint_as_float(d[n]);
-        }
-        const int r = 128 * h + 32 * sub + lane;
-        if (r < p.r_tot) {
+            for (int n = 0; n < 32; ++n) d[n] = 0u;
+          }
 #pragma unroll
-          for (int n = 0; n < BM; ++n)
-            if (m0 + n < p.M) p.LR[(size_t)(m0 + n) * p.r_pad + r] = __float2bfloat16_rn(acc[n]);
+          for (int n = 0; n < 32; n += 4)
+            if (lane < 16 && c0 + n < p.r_tot) sts128(part + (uint32_t)(row * ps + c0 + n) * 4, d[n], d[n + 1], d[n + 2], d[n + 3]);
         }
       }
     }
-  }
-  if (p.do_lr) {
-    // zero padding columns [r_tot, r_pad)
-    const int padc = p.r_pad - p.r_tot;
-    for (int i = tid; i < BM * padc; i += THREADS) {
-      const int r = m0 + i / padc, c = p.r_tot + i % padc;
-      if (r < p.M) p.LR[(size_t)r * p.r_pad + c] = __float2bfloat16(0.f);
+    cluster_sync_all();
+    // ---------------------------------------------------------------- cluster reduction
+    // this CTA's 32 rows; four consecutive columns per task; pad columns -> 0
+    const int rows_per = BM / KSPLIT, quads = p.r_pad / 4;
+    for (int i = tid; i < rows_per * quads; i += THREADS) {
+      const int rr = split * rows_per + i / quads, c = (i % quads) * 4;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (c < p.r_tot) {
+        const uint32_t a = part + (uint32_t)(rr * ps + c) * 4;
+#pragma unroll
+        for (int q = 0; q < KSPLIT; ++q) {   // fixed order: CTA 0, 1
+          const float4 v = dsmem_ld_f32x4(dsmem_map(a, (uint32_t)q));
+          acc.x += v.x;
+          acc.y += v.y;
+          acc.z += v.z;
+          acc.w += v.w;
+        }
+      }
+      const int m = m0 + rr;
+      if (m < p.M) {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+        uint2 pk;
+        pk.x = *reinterpret_cast<uint32_t*>(&lo);
+        pk.y = *reinterpret_cast<uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(p.LR + (size_t)m * p.r_pad + c) = pk;
+      }
     }
+    cluster_sync_all();   // no CTA leaves while another still reads its partial
   }
 
   // Every thread reaches this point, also after a timeout (the loops above
@@ -273,26 +310,37 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-size_t quant_down_smem_bytes(int r_tot, bool do_lr, int* stages_out, int nk) {
-  const int stage_bytes = X_BYTES + IL_BYTES + (do_lr ? 4 * r_tot * 128 : 0);
-  const int tail = do_lr ? (r_tot > 128 ? 32768 : 16384) : 0;
-  int stages = (200 * 1024 - tail) / stage_bytes;
-  stages = stages < 2 ? 2 : (stages > 6 ? 6 : stages);
-  if (stages > nk) stages = nk < 1 ? 1 : nk;
+size_t quant_down_smem_bytes(int r_tot, bool do_lr, int* stages_out, int ns) {
+  const int stage_bytes = X_BYTES + IL_BYTES + (do_lr ? 2 * r_tot * 128 : 0);
+  int stages = (200 * 1024) / stage_bytes;
+  stages = stages < 2 ? 2 : (stages > MAX_STAGES ? MAX_STAGES : stages);
+  if (stages > ns) stages = ns < 1 ? 1 : ns;
   *stages_out = stages;
   const Layout L = make_layout(stages, r_tot, do_lr);
   return (size_t)L.bar_off + 1024 /*alignment slack*/ + 8 * (2 * stages + 1) + 16 + 128 * 4 + 64;
 }
 
 cudaError_t launch_quant_down(const CUtensorMap& tmX, K1Params p, cudaStream_t stream) {
-  const int nk = p.K_pad / BK;
-  const size_t smem = quant_down_smem_bytes(p.r_tot, p.do_lr != 0, &p.stages, nk);
+  const int ns = p.K_pad / BK / KSPLIT;
+  const size_t smem = quant_down_smem_bytes(p.r_tot, p.do_lr != 0, &p.stages, ns);
   cudaError_t e = cudaFuncSetAttribute(quant_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  const int grid = round_up(p.M, 128) / BM;
-  quant_down_kernel<<<grid, THREADS, smem, stream>>>(tmX, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  // row blocks up to the next multiple of 128, so that every row of the last
+  // 128-row scale block gets its (zero) scales
+  cfg.gridDim = dim3((unsigned)(KSPLIT * (round_up(p.M, 128) / BM)));
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = KSPLIT;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = p.do_lr ? 1 : 0;   // only the LR reduction needs the cluster
+  return cudaLaunchKernelEx(&cfg, quant_down_kernel, tmX, p);
 }
 
 }  // namespace svdq
