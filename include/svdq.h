@@ -43,11 +43,15 @@
  *   r_pad = r_tot rounded up to a multiple of 64.
  *   qX    uint8 [M][K_pad/2]: two 4-bit codes per byte, even k in the low
  *         nibble; columns k >= K hold code 0.
- *   sX    NVFP4: E4M3 block scales (one per 16 k) in tcgen05 scale-factor
- *         atoms: atom (i, j) for rows 128i..128i+127 and k in [64j, 64j+64)
- *         is 512 contiguous bytes at ((i * K_pad/64) + j) * 512; inside it
- *         the scale of row r and 16-group g (0..3) sits at byte
- *         (r % 32) * 16 + ((r % 128) / 32) * 4 + g.  Rows >= M hold 0.
+ *   sX    NVFP4: E4M3 block scales (one per 16 k), each stored four times
+ *         (once per tensor-memory sub-partition, the form kernel 2 copies
+ *         into tensor memory): the scale of row r and 16-group g (0..3) of
+ *         the 64-column block kb sits at byte
+ *           ((((r / 128) * (K_pad/256) + kb / 4) * 2 + (kb % 4) / 2) * 4096
+ *           + (L / 8) * 256 + (kb % 2) * 128 + (L % 8) * 16
+ *           + ((r % 128) / 32) * 4 + g
+ *         for each replica L = r % 32 + 32 q, q = 0..3.  4 * M_128 * K_pad/16
+ *         bytes (M_128 = M rounded up to 128); rows >= M hold 0.
  *         INT4: binary16 block scales (one per 64 k) in 512-byte chunks of
  *         128 rows x 2 groups: the scale of row r and 64-group g sits at
  *         element (((r / 128) * (K_pad/128) + g / 2) * 2 + g % 2) * 128 + r % 128;
@@ -91,7 +95,10 @@ typedef struct {
   int K, N, rank, lora_rank, r_tot;
   int K_pad, N_pad, r_pad; /* N_pad = N rounded up to a multiple of 256 */
   const void* qR;          /* dev uint8 [N_pad][K_pad/2], packed like qX (rows = output features) */
-  const void* sR;          /* dev: scales of R laid out like sX, over N_pad rows */
+  const void* sR;          /* dev: scales of R, one copy each (NVFP4: 512-byte atoms
+                              of 128 rows x 64 k at ((n/128) * (K_pad/64) + k/64) * 512,
+                              byte (n % 32) * 16 + ((n % 128) / 32) * 4 + (k % 64) / 16;
+                              INT4: laid out like sX), over N_pad rows */
   const void* L1t;         /* dev bf16 (lambda^-1-folded L1 | LoRA A)^T in kernel 1's staged layout:
                               one [r_tot x 64] box per 64-wide k block, in k order; chunk c of row r at c ^ (r % 8) */
   const void* L2a;         /* dev bf16 [N_pad][r_pad]: (L2 ; LoRA B) transposed, divided by alpha */

@@ -28,6 +28,7 @@ struct svdq_weights {
   int K, N, rank, lora_rank, r_tot, K_pad, N_pad, r_pad;
   uint8_t* qR;
   uint8_t* sR;
+  uint8_t* sR_rep;   // NVFP4: kernel 2's replicated copy of sR
   __nv_bfloat16* L1t;
   __nv_bfloat16* L2a;
   float* bias_f;
@@ -134,7 +135,8 @@ bool tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t i
 size_t qx_bytes(const svdq_weights* w, int M) { return (size_t)M * (w->K_pad / 2); }
 size_t sx_bytes(const svdq_weights* w, int M) {
   const size_t rows = (size_t)round_up(M, 128);
-  return w->fmt == SVDQ_NVFP4 ? rows * (w->K_pad / 16) : rows * (w->K_pad / 64) * 2;
+  // NVFP4: four replicas of every scale word (see sfx_rep_offset)
+  return w->fmt == SVDQ_NVFP4 ? rows * (w->K_pad / 16) * 4 : rows * (w->K_pad / 64) * 2;
 }
 size_t lr_bytes(const svdq_weights* w, int M) { return (size_t)M * w->r_pad * 2; }
 
@@ -207,7 +209,7 @@ svdq_status run_k2(const svdq_weights* w, int M, const void* qX, const void* sX,
     p.nk = w->K_pad / 256;
     p.nl = lowrank ? w->r_pad / 64 : 0;
     p.sX = static_cast<const uint8_t*>(sX);
-    p.sR = w->sR;
+    p.sR = w->sR_rep;
     p.bias = w->bias_f;
     p.alpha = w->alpha;
     p.epi = (int)epi;
@@ -242,6 +244,7 @@ svdq_status run_k2(const svdq_weights* w, int M, const void* qX, const void* sX,
 void free_buffers(svdq_weights* w) {
   cudaFree(w->qR);
   cudaFree(w->sR);
+  cudaFree(w->sR_rep);
   cudaFree(w->L1t);
   cudaFree(w->L2a);
   cudaFree(w->bias_f);
@@ -330,6 +333,7 @@ svdq_status svdq_prepare_weights(svdq_format fmt, int K, int N, int rank, const 
   float* R = nullptr;
   unsigned* amax = nullptr;
   bool ok = cudaMalloc(&w->qR, qr_b) == cudaSuccess && cudaMalloc(&w->sR, sr_b) == cudaSuccess &&
+            (fmt != SVDQ_NVFP4 || cudaMalloc(&w->sR_rep, 4 * sr_b) == cudaSuccess) &&
             cudaMalloc(&w->L1t, (size_t)r_tot * w->K_pad * 2) == cudaSuccess &&
             cudaMalloc(&w->L2a, (size_t)w->N_pad * w->r_pad * 2) == cudaSuccess &&
             cudaMalloc(&w->bias_f, (size_t)w->N_pad * 4) == cudaSuccess &&
@@ -365,6 +369,7 @@ svdq_status svdq_prepare_weights(svdq_format fmt, int K, int N, int rank, const 
   p.amax_bits = amax;
   p.qR = w->qR;
   p.sR = w->sR;
+  p.sR_rep = w->sR_rep;
   p.L1t = w->L1t;
   p.L2a = w->L2a;
   p.bias_f = w->bias_f;

@@ -40,6 +40,12 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 u;
+  asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w) : "r"(addr));
+  return u;
+}
+
 // ----------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
@@ -234,6 +240,12 @@ __device__ __forceinline__ void tmem_cp_sf_atom(uint32_t taddr, uint32_t smem_ad
                : "memory");
 }
 
+// One 4 KB replicated scale block (see sfx_rep_offset) -> 8 TMEM columns of all 128 lanes.
+__device__ __forceinline__ void tmem_cp_sf_block(uint32_t taddr, uint32_t smem_addr) {
+  const uint64_t d = smem_desc(smem_addr, 128, 256, 0);
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(d) : "memory");
+}
+
 // 32 lanes x 32 consecutive 32-bit columns -> 32 registers per thread.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
@@ -250,6 +262,95 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+
+// 16 consecutive 32-bit columns of this warp's 32 TMEM lanes <- 16 registers per thread.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Per-warpgroup register budget change (every warp of the warpgroup runs it).
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// ----------------------------------------------------------------- CTA pairs (cta_group::2)
+// Two CTAs of a cluster (ranks 2i, 2i+1) run one MMA over both SMs: A rows
+// and B rows come half from each CTA's shared memory (same offsets), D rows
+// 0-127 land in the even CTA's TMEM and 128-255 in the odd CTA's.  TMA loads
+// of both CTAs complete on the even CTA's mbarrier (`bar` is a
+// shared::cluster address, see dsmem_map).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* tmap, int x, int y,
+                                                 uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(bar_cluster)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+// Arrives once on the barrier at offset `bar` in every CTA of `cta_mask` when
+// the tcgen05 operations this thread issued before have completed.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          bar),
+      "h"(cta_mask)
+      : "memory");
+}
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_nvf4_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                              uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], "
+      "p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+// tmem_cp_sf_atom for the pair: each CTA's atom at `smem_addr` goes to its own TMEM.
+__device__ __forceinline__ void tmem_cp_sf_atom_pair(uint32_t taddr, uint32_t smem_addr) {
+  const uint64_t d = smem_desc(smem_addr, 0, 128, 0);
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d)
+               : "memory");
+}
+// Arrive on an mbarrier of another CTA of the cluster (shared::cluster address).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+
 
 // ----------------------------------------------------------------- conversions
 // Eight floats -> eight E2M1 codes in one word (element j in bits 4j..4j+3),
@@ -391,6 +492,31 @@ __host__ __device__ __forceinline__ size_t sf_atom_offset(int row, int g16, int 
   const int rb = row >> 7, kb = g16 >> 2;
   return ((size_t)rb * (kpad >> 6) + kb) * 512 + (size_t)(row & 31) * 16 + ((row & 127) >> 5) * 4 +
          (g16 & 3);
+}
+
+// NVFP4 scales as kernel 2 moves them into TMEM: 4 KB blocks, each the
+// source of one tcgen05.cp.128x256b (128 lanes x 32 bytes, canonical
+// no-swizzle K-major form: 8-lane groups 256 bytes apart, the two 16-byte
+// halves of a lane 128 bytes apart).  Lane L carries row L % 32 of two scale
+// atoms (each the 16 bytes of rows r, r+32, r+64, r+96 x 4 groups), so all
+// four TMEM sub-partitions receive every atom, as the block-scaled MMA reads
+// them.  One copy per 8 TMEM columns instead of one per 4: the scale copies
+// cost per instruction.
+//   activations: per (128-row block, 256-wide k-tile) two blocks; block j
+//     holds 64-k blocks 2j (first half) and 2j+1 (second half);
+//   weights: per (256-row block, 256-wide k-tile) four blocks; block kb holds
+//     64-k block kb of rows 0-127 (first half) and of rows 128-255 (second).
+// These return the byte offset of the word with the four scales of (row, 64-k
+// block kb) in replica q (0..3).
+__host__ __device__ __forceinline__ size_t sfx_rep_offset(int row, int kb, int q, int kpad) {
+  const int rb = row >> 7, r = row & 127, kt = kb >> 2, kin = kb & 3, lane = (r & 31) + 32 * q;
+  return (((size_t)rb * (kpad >> 8) + kt) * 2 + (kin >> 1)) * 4096 + (size_t)(lane >> 3) * 256 + (kin & 1) * 128 +
+         (lane & 7) * 16 + (r >> 5) * 4;
+}
+__host__ __device__ __forceinline__ size_t sfw_rep_offset(int row, int kb, int q, int kpad) {
+  const int nb = row >> 8, h = (row >> 7) & 1, r = row & 127, kt = kb >> 2, kin = kb & 3, lane = (r & 31) + 32 * q;
+  return (((size_t)nb * (kpad >> 8) + kt) * 4 + kin) * 4096 + (size_t)(lane >> 3) * 256 + h * 128 + (lane & 7) * 16 +
+         (r >> 5) * 4;
 }
 
 // Element offset of (row, 64-group) in the INT4 binary16 scale layout:

@@ -7,13 +7,17 @@
 // Persistent, warp-specialized, one 128 x 256 output tile per CTA at a time:
 //   warp 0      TMA producer: per 256-wide k-tile, the [128 x 128 B] tile of qX,
 //               the [256 x 128 B] tile of qR (both 128-byte swizzled) and the
-//               2 + 4 KB of E4M3 scale atoms (plain bulk copies); then, per
+//               8 + 16 KB of E4M3 scales in their replicated layout (plain
+//               bulk copies); then, per
 //               64-wide chunk of the low-rank dimension, the [128 x 64] bf16 tile
 //               of LR and the [256 x 64] bf16 tile of L2/alpha, into the same
 //               ring slots (a bf16 tile of 64 columns has the byte shape of an
 //               FP4 tile of 256 columns).
-//   warp 1      TMEM owner and single-thread MMA issuer: tcgen05.cp moves the
-//               scale atoms to TMEM, tcgen05.mma.kind::mxf4nvf4 (block16,
+//   warp 1      TMEM owner and single-thread MMA issuer: six
+//               tcgen05.cp.128x256b move a k-tile's scales to TMEM (the copies
+//               cost per instruction, so the scales are stored pre-replicated
+//               for the four TMEM sub-partitions and moved 8 columns at a
+//               time), tcgen05.mma.kind::mxf4nvf4 (block16,
 //               E4M3 scales) accumulates Q(X^) Q(R) in a 128 x 256 fp32 TMEM
 //               tile, then tcgen05.mma.kind::f16 adds LR (L2/alpha) into the
 //               same tile; tcgen05.commit releases ring slots and hands the
@@ -30,12 +34,13 @@ namespace svdq {
 
 namespace {
 
-constexpr int BLOCK_M = 128, BLOCK_N = 256, STAGES = 4;
+constexpr int BLOCK_M = 128, BLOCK_N = 256, STAGES = 3;
 constexpr int A_BYTES = BLOCK_M * 128;          // 16 KB
 constexpr int B_BYTES = BLOCK_N * 128;          // 32 KB
-constexpr int SFA_BYTES = 4 * 512;              // 4 k-blocks of 64 x 128 rows
-constexpr int SFB_BYTES = 2 * 4 * 512;          // 2 row halves x 4 k-blocks
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;   // 54 KB
+constexpr int SF_BLOCK = 4096;                  // one replicated scale block (8 TMEM columns)
+constexpr int SFA_BYTES = 2 * SF_BLOCK;         // 4 k-blocks x 128 rows
+constexpr int SFB_BYTES = 4 * SF_BLOCK;         // 4 k-blocks x 2 row halves
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;   // 72 KB
 constexpr int THREADS = 320;              // producer, MMA, 8 epilogue warps
 constexpr int EPI_WARPS = 8;
 constexpr uint32_t TMEM_COLS = 512;
@@ -115,7 +120,6 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int num_tiles = p.num_m_blocks * p.num_n_blocks;
   const int kiters = p.nk + p.nl;
-  const size_t kb_per_row = (size_t)(p.K_pad / 64);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -137,12 +141,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_arrive_expect_tx(bar, STAGE_BYTES);
             tma_load_2d(st, &tmA, it * 128, mb * BLOCK_M, bar);
             tma_load_2d(st + A_BYTES, &tmB, it * 128, nb * BLOCK_N, bar);
-            bulk_load(st + A_BYTES + B_BYTES, p.sX + ((size_t)mb * kb_per_row + it * 4) * 512,
-                      SFA_BYTES, bar);
-            bulk_load(st + A_BYTES + B_BYTES + SFA_BYTES,
-                      p.sR + ((size_t)(2 * nb) * kb_per_row + it * 4) * 512, SFB_BYTES / 2, bar);
-            bulk_load(st + A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES / 2,
-                      p.sR + ((size_t)(2 * nb + 1) * kb_per_row + it * 4) * 512, SFB_BYTES / 2, bar);
+            bulk_load(st + A_BYTES + B_BYTES, p.sX + ((size_t)mb * p.nk + it) * SFA_BYTES, SFA_BYTES, bar);
+            bulk_load(st + A_BYTES + B_BYTES + SFA_BYTES, p.sR + ((size_t)nb * p.nk + it) * SFB_BYTES, SFB_BYTES,
+                      bar);
           } else {
             const int c = it - p.nk;
             mbar_arrive_expect_tx(bar, A_BYTES + B_BYTES);
@@ -175,13 +176,11 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t b = a + A_BYTES;
           if (it < p.nk) {
             const uint32_t sfa = b + B_BYTES, sfb = sfa + SFA_BYTES;
+            // six copies of 8 columns: SFA k-blocks (0,1), (2,3); SFB k-block kb, both row halves
 #pragma unroll
-            for (int kb = 0; kb < 4; ++kb) tmem_cp_sf_atom(tmem + SFA_COL + 4 * kb, sfa + kb * 512);
+            for (int j = 0; j < 2; ++j) tmem_cp_sf_block(tmem + SFA_COL + 8 * j, sfa + j * SF_BLOCK);
 #pragma unroll
-            for (int kb = 0; kb < 4; ++kb) {
-              tmem_cp_sf_atom(tmem + SFB_COL + 8 * kb, sfb + kb * 512);
-              tmem_cp_sf_atom(tmem + SFB_COL + 8 * kb + 4, sfb + SFB_BYTES / 2 + kb * 512);
-            }
+            for (int kb = 0; kb < 4; ++kb) tmem_cp_sf_block(tmem + SFB_COL + 8 * kb, sfb + kb * SF_BLOCK);
 #pragma unroll
             for (int kb = 0; kb < 4; ++kb)
               mma_nvf4(tmem + ACC_COL, desc_k_sw128(a + 32 * kb), desc_k_sw128(b + 32 * kb), IDESC_F4,

@@ -36,8 +36,8 @@ struct K2Params {
   int num_m_blocks, num_n_blocks;
   int nk;                  // K_pad / 256 4-bit k-tiles
   int nl;                  // r_pad / 64 low-rank k-tiles (0: plain W4A4 GEMM)
-  const uint8_t* sX;       // activation scales
-  const uint8_t* sR;       // weight scales
+  const uint8_t* sX;       // activation scales, replicated layout (sfx_rep_offset)
+  const uint8_t* sR;       // weight scales, replicated layout (sfw_rep_offset)
   const float* bias;       // [N_pad]
   float alpha;             // s_tX * s_tR
   int epi;                 // 0 none, 1 GELU (tanh form)
@@ -92,11 +92,12 @@ struct PrepParams {
   unsigned* amax_bits;         // scratch, 1 word
   uint8_t* qR;                 // [N_pad][K_pad/2]
   uint8_t* sR;                 // scales
-  __nv_bfloat16* L1t;          // [K_pad/256][4][r_tot][64], 128-byte swizzled
+  uint8_t* sR_rep;             // NVFP4: kernel 2's replicated copy (sfw_rep_offset)
+  __nv_bfloat16* L1t;          // [K_pad/64][r_tot][64], 128-byte swizzled
   __nv_bfloat16* L2a;          // [N_pad][r_pad]
   float* bias_f;               // [N_pad]
   float* lambda_inv;           // [K]
-  float* lambda_inv_k1;        // [K_pad], permuted per 256-wide stage for kernel 1
+  float* lambda_inv_k1;        // [K_pad], permuted per 64-wide stage for kernel 1
 };
 cudaError_t launch_prepare_residual(const PrepParams& p, cudaStream_t stream);
 cudaError_t launch_prepare_quantize(const PrepParams& p, float s_tR, float alpha,

@@ -196,6 +196,19 @@ __global__ void factors_kernel(PrepParams p, float alpha) {
   }
 }
 
+// Kernel 2's copy of the NVFP4 weight scales: every (row, 64-k block) word
+// of the atom layout written to its four replicas (see sfw_rep_offset).
+__global__ void replicate_weight_scales_kernel(PrepParams p) {
+  const int kbs = p.K_pad / 64;
+  const size_t total = (size_t)p.N_pad * kbs;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+    const int n = (int)(i / kbs), kb = (int)(i % kbs);
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(p.sR + sf_atom_offset(n, kb * 4, p.K_pad));
+#pragma unroll
+    for (int q = 0; q < 4; ++q) *reinterpret_cast<uint32_t*>(p.sR_rep + sfw_rep_offset(n, kb, q, p.K_pad)) = w;
+  }
+}
+
 __global__ void selftest_timeout_kernel(DeviceErr err) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
@@ -244,6 +257,9 @@ cudaError_t launch_prepare_quantize(const PrepParams& p, float s_tR, float alpha
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   factors_kernel<<<592, 256, 0, stream>>>(p, alpha);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || p.fmt != 0) return e;
+  replicate_weight_scales_kernel<<<592, 256, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -46,12 +46,6 @@ constexpr int IL_BYTES = BK * 4;             // 1/lambda for the stage
 constexpr int W_PROD = 0, W_MMA = 1, W_Q0 = 2;
 constexpr int MAX_STAGES = 8;
 
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-  uint4 u;
-  asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w) : "r"(addr));
-  return u;
-}
-
 __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
@@ -227,11 +221,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (p.fmt == 0) {
         uint32_t sc;
         quant_nvfp4_16_tab(v, p.six_st, inv_tab, codes, sc);
-        // the row's four scale bytes are adjacent in the scale atom: one word
+        // the row's four scale bytes form one word; kernel 2 wants it in four
+        // replicas (one per TMEM sub-partition): lane qg of the quad writes replica qg
         uint32_t sw = sc << (8 * qg);
         sw |= __shfl_xor_sync(0xffffffffu, sw, 1);
         sw |= __shfl_xor_sync(0xffffffffu, sw, 2);
-        if (qg == 0) *reinterpret_cast<uint32_t*>(p.sX + sf_atom_offset(m, kb * 4, p.K_pad)) = sw;
+        *reinterpret_cast<uint32_t*>(p.sX + sfx_rep_offset(m, kb, qg, p.K_pad)) = sw;
       } else {
         __half sc;
         quant_int4_16of64(v, codes, sc);

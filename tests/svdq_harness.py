@@ -31,6 +31,26 @@ def sf_atoms_to_canonical(raw: np.ndarray, rows: int, K: int, K_pad: int) -> np.
     return raw.reshape(-1)[off]
 
 
+def sfx_replicated_to_canonical(raw: np.ndarray, rows: int, K: int, K_pad: int) -> np.ndarray:
+    """Kernel 1's NVFP4 activation scales (every word stored in four replicas)
+    -> (rows, K/16) uint8.  Asserts that the four replicas agree."""
+    r = np.arange(rows)[:, None]
+    g = np.arange(K // 16)[None, :]
+    kb = g // 4
+    flat = raw.reshape(-1)
+    out = None
+    for q in range(4):
+        L = r % 32 + 32 * q
+        off = ((((r // 128) * (K_pad // 256) + kb // 4) * 2 + (kb % 4) // 2) * 4096 + (L // 8) * 256
+               + (kb % 2) * 128 + (L % 8) * 16 + ((r % 128) // 32) * 4 + g % 4)
+        v = flat[off]
+        if out is None:
+            out = v
+        else:
+            assert np.array_equal(out, v), "scale replicas differ"
+    return out
+
+
 def unpack_codes(raw: np.ndarray, rows: int, K: int, K_pad: int, fmt: str) -> np.ndarray:
     b = raw.reshape(-1)[: rows * (K_pad // 2)].reshape(rows, K_pad // 2)
     c = F.unpack_nibbles(b)[:, :K]
@@ -215,7 +235,7 @@ class GpuLayer:
         i = self.info
         q = unpack_codes(to_np(qX), M, self.K, i.K_pad, self.fmt)
         if self.fmt == "nvfp4":
-            s = sf_atoms_to_canonical(to_np(sX), M, self.K, i.K_pad)
+            s = sfx_replicated_to_canonical(to_np(sX), M, self.K, i.K_pad)
         else:
             s = int4_scales(to_np(sX), M, self.K, i.K_pad)
         lr = to_np(LR)[: M * i.r_pad * 2].view(np.uint16).reshape(M, i.r_pad)
