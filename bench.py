@@ -53,14 +53,24 @@ def measured_peaks():
         return dict(bf16=FALLBACK_BF16_TFLOPS, bf16_sustained=None, hbm=FALLBACK_HBM_GBS, source="fallback")
 
 
-def file_sha(path):
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def file_sha(paths):
+    """First 16 hex digits of the sha256 of the files' contents, in order."""
+    h = hashlib.sha256()
+    for path in paths:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def kernel_sources(name):
+    d = os.path.join(ROOT, "rank_gemm_b200", "csrc")
+    return [os.path.join(d, name), os.path.join(d, "common.cuh"), os.path.join(d, "kernels.h")]
 
 
 def profiled_traffic(profile_name, kernel_src):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the kernel source as it is now; else None."""
+    the kernel source (the kernel file, common.cuh, kernels.h) as it is now;
+    else None."""
     path = os.path.join(ROOT, "profiles", profile_name)
     if not os.path.exists(path):
         return None
@@ -323,9 +333,13 @@ def run_ours(args, world, rank, local):
     peaks = measured_peaks()
     fp4_peak = peaks["bf16"] * FP4_PER_BF16
     k2_tflops = flops / (k2_ms * 1e-3) / 1e12
-    bytes_k1 = M * K * 2 + K * 4 + r * K * 2 + qb + sb + lb
-    bytes_k2 = qb + sb + lb + (N * K // 2) + (N * K // 16) + N * 64 * 2 + N * 4 + M * N * 2
-    traffic = profiled_traffic("gemm_nvfp4_qkv.md", os.path.join(ROOT, "rank_gemm_b200", "csrc", "gemm_nvfp4.cu"))
+    # algorithmic bytes: each operand once, scales counted once (the four
+    # replicas kernel 2 reads are an implementation cost and show in traffic)
+    sx_once = -(-M // 128) * 128 * (K // 16)
+    bytes_k1 = M * K * 2 + K * 4 + r * K * 2 + M * K // 2 + sx_once + lb
+    bytes_k2 = M * K // 2 + sx_once + lb + (N * K // 2) + (N * K // 16) + N * 64 * 2 + N * 4 + M * N * 2
+    traffic = profiled_traffic("gemm_nvfp4_qkv.md", kernel_sources("gemm_nvfp4.cu"))
+    traffic_k1 = profiled_traffic("quant_down_qkv.md", kernel_sources("quant_down.cu"))
 
     # low-rank overhead (the "Nunchaku engine design" figure's comparison):
     # plain W4A4 path (quantize + GEMM, no low-rank branch), the fused layer,
@@ -403,7 +417,7 @@ def run_ours(args, world, rank, local):
                "roofline_k1": {"kernel": "quant_down (kernel 1)", "bound": "hbm",
                                "achieved": round(bytes_k1 / (k1_ms * 1e-3) / 1e9, 1), "peak": peaks["hbm"],
                                "unit": "GB/s", "frac": round(bytes_k1 / (k1_ms * 1e-3) / 1e9 / peaks["hbm"], 4),
-                               "algorithmic_bytes": bytes_k1, "us": round(k1_ms * 1e3, 2)},
+                               "traffic": traffic_k1, "algorithmic_bytes": bytes_k1, "us": round(k1_ms * 1e3, 2)},
                "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": M * K * 2,
                        "d2h_bytes_per_step": M * N * 2, "ms_per_step": round(e2e_ms, 4)},
                "lowrank_overhead": {"plain_w4a4_us": round(t_plain * 1e3, 2), "fused_us": round(t_fused * 1e3, 2),
