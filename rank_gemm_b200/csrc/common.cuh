@@ -152,6 +152,20 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
                : "memory");
 }
 
+// ----------------------------------------------------------------- programmatic dependent launch
+// Kernels 1 and 2 are launched with programmatic stream serialization: a
+// kernel may start (set up barriers and TMEM) while the previous kernel on
+// the stream is still running, and waits here before its first global
+// memory access; the previous kernel's writes are visible after the wait.
+// Without that launch attribute both instructions do nothing.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// Lets the next kernel on the stream be scheduled onto SMs this grid frees.
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ----------------------------------------------------------------- thread-block clusters
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;

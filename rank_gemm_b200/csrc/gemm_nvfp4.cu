@@ -117,6 +117,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
+  grid_launch_dependents();
+  grid_dependency_wait();   // qX, sX and LR from kernel 1 are visible from here
 
   const int num_tiles = p.num_m_blocks * p.num_n_blocks;
   const int kiters = p.nk + p.nl;
@@ -278,8 +280,17 @@ cudaError_t launch_gemm_nvfp4(const CUtensorMap& tmA, const CUtensorMap& tmB, co
   if (e != cudaSuccess) return e;
   const int tiles = p.num_m_blocks * p.num_n_blocks;
   const int grid = tiles < num_sms ? tiles : num_sms;
-  gemm_nvfp4_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmLR, tmL2, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_nvfp4_kernel, tmA, tmB, tmLR, tmL2, p);
 }
 
 }  // namespace svdq

@@ -136,6 +136,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = p.do_lr ? *tmem_slot : 0u;
+  grid_launch_dependents();
+  grid_dependency_wait();   // X, the weights and the output buffers are safe to touch from here
 
   if (warp == W_PROD) {
     // ---------------------------------------------------------------- producer
@@ -328,13 +330,15 @@ cudaError_t launch_quant_down(const CUtensorMap& tmX, K1Params p, cudaStream_t s
   cfg.blockDim = dim3(THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = KSPLIT;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = KSPLIT;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = p.do_lr ? 1 : 0;   // only the LR reduction needs the cluster
+  cfg.numAttrs = p.do_lr ? 2 : 1;   // only the LR reduction needs the cluster
   return cudaLaunchKernelEx(&cfg, quant_down_kernel, tmX, p);
 }
 
