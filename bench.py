@@ -40,6 +40,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 WORKLOAD = dict(name="nvfp4_qkv_M4608_K3072_N9216_r32", fmt="nvfp4", M=4608, K=3072, N=9216, rank=32)
+# --workload: the QKV projection is the bench line; the others are the
+# remaining parity configurations, timed the same way for their profiles.
+WORKLOADS = ("qkv", "int4_qkv", "mlp_fc1", "mlp_fc2", "lora")
+INT8_PER_BF16 = 2.0         # nominal dense INT8 : BF16 tensor throughput (4.5 : 2.25)
 METRIC = "SVDQuant W4A4 linear effective TFLOPS & % of FP4 tensor peak; µs/layer"
 UNIT = "TFLOP/s"
 FP4_PER_BF16 = 4.0          # nominal dense FP4 : BF16 tensor throughput (9 : 2.25 PFLOP/s)
@@ -266,6 +270,54 @@ def gpu_factors(B, Wt, X, rank, torch):
     return lam, float(act.item()), L1f, L2
 
 
+def build_layer(name, B, torch, dev):
+    """Device tensors of one workload plus its prepared weights handle."""
+    import numpy as np
+    import workloads
+
+    def dev_bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16).to(dev)
+
+    def prepare(fmt, X0, W, bias, rank, lora=None):
+        Wt = dev_bf16(W.T)
+        lam, act, L1f, L2 = gpu_factors(B, Wt, X0, rank, torch)
+        la, lb, lr = (dev_bf16(lora[0]), dev_bf16(lora[1]), lora[0].shape[1]) if lora else (None, None, 0)
+        return B.svdq_prepare_weights(fmt, W.shape[0], W.shape[1], rank, Wt, lam, L1f, L2, dev_bf16(bias),
+                                      la, lb, lr, act)
+
+    epi = B.SVDQ_EPI_NONE
+    if name in ("qkv", "int4_qkv"):
+        L = workloads.qkv() if name == "qkv" else workloads.int4_qkv()
+        X0 = dev_bf16(L.X)
+        h = prepare(L.fmt, X0, L.W, L.bias, L.rank)
+        return dict(name=L.name, fmt=L.fmt, X0=X0, h=h, M=L.M, K=L.K, N=L.N, rank=L.rank, lora=0, epi=epi)
+    if name in ("mlp_fc1", "mlp_fc2"):
+        fc1, (W2, b2, _) = workloads.mlp_pair()
+        X1 = dev_bf16(fc1.X)
+        h1 = prepare("nvfp4", X1, fc1.W, fc1.bias, fc1.rank)
+        if name == "mlp_fc1":
+            return dict(name=fc1.name, fmt="nvfp4", X0=X1, h=h1, M=fc1.M, K=fc1.K, N=fc1.N, rank=fc1.rank, lora=0,
+                        epi=B.SVDQ_EPI_GELU_TANH)
+        # fc2's activation: this library's fc1 output (GELU), computed once
+        Y1 = torch.empty(fc1.M, fc1.N, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(B.svdq_linear_workspace_bytes(h1, fc1.M), dtype=torch.uint8, device=dev)
+        B.svdq_linear(h1, fc1.M, X1, B.SVDQ_EPI_GELU_TANH, Y1, ws)
+        torch.cuda.synchronize()
+        B.svdq_free_weights(h1)
+        del ws
+        h2 = prepare("nvfp4", Y1, W2, b2, 32)
+        return dict(name="nvfp4_mlp_fc2_M%d_K12288_N3072_r32" % fc1.M, fmt="nvfp4", X0=Y1, h=h2, M=fc1.M,
+                    K=12288, N=3072, rank=32, lora=0, epi=epi)
+    if name == "lora":
+        base = workloads.lora_sweep_base()
+        M = 4096
+        X0 = dev_bf16(base.X[:M])
+        h = prepare("nvfp4", X0, base.W, base.bias, 32, (base.lora_A, base.lora_B))
+        return dict(name="nvfp4_lora_M4096_K3072_N3072_r32_lora%d" % base.lora_A.shape[1], fmt="nvfp4", X0=X0,
+                    h=h, M=M, K=3072, N=3072, rank=32, lora=base.lora_A.shape[1], epi=epi)
+    raise ValueError(name)
+
+
 def run_ours(args, world, rank, local):
     import numpy as np
     import torch
@@ -282,13 +334,10 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
 
-    Lw = workloads.qkv()
-    M, K, N, r = Lw.M, Lw.K, Lw.N, Lw.rank
-    X0 = torch.from_numpy(Lw.X).to(torch.bfloat16).to(dev)
-    Wt = torch.from_numpy(np.ascontiguousarray(Lw.W.T)).to(torch.bfloat16).to(dev)
-    bias = torch.from_numpy(Lw.bias).to(torch.bfloat16).to(dev)
-    lam, act, L1f, L2 = gpu_factors(B, Wt, X0, r, torch)
-    h = B.svdq_prepare_weights("nvfp4", K, N, r, Wt, lam, L1f, L2, bias, None, None, 0, act)
+    lay = build_layer(args.workload, B, torch, dev)
+    M, K, N, r, h, X0, fmt, epi = (lay[k] for k in ("M", "K", "N", "rank", "h", "X0", "fmt", "epi"))
+    r_tot = r + lay["lora"]
+    nv = fmt == "nvfp4"
 
     sets = 3
     Xs = [X0] + [X0.clone() for _ in range(sets - 1)]
@@ -305,7 +354,7 @@ def run_ours(args, world, rank, local):
         B.svdq_quantize_act_lowrank_down(h, M, Xs[i % sets], qX, sX, LR, stream)
         if ev:
             ev[1].record(stream)
-        B.svdq_w4a4_gemm_lowrank_up(h, M, qX, sX, LR, B.SVDQ_EPI_NONE, Ys[i % sets], stream)
+        B.svdq_w4a4_gemm_lowrank_up(h, M, qX, sX, LR, epi, Ys[i % sets], stream)
         if ev:
             ev[2].record(stream)
 
@@ -346,15 +395,23 @@ def run_ours(args, world, rank, local):
     flops = 2.0 * M * N * K
     value = weak_scaling_value(flops, K_steps, world, max_ms)
     peaks = measured_peaks()
-    fp4_peak = peaks["bf16"] * FP4_PER_BF16
+    # the contraction's own peak: FP4 (NVFP4) or INT8 (INT4 codes run on the
+    # int8 tensor core), each the measured bf16 peak times the nominal ratio
+    ratio = FP4_PER_BF16 if nv else INT8_PER_BF16
+    tc_peak = peaks["bf16"] * ratio
     k2_tflops = flops / (k2_ms * 1e-3) / 1e12
     # algorithmic bytes: each operand once, scales counted once (the four
     # replicas kernel 2 reads are an implementation cost and show in traffic)
-    sx_once = -(-M // 128) * 128 * (K // 16)
-    bytes_k1 = M * K * 2 + K * 4 + r * K * 2 + M * K // 2 + sx_once + lb
-    bytes_k2 = M * K // 2 + sx_once + lb + (N * K // 2) + (N * K // 16) + N * 64 * 2 + N * 4 + M * N * 2
-    traffic = profiled_traffic("gemm_nvfp4_qkv.md", kernel_sources("gemm_nvfp4.cu"))
-    traffic_k1 = profiled_traffic("quant_down_qkv.md", kernel_sources("quant_down.cu"))
+    g = 16 if nv else 64
+    sbytes = 1 if nv else 2
+    sx_once = -(-M // 128) * 128 * (K // g) * sbytes
+    r_pad = -(-r_tot // 64) * 64
+    bytes_k1 = M * K * 2 + K * 4 + r_tot * K * 2 + M * K // 2 + sx_once + M * r_pad * 2
+    bytes_k2 = (M * K // 2 + sx_once + M * r_pad * 2 + (N * K // 2) + N * (K // g) * sbytes + N * r_pad * 2 + N * 4
+                + M * N * 2)
+    k2_src = "gemm_nvfp4.cu" if nv else "gemm_int4.cu"
+    traffic = profiled_traffic("%s_%s.md" % (k2_src[:-3], args.workload), kernel_sources(k2_src))
+    traffic_k1 = profiled_traffic("quant_down_%s.md" % args.workload, kernel_sources("quant_down.cu"))
 
     # low-rank overhead (the "Nunchaku engine design" figure's comparison):
     # plain W4A4 path (quantize + GEMM, no low-rank branch), the fused layer,
@@ -374,19 +431,19 @@ def run_ours(args, world, rank, local):
     def plain(i):
         qX, sX, LR = acts[i % sets]
         B.svdq_quantize_act(h, M, Xs[i % sets], qX, sX, stream)
-        B.svdq_w4a4_gemm(h, M, qX, sX, Ys[i % sets], stream)
+        B.svdq_w4a4_gemm(h, M, qX, sX, Ys[i % sets], stream)   # no GELU: timing only
 
     def unfused(i):
         qX, sX, LR = acts[i % sets]
         B.svdq_quantize_act(h, M, Xs[i % sets], qX, sX, stream)
         B.svdq_lowrank_down(h, M, Xs[i % sets], LR, stream)
         B.svdq_w4a4_gemm(h, M, qX, sX, Ys[i % sets], stream)
-        B.svdq_lowrank_up(h, M, LR, B.SVDQ_EPI_NONE, Ys[i % sets], stream)
+        B.svdq_lowrank_up(h, M, LR, epi, Ys[i % sets], stream)
 
     n_ov = min(K_steps, 100)
     t_plain = timed(plain, n_ov)
     t_fused = timed(lambda i: (B.svdq_quantize_act_lowrank_down(h, M, Xs[i % sets], *acts[i % sets], stream),
-                               B.svdq_w4a4_gemm_lowrank_up(h, M, *acts[i % sets], B.SVDQ_EPI_NONE,
+                               B.svdq_w4a4_gemm_lowrank_up(h, M, *acts[i % sets], epi,
                                                            Ys[i % sets], stream)), n_ov)
     t_unfused = timed(unfused, n_ov)
 
@@ -399,14 +456,14 @@ def run_ours(args, world, rank, local):
     Xd, Yd = Xs[0], Ys[0]
     for _ in range(3):
         Xd.copy_(Xh, non_blocking=True)
-        B.svdq_linear(h, M, Xd, B.SVDQ_EPI_NONE, Yd, ws, None, stream)
+        B.svdq_linear(h, M, Xd, epi, Yd, ws, None, stream)
         Yh.copy_(Yd, non_blocking=True)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
         Xd.copy_(Xh, non_blocking=True)
-        B.svdq_linear(h, M, Xd, B.SVDQ_EPI_NONE, Yd, ws, None, stream)
+        B.svdq_linear(h, M, Xd, epi, Yd, ws, None, stream)
         Yh.copy_(Yd, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
@@ -417,17 +474,19 @@ def run_ours(args, world, rank, local):
     if rank == 0:
         out = {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": K_steps,
                "warmup": W_steps, "ms_per_step": round(max_ms / K_steps, 5), "us_per_layer": round(max_ms / K_steps * 1e3, 2),
-               "fp4_peak_frac": round(value / world / fp4_peak, 4), "higher_is_better": True, "scaling": "weak",
-               "vs_baseline": None, "dtype": "nvfp4",
+               "fp4_peak_frac" if nv else "int8_peak_frac": round(value / world / tc_peak, 4),
+               "higher_is_better": True, "scaling": "weak",
+               "vs_baseline": None, "dtype": fmt,
                "data": "synthetic (seeded, FLUX-shaped, 0.5% outlier channels x20 / x5), random-init weights",
-               "config": {"workload": WORKLOAD["name"], "M": M, "K": K, "N": N, "rank": r, "format": "nvfp4",
-                          "group": 16, "parallelism": "replicas x%d (each rank its own batch)" % world,
+               "config": {"workload": lay["name"], "M": M, "K": K, "N": N, "rank": r, "lora_rank": lay["lora"],
+                          "format": fmt, "group": g, "epilogue": "gelu_tanh" if epi else "none",
+                          "parallelism": "replicas x%d (each rank its own batch)" % world,
                           "l2": "3 rotating X/Y/workspace sets (%.0f MB) > 126 MB L2"
                                 % (sets * (M * K * 2 + M * N * 2 + qb + sb + lb) / 1e6)},
-               "roofline": {"kernel": "gemm_nvfp4 (kernel 2)", "bound": "tensor", "achieved": round(k2_tflops, 2),
-                            "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(k2_tflops / fp4_peak, 4),
-                            "peak_source": "%s bf16 %.1f TFLOP/s x %.0f (nominal FP4:BF16)"
-                                           % (peaks["source"], peaks["bf16"], FP4_PER_BF16),
+               "roofline": {"kernel": "%s (kernel 2)" % k2_src[:-3], "bound": "tensor", "achieved": round(k2_tflops, 2),
+                            "peak": round(tc_peak, 1), "unit": "TFLOP/s", "frac": round(k2_tflops / tc_peak, 4),
+                            "peak_source": "%s bf16 %.1f TFLOP/s x %.0f (nominal %s:BF16)"
+                                           % (peaks["source"], peaks["bf16"], ratio, "FP4" if nv else "INT8"),
                             "traffic": traffic, "algorithmic_bytes": bytes_k2, "us": round(k2_ms * 1e3, 2)},
                "roofline_k1": {"kernel": "quant_down (kernel 1)", "bound": "hbm",
                                "achieved": round(bytes_k1 / (k1_ms * 1e-3) / 1e9, 1), "peak": peaks["hbm"],
@@ -447,7 +506,7 @@ def run_ours(args, world, rank, local):
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
     if rank == 0:
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and args.workload == "qkv":
             L, pw = oracle_setup()
             out["cpu_baseline"] = cpu_baseline(L, pw)
         print(json.dumps(out), flush=True)
@@ -460,6 +519,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=WORKLOADS, default="qkv")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
