@@ -52,9 +52,10 @@
  *           + ((r % 128) / 32) * 4 + g
  *         for each replica L = r % 32 + 32 q, q = 0..3.  4 * M_128 * K_pad/16
  *         bytes (M_128 = M rounded up to 128); rows >= M hold 0.
- *         INT4: binary16 block scales (one per 64 k) in 512-byte chunks of
- *         128 rows x 2 groups: the scale of row r and 64-group g sits at
- *         element (((r / 128) * (K_pad/128) + g / 2) * 2 + g % 2) * 128 + r % 128;
+ *         INT4: block scales (one per 64 k) rounded to binary16 and stored
+ *         widened to float32 (exactly), in 1 KB chunks of 128 rows x 2
+ *         groups: the scale of row r and 64-group g sits at float32 element
+ *         (((r / 128) * (K_pad/128) + g / 2) * 2 + g % 2) * 128 + r % 128;
  *         rows >= M and groups >= K/64 hold 0.
  *   LR    bf16 [M][r_pad]: X L1f for the r_tot low-rank columns, zeros after.
  */

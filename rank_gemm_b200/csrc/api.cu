@@ -136,7 +136,7 @@ size_t qx_bytes(const svdq_weights* w, int M) { return (size_t)M * (w->K_pad / 2
 size_t sx_bytes(const svdq_weights* w, int M) {
   const size_t rows = (size_t)round_up(M, 128);
   // NVFP4: four replicas of every scale word (see sfx_rep_offset)
-  return w->fmt == SVDQ_NVFP4 ? rows * (w->K_pad / 16) * 4 : rows * (w->K_pad / 64) * 2;
+  return w->fmt == SVDQ_NVFP4 ? rows * (w->K_pad / 16) * 4 : rows * (w->K_pad / 64) * 4;
 }
 size_t lr_bytes(const svdq_weights* w, int M) { return (size_t)M * w->r_pad * 2; }
 
@@ -232,8 +232,8 @@ svdq_status run_k2(const svdq_weights* w, int M, const void* qX, const void* sX,
   p.num_n_blocks = w->N_pad / 128;   // the INT4 kernel's tiles are 128 wide
   p.nk = w->K_pad / 128;
   p.nl = lowrank ? (w->r_tot + 31) / 32 : 0;
-  p.sX = static_cast<const __half*>(sX);
-  p.sR = reinterpret_cast<const __half*>(w->sR);
+  p.sX = static_cast<const float*>(sX);
+  p.sR = reinterpret_cast<const float*>(w->sR);
   p.bias = w->bias_f;
   p.epi = (int)epi;
   p.Y = static_cast<__nv_bfloat16*>(Y);
@@ -329,7 +329,7 @@ svdq_status svdq_prepare_weights(svdq_format fmt, int K, int N, int rank, const 
   w->N_pad = round_up(N, 256);
   w->r_pad = round_up(r_tot, 64);
   const size_t qr_b = (size_t)w->N_pad * (w->K_pad / 2);
-  const size_t sr_b = fmt == SVDQ_NVFP4 ? (size_t)w->N_pad * (w->K_pad / 16) : (size_t)w->N_pad * (w->K_pad / 64) * 2;
+  const size_t sr_b = fmt == SVDQ_NVFP4 ? (size_t)w->N_pad * (w->K_pad / 16) : (size_t)w->N_pad * (w->K_pad / 64) * 4;
   float* R = nullptr;
   unsigned* amax = nullptr;
   bool ok = cudaMalloc(&w->qR, qr_b) == cudaSuccess && cudaMalloc(&w->sR, sr_b) == cudaSuccess &&

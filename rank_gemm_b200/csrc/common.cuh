@@ -68,14 +68,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
+// The suspend-time hint lets a waiting warp sleep until the phase completes
+// (or up to 1 ms) instead of polling, so waiting warps leave the issue slots
+// to the warps that work.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(1000000u)
       : "memory");
   return ok != 0;
 }
@@ -407,6 +410,16 @@ __device__ __forceinline__ void mul2_rn(float a0, float a1, float b0, float b1, 
   asm("mov.b64 {%0, %1}, %2;" : "=f"(r0), "=f"(r1) : "l"(r));
 }
 
+// (r0, r1) = fl32(a * b + c) element-wise, one packed instruction.
+__device__ __forceinline__ void fma2_rn(float a0, float a1, float b0, float b1, float& c0, float& c1) {
+  uint64_t a, b, c, r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(b) : "f"(b0), "f"(b1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(c) : "f"(c0), "f"(c1));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(c0), "=f"(c1) : "l"(r));
+}
+
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -533,7 +546,8 @@ __host__ __device__ __forceinline__ size_t sfw_rep_offset(int row, int kb, int q
          (r >> 5) * 4;
 }
 
-// Element offset of (row, 64-group) in the INT4 binary16 scale layout:
+// Element offset of (row, 64-group) in the INT4 scale layout (binary16
+// values stored widened to float32):
 // 512-byte chunks of 128 rows x 2 groups (one 128-wide k-tile), ordered
 // (row block, k-tile), group-major inside a chunk.
 __host__ __device__ __forceinline__ size_t int4_scale_offset(int row, int g64, int kpad) {

@@ -3,23 +3,25 @@
 // card), on the int8 tensor-core path.
 //
 // INT4 block scales are binary16 per 64 elements, which no block-scaled MMA
-// kind can take, so each 64-group is its own integer product:
+// kind can take, so each 64-group is its own product:
 //     y[m,n] = sum_g sX[m,g] sR[n,g] (sum_{k in g} qX[m,k] qR[n,k]) + LR[m,:] L2[n,:] + b[n]
-// The int4 codes are unpacked to int8 in shared memory, every group runs as
-// two tcgen05.mma.kind::i8 (K = 32) into a fresh int32 TMEM tile, and CUDA
-// cores apply sX sR and accumulate in fp32 registers.  That per-group rescale
-// (about three ALU operations per output element per group) bounds this kernel,
-// not the int8 tensor core.
+// The int4 codes (-8..7) are unpacked in shared memory to FP8 E4M3, which
+// holds them exactly; every group runs as two tcgen05.mma.kind::f8f6f4
+// (K = 32) into a fresh fp32 TMEM tile, whose sums (|.| <= 64 * 64) are exact,
+// so the group product needs no integer-to-float conversion.  CUDA cores apply
+// sX sR and accumulate in fp32 registers with packed (f32x2) multiply and FMA:
+// one instruction per output element per group, the bound of this kernel.
 //
 // One 128 x 128 output tile per CTA at a time, persistent over tiles:
 //   warp 0       TMA producer: packed int4 tiles of qX and qR (128 rows x 64 B
-//                per 128-wide k-tile) into a staging ring, then the low-rank
-//                chunks (LR and L2, 32 columns, 64-byte swizzle).
-//   warps 1-4    unpack: staging int4 -> int8 operand tiles (128-byte swizzle)
-//                in the MMA ring.
-//   warp 5       TMEM owner and MMA issuer (kind::i8 per group into one of two
-//                TMEM buffers; the low-rank chunks as kind::f16 straight from
-//                the staging ring into one more buffer use).
+//                per 128-wide k-tile) into a staging ring, the k-tile's scale
+//                chunks of both (1 KB each) into a scale ring, then the
+//                low-rank chunks (LR and L2, 32 columns, 64-byte swizzle).
+//   warps 1-4    unpack: staging int4 -> E4M3 operand tiles (128-byte
+//                swizzle) in the MMA ring, three byte permutes per 4 codes.
+//   warp 5       TMEM owner and MMA issuer (per group into one of four TMEM
+//                buffers; the low-rank chunks as kind::f16 straight from the
+//                staging ring into one more buffer use).
 //   warps 6-13   rescale + epilogue: 2 warps per TMEM sub-partition, 64 columns
 //                each; fp32 accumulators in registers; bias, GELU, bf16 store.
 #include "common.cuh"
@@ -31,31 +33,36 @@ namespace {
 
 constexpr int BM = 128, BN = 128;
 constexpr int ST = 6;                    // staging ring (packed int4 / low-rank chunks)
-constexpr int MS = 3;                    // MMA ring (unpacked int8 tiles)
+constexpr int MS = 3;                    // MMA ring (E4M3 tiles)
+constexpr int SC = 8;                    // scale ring (one k-tile's scales of qX and qR)
 constexpr int STG_HALF = 8192;           // packed [128 x 64 B] or bf16 [128 x 32]
 constexpr int STG_BYTES = 2 * STG_HALF;
-constexpr int OP_BYTES = 16384;          // int8 [128 x 128 B]
+constexpr int OP_BYTES = 16384;          // E4M3 [128 x 128 B]
 constexpr int MMA_BYTES = 2 * OP_BYTES;
+constexpr int SC_HALF = 1024;            // float32 [2 groups][128 rows]
+constexpr int SC_BYTES = 2 * SC_HALF;
 constexpr int WARPS = 14, THREADS = WARPS * 32;
 constexpr int W_UNPACK = 1, W_MMA = 5, W_RESCALE = 6;
-constexpr uint32_t TMEM_COLS = 256;
-constexpr uint32_t IDESC_I8 = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                              ((uint32_t)(BM >> 4) << 24);
+constexpr int NBUF = 4;                  // TMEM group buffers of BN columns
+constexpr uint32_t TMEM_COLS = NBUF * BN;
+// kind::f8f6f4: fp32 D, E4M3 A and B (format code 0), K-major
+constexpr uint32_t IDESC_F8 = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 constexpr uint32_t IDESC_BF = idesc_bf16_f32(BM, BN);
 
 struct Ctl {
-  uint64_t sfull[ST], sempty[ST], mfull[MS], mempty[MS], dfull[2], dempty[2];
+  uint64_t sfull[ST], sempty[ST], mfull[MS], mempty[MS], cfull[SC], cempty[SC], dfull[NBUF], dempty[NBUF];
   uint32_t unpack_done[ST];
   uint32_t tmem_base;
   int abort;
 };
-constexpr size_t SMEM_BYTES = (size_t)ST * STG_BYTES + (size_t)MS * MMA_BYTES + 1024 + sizeof(Ctl);
+constexpr size_t SMEM_BYTES =
+    (size_t)ST * STG_BYTES + (size_t)MS * MMA_BYTES + (size_t)SC * SC_BYTES + 1024 + sizeof(Ctl);
 
-__device__ __forceinline__ void mma_i8(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+__device__ __forceinline__ void mma_f8(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
       "l"(a), "l"(b), "r"(idesc), "r"(acc)
       : "memory");
 }
@@ -63,24 +70,51 @@ __device__ __forceinline__ void mma_i8(uint32_t d, uint64_t a, uint64_t b, uint3
 // K-major bf16 tile with 64-byte rows in the 64-byte swizzle (8-row groups 512 B apart).
 __device__ __forceinline__ uint64_t desc_k_sw64(uint32_t addr) { return smem_desc(addr, 16, 512, 4); }
 
-// Sign-extends the four 4-bit values held in the low nibbles of the bytes of x.
-__device__ __forceinline__ uint32_t sext4x4(uint32_t x) {
-  return ((x ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
+// Packed float32 pairs kept in 64-bit registers (element 0 in the low half).
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
 }
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t u2(uint32_t lo, uint32_t hi) { return ((uint64_t)hi << 32) | lo; }
+__device__ __forceinline__ void lds2x64(uint32_t addr, uint64_t& a, uint64_t& b) {
+  asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "r"(addr));
+}
+
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t r;
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
   return r;
 }
-// 16 packed bytes (32 int4, element 2j in the low nibble of byte j) -> 32 int8.
+// E4M3 bytes of the int4 codes 0..7 (values 0..7) and 8..15 (values -8..-1),
+// four per word, code c at byte c % 4.
+constexpr uint32_t E4M3_POS_LO = 0x44403800u, E4M3_POS_HI = 0x4E4C4A48u;   // 0, 1, 2, 3 | 4, 5, 6, 7
+constexpr uint32_t E4M3_NEG_LO = 0xCACCCED0u, E4M3_NEG_HI = 0xB8C0C4C8u;   // -8, -7, -6, -5 | -4, -3, -2, -1
+// Four codes (the 4 nibbles of sel, in k order) -> four E4M3 bytes: look up
+// code & 7 in both halves of the table, then pick per byte by bit 3.
+__device__ __forceinline__ uint32_t e4m3x4(uint32_t sel) {
+  const uint32_t s7 = sel & 0x7777u;
+  const uint32_t pos = prmt(E4M3_POS_LO, E4M3_POS_HI, s7), neg = prmt(E4M3_NEG_LO, E4M3_NEG_HI, s7);
+  return prmt(pos, neg, ((sel >> 1) & 0x4444u) | 0x3210u);
+}
+// 16 packed bytes (32 int4, element 2j in the low nibble of byte j) -> 32 E4M3 bytes.
 __device__ __forceinline__ void unpack32(const uint4 p, uint4& o0, uint4& o1) {
   const uint32_t w[4] = {p.x, p.y, p.z, p.w};
   uint32_t o[8];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const uint32_t lo = sext4x4(w[i] & 0x0F0F0F0Fu), hi = sext4x4((w[i] >> 4) & 0x0F0F0F0Fu);
-    o[2 * i] = prmt(lo, hi, 0x5140u);
-    o[2 * i + 1] = prmt(lo, hi, 0x7362u);
+    o[2 * i] = e4m3x4(w[i] & 0xFFFFu);
+    o[2 * i + 1] = e4m3x4(w[i] >> 16);
   }
   o0 = make_uint4(o[0], o[1], o[2], o[3]);
   o1 = make_uint4(o[4], o[5], o[6], o[7]);
@@ -106,7 +140,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stg = base;                              // ST x 16 KB
   uint8_t* mring = base + ST * STG_BYTES;           // MS x 32 KB
-  Ctl* ctl = reinterpret_cast<Ctl*>(mring + MS * MMA_BYTES);
+  uint8_t* sring = mring + MS * MMA_BYTES;          // SC x 2 KB
+  Ctl* ctl = reinterpret_cast<Ctl*>(sring + SC * SC_BYTES);
   volatile int* abort_flag = &ctl->abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -126,7 +161,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(smem_u32(&ctl->mfull[s]), 4);
       mbar_init(smem_u32(&ctl->mempty[s]), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int c = 0; c < SC; ++c) {
+      mbar_init(smem_u32(&ctl->cfull[c]), 1);
+      mbar_init(smem_u32(&ctl->cempty[c]), 8);
+    }
+    for (int b = 0; b < NBUF; ++b) {
       mbar_init(smem_u32(&ctl->dfull[b]), 1);
       mbar_init(smem_u32(&ctl->dempty[b]), 8);
     }
@@ -148,8 +187,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0) {
     if (lane == 0) {
       // -------------------------------------------------------------- producer
-      int s = 0;
-      uint32_t ph = 0;
+      int s = 0, c = 0;
+      uint32_t ph = 0, cph = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
         const int mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
@@ -163,6 +202,19 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (it < nk) {
             tma_load_2d(dst, &tmXp, it * 64, mb * BM, bar);
             tma_load_2d(dst + STG_HALF, &tmRp, it * 64, nb * BN, bar);
+            // the k-tile's scale chunks: 128 rows x 2 groups of float32 each
+            if (!mbar_wait(smem_u32(&ctl->cempty[c]), cph ^ 1, abort_flag, p.err)) {
+              ok = false;
+              break;
+            }
+            const uint32_t cdst = smem_u32(sring + c * SC_BYTES), cbar = smem_u32(&ctl->cfull[c]);
+            mbar_arrive_expect_tx(cbar, SC_BYTES);
+            bulk_load(cdst, p.sX + ((size_t)mb * nk + it) * 256, SC_HALF, cbar);
+            bulk_load(cdst + SC_HALF, p.sR + ((size_t)nb * nk + it) * 256, SC_HALF, cbar);
+            if (++c == SC) {
+              c = 0;
+              cph ^= 1;
+            }
           } else {
             tma_load_2d(dst, &tmLR, (it - nk) * 32, mb * BM, bar);
             tma_load_2d(dst + STG_HALF, &tmL2, (it - nk) * 32, nb * BN, bar);
@@ -239,15 +291,15 @@ __global__ void __launch_bounds__(THREADS, 1)
           tc_fence_after();
           const uint32_t a = smem_u32(mring + t * MMA_BYTES), b = a + OP_BYTES;
           for (int j = 0; j < 2; ++j, ++uses) {
-            const uint32_t buf = uses & 1, dph = (uses >> 1) & 1;
+            const uint32_t buf = uses % NBUF, dph = (uses / NBUF) & 1;
             if (!mbar_wait(smem_u32(&ctl->dempty[buf]), dph ^ 1, abort_flag, p.err)) {
               ok = false;
               break;
             }
             tc_fence_after();
             const uint32_t d = tmem + buf * BN;
-            mma_i8(d, desc_k_sw128(a + 64 * j), desc_k_sw128(b + 64 * j), IDESC_I8, 0);
-            mma_i8(d, desc_k_sw128(a + 64 * j + 32), desc_k_sw128(b + 64 * j + 32), IDESC_I8, 1);
+            mma_f8(d, desc_k_sw128(a + 64 * j), desc_k_sw128(b + 64 * j), IDESC_F8, 0);
+            mma_f8(d, desc_k_sw128(a + 64 * j + 32), desc_k_sw128(b + 64 * j + 32), IDESC_F8, 1);
             tc_commit(smem_u32(&ctl->dfull[buf]));
           }
           if (!ok) break;
@@ -263,7 +315,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         if (!ok) break;
         if (nl) {
-          const uint32_t buf = uses & 1, dph = (uses >> 1) & 1;
+          const uint32_t buf = uses % NBUF, dph = (uses / NBUF) & 1;
           if (!mbar_wait(smem_u32(&ctl->dempty[buf]), dph ^ 1, abort_flag, p.err)) break;
           for (int c = 0; c < nl; ++c) {
             if (!mbar_wait(smem_u32(&ctl->sfull[s]), sph, abort_flag, p.err)) {
@@ -294,56 +346,80 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int sub = warp & 3, half = rw >> 2;        // TMEM sub-partition, 64-column half
     const int row = sub * 32 + lane;
     uint32_t uses = 0;
-    const __half* sX = p.sX;
-    const __half* sR = p.sR;
+    int c = 0;
+    uint32_t cph = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const int mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
       const int m = mb * BM + row, n0 = nb * BN + half * 64;
-      float acc[64];
+      uint64_t acc[32];                            // 64 columns as float32 pairs
 #pragma unroll
-      for (int c = 0; c < 64; ++c) acc[c] = 0.f;
+      for (int i = 0; i < 32; ++i) acc[i] = 0ull;
       bool ok = true;
-      const int groups = 2 * nk;
-      for (int g = 0; g < groups + (nl ? 1 : 0); ++g, ++uses) {
-        float sx = 0.f;
-        if (g < groups) sx = __half2float(sX[int4_scale_offset(m, g, p.K_pad)]);
-        const uint32_t buf = uses & 1, dph = (uses >> 1) & 1;
-        if (!mbar_wait(smem_u32(&ctl->dfull[buf]), dph, abort_flag, p.err)) {
+      for (int kt = 0; ok && kt < nk; ++kt) {
+        if (!mbar_wait(smem_u32(&ctl->cfull[c]), cph, abort_flag, p.err)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-#pragma unroll
-        for (int hc = 0; hc < 2; ++hc) {
-          uint32_t r[32];
-          tmem_ld32(tmem + ((uint32_t)(sub * 32) << 16) + buf * BN + half * 64 + hc * 32, r);
-          tmem_wait_ld();
-          if (hc == 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&ctl->dempty[buf]));
+        const float* sc = reinterpret_cast<const float*>(sring + c * SC_BYTES);
+        for (int j = 0; j < 2; ++j, ++uses) {        // the k-tile's two 64-groups
+          const uint32_t sxb = __float_as_uint(sc[j * 128 + row]);
+          const uint64_t sx2 = u2(sxb, sxb);
+          const uint32_t sra = smem_u32(sc + 256 + j * 128 + half * 64);
+          const uint32_t buf = uses % NBUF, dph = (uses / NBUF) & 1;
+          if (!mbar_wait(smem_u32(&ctl->dfull[buf]), dph, abort_flag, p.err)) {
+            ok = false;
+            break;
           }
-          if (g < groups) {
-            // weight scales of these 32 columns: 64 contiguous bytes, the same for the whole warp
-            const uint4* sp = reinterpret_cast<const uint4*>(sR + int4_scale_offset(n0 + hc * 32, g, p.K_pad));
+          tc_fence_after();
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const uint4 v = __ldg(sp + i);
-              const __half2* h2 = reinterpret_cast<const __half2*>(&v);
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float2 srf = __half22float2(h2[e]);
-                const int c = 8 * i + 2 * e;
-                // exact int32 -> float for |d| < 2^22 (here |d| <= 64 * 8 * 8)
-                const float d0 = __int_as_float(0x4B400000 + (int)r[c]) - 12582912.0f;
-                const float d1 = __int_as_float(0x4B400000 + (int)r[c + 1]) - 12582912.0f;
-                acc[hc * 32 + c] = fmaf(sx * srf.x, d0, acc[hc * 32 + c]);
-                acc[hc * 32 + c + 1] = fmaf(sx * srf.y, d1, acc[hc * 32 + c + 1]);
-              }
+          for (int hc = 0; hc < 2; ++hc) {
+            uint32_t r[32];
+            tmem_ld32(tmem + ((uint32_t)(sub * 32) << 16) + buf * BN + half * 64 + hc * 32, r);
+            tmem_wait_ld();
+            if (hc == 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(smem_u32(&ctl->dempty[buf]));
             }
-          } else {
+            // acc += (sx sr) d: the group's exact fp32 sum, rescaled by the
+            // product of two binary16 scales (exact in fp32), then one FMA
 #pragma unroll
-            for (int c = 0; c < 32; ++c) acc[hc * 32 + c] += __uint_as_float(r[c]);
+            for (int q = 0; q < 8; ++q) {
+              uint64_t sr01, sr23;
+              lds2x64(sra + (hc * 8 + q) * 16, sr01, sr23);
+              const int i = hc * 16 + 2 * q;
+              acc[i] = f2_fma(f2_mul(sx2, sr01), u2(r[4 * q], r[4 * q + 1]), acc[i]);
+              acc[i + 1] = f2_fma(f2_mul(sx2, sr23), u2(r[4 * q + 2], r[4 * q + 3]), acc[i + 1]);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&ctl->cempty[c]));   // this warp is done with the k-tile's scales
+        if (++c == SC) {
+          c = 0;
+          cph ^= 1;
+        }
+      }
+      if (ok && nl) {
+        // the low-rank branch: LR (L2) accumulated in fp32 by the tensor core
+        const uint32_t buf = uses % NBUF, dph = (uses / NBUF) & 1;
+        ++uses;
+        if (!mbar_wait(smem_u32(&ctl->dfull[buf]), dph, abort_flag, p.err)) {
+          ok = false;
+        } else {
+          tc_fence_after();
+#pragma unroll
+          for (int hc = 0; hc < 2; ++hc) {
+            uint32_t r[32];
+            tmem_ld32(tmem + ((uint32_t)(sub * 32) << 16) + buf * BN + half * 64 + hc * 32, r);
+            tmem_wait_ld();
+            if (hc == 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(smem_u32(&ctl->dempty[buf]));
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) acc[hc * 16 + i] = f2_add(acc[hc * 16 + i], u2(r[2 * i], r[2 * i + 1]));
           }
         }
       }
@@ -359,7 +435,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             float y[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              y[e] = acc[c8 + e] + bb[e];
+              const uint64_t a2 = acc[(c8 + e) >> 1];
+              y[e] = __uint_as_float((e & 1) ? (uint32_t)(a2 >> 32) : (uint32_t)a2) + bb[e];
               if (p.epi == 1) y[e] = gelu_tanh(y[e]);
             }
             uint4 o;

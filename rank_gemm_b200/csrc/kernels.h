@@ -53,8 +53,8 @@ struct K2I8Params {
   int num_m_blocks, num_n_blocks;
   int nk;                  // K_pad / 128 int8 k-tiles (two 64-groups each)
   int nl;                  // ceil(r_tot / 32) low-rank chunks (0: plain W4A4 GEMM)
-  const __half* sX;        // [M_pad128][K_pad/64]
-  const __half* sR;        // [N_pad][K_pad/64]
+  const float* sX;         // binary16 values widened to float32, chunked (int4_scale_offset)
+  const float* sR;
   const float* bias;
   int epi;
   __nv_bfloat16* Y;

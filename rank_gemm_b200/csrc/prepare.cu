@@ -152,7 +152,7 @@ __global__ void quantize_weights_kernel(PrepParams p, float s_tR, float six_st) 
   } else {
     __half sc;
     quant_int4_16of64(v, codes, sc);
-    if ((g & 3) == 0) reinterpret_cast<__half*>(p.sR)[int4_scale_offset(n, g / 4, p.K_pad)] = sc;
+    if ((g & 3) == 0) reinterpret_cast<float*>(p.sR)[int4_scale_offset(n, g / 4, p.K_pad)] = __half2float(sc);
   }
   *reinterpret_cast<uint2*>(p.qR + (size_t)n * (p.K_pad / 2) + k0 / 2) = codes;
 }

@@ -232,7 +232,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       } else {
         __half sc;
         quant_int4_16of64(v, codes, sc);
-        if (qg == 0) reinterpret_cast<__half*>(p.sX)[int4_scale_offset(m, kb, p.K_pad)] = sc;
+        // stored widened to float32 (exact): kernel 2 multiplies in float32
+        if (qg == 0) reinterpret_cast<float*>(p.sX)[int4_scale_offset(m, kb, p.K_pad)] = __half2float(sc);
       }
       if (m < p.M) *reinterpret_cast<uint2*>(p.qX + (size_t)m * qx_row_bytes + (size_t)kb * 32 + qg * 8) = codes;
     }

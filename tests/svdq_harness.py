@@ -58,8 +58,12 @@ def unpack_codes(raw: np.ndarray, rows: int, K: int, K_pad: int, fmt: str) -> np
 
 
 def int4_scales(raw: np.ndarray, rows: int, K: int, K_pad: int) -> np.ndarray:
-    """binary16 scale chunks (128 rows x 2 groups per 128-wide k-tile) -> (rows, K/64)."""
-    h = raw.reshape(-1).view(np.float16)
+    """Scale chunks (128 rows x 2 groups per 128-wide k-tile; binary16 values
+    stored as float32) -> (rows, K/64) float16.  Asserts every stored value is
+    a binary16 value."""
+    f = raw.reshape(-1).view(np.float32)
+    h = f.astype(np.float16)
+    assert np.array_equal(h.astype(np.float32), f), "INT4 scale not a binary16 value"
     r = np.arange(rows)[:, None]
     g = np.arange(K // 64)[None, :]
     off = (((r // 128) * (K_pad // 128) + g // 2) * 2 + g % 2) * 128 + r % 128
@@ -215,7 +219,7 @@ class GpuLayer:
             sraw = read_device(i.sR, i.N_pad * i.K_pad // 16)
             sR = sf_atoms_to_canonical(sraw, self.N, self.K, i.K_pad)
         else:
-            sraw = read_device(i.sR, i.N_pad * (i.K_pad // 64) * 2)
+            sraw = read_device(i.sR, i.N_pad * (i.K_pad // 64) * 4)
             sR = int4_scales(sraw, self.N, self.K, i.K_pad)
         return qR, sR, np.float32(i.s_tR)
 
