@@ -91,6 +91,11 @@ __device__ __forceinline__ void lds2x64(uint32_t addr, uint64_t& a, uint64_t& b)
   asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "r"(addr));
 }
 
+__device__ __forceinline__ void sts128v(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t r;
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
@@ -240,21 +245,29 @@ __global__ void __launch_bounds__(THREADS, 1)
             ok = false;
             break;
           }
-          const uint8_t* src = stg + s * STG_BYTES;
-          uint8_t* dst = mring + t * MMA_BYTES;
+          const uint32_t src = smem_u32(stg + s * STG_BYTES);
+          const uint32_t dst = smem_u32(mring + t * MMA_BYTES);
+          // all loads first, then the permutes and stores (explicit shared-memory
+          // instructions: the generic path is several times slower here)
+          uint4 pk[8];
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {           // h = 0: A (activations), 1: B (weights)
+          for (int h = 0; h < 2; ++h)              // h = 0: A (activations), 1: B (weights)
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const int u = ut + 128 * j, row = u >> 2, c16 = u & 3;
-              const uint4 pk = *reinterpret_cast<const uint4*>(src + h * STG_HALF + row * 64 + c16 * 16);
-              uint4 o0, o1;
-              unpack32(pk, o0, o1);
-              uint8_t* rbase = dst + h * OP_BYTES + row * 128;
-              *reinterpret_cast<uint4*>(rbase + (((2 * c16) ^ (row & 7)) << 4)) = o0;
-              *reinterpret_cast<uint4*>(rbase + (((2 * c16 + 1) ^ (row & 7)) << 4)) = o1;
+              pk[4 * h + j] = lds128(src + h * STG_HALF + row * 64 + c16 * 16);
             }
-          }
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int u = ut + 128 * j, row = u >> 2, c16 = u & 3;
+              uint4 o0, o1;
+              unpack32(pk[4 * h + j], o0, o1);
+              const uint32_t rbase = dst + h * OP_BYTES + row * 128;
+              sts128v(rbase + (((2 * c16) ^ (row & 7)) << 4), o0);
+              sts128v(rbase + (((2 * c16 + 1) ^ (row & 7)) << 4), o1);
+            }
           fence_proxy_async_smem();                // generic-proxy writes -> tensor core
           __syncwarp();
           if (lane == 0) {
