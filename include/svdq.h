@@ -41,8 +41,10 @@
  * Library-defined layouts (svdq_weights_view reports them):
  *   K_pad = K rounded up to a multiple of 256, r_tot = rank + lora_rank,
  *   r_pad = r_tot rounded up to a multiple of 64.
- *   qX    uint8 [M][K_pad/2]: two 4-bit codes per byte, even k in the low
- *         nibble; columns k >= K hold code 0.
+ *   qX    NVFP4: uint8 [M][K_pad/2]: two 4-bit codes per byte, even k in the
+ *         low nibble.  INT4: uint8 [M][K_pad]: every code (-8..7) as its FP8
+ *         E4M3 byte (the operand form of kernel 2's tensor-core product).
+ *         Columns k >= K hold code 0.
  *   sX    NVFP4: E4M3 block scales (one per 16 k), each stored four times
  *         (once per tensor-memory sub-partition, the form kernel 2 copies
  *         into tensor memory): the scale of row r and 16-group g (0..3) of
@@ -95,7 +97,9 @@ typedef struct {
   int fmt;                 /* svdq_format */
   int K, N, rank, lora_rank, r_tot;
   int K_pad, N_pad, r_pad; /* N_pad = N rounded up to a multiple of 256 */
-  const void* qR;          /* dev uint8 [N_pad][K_pad/2], packed like qX (rows = output features) */
+  const void* qR;          /* dev uint8 [N_pad][K_pad/2]: two 4-bit codes per byte, even k in the
+                              low nibble (rows = output features; INT4 kernel 2 reads an E4M3
+                              copy the handle also holds) */
   const void* sR;          /* dev: scales of R, one copy each (NVFP4: 512-byte atoms
                               of 128 rows x 64 k at ((n/128) * (K_pad/64) + k/64) * 512,
                               byte (n % 32) * 16 + ((n % 128) / 32) * 4 + (k % 64) / 16;

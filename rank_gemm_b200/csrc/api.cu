@@ -29,6 +29,7 @@ struct svdq_weights {
   uint8_t* qR;
   uint8_t* sR;
   uint8_t* sR_rep;   // NVFP4: kernel 2's replicated copy of sR
+  uint8_t* qR8;      // INT4: kernel 2's copy of qR, one E4M3 byte per code [N_pad][K_pad]
   __nv_bfloat16* L1t;
   __nv_bfloat16* L2a;
   float* bias_f;
@@ -36,7 +37,7 @@ struct svdq_weights {
   float* lambda_inv_k1;
   float s_tR, s_tX, alpha;
   CUtensorMap tm_qR, tm_L2a;
-  CUtensorMap tm_qR_i4, tm_L2a_i4;   // INT4 kernel: packed 64-byte rows / 32-column low-rank chunks
+  CUtensorMap tm_qR8, tm_L2a_i4;      // INT4 kernel: E4M3 codes and L2a in 128-row boxes
 };
 
 namespace {
@@ -132,7 +133,10 @@ bool tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t i
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-size_t qx_bytes(const svdq_weights* w, int M) { return (size_t)M * (w->K_pad / 2); }
+// NVFP4: packed codes; INT4: one E4M3 byte per code
+size_t qx_bytes(const svdq_weights* w, int M) {
+  return (size_t)M * (w->fmt == SVDQ_NVFP4 ? w->K_pad / 2 : w->K_pad);
+}
 size_t sx_bytes(const svdq_weights* w, int M) {
   const size_t rows = (size_t)round_up(M, 128);
   // NVFP4: four replicas of every scale word (see sfx_rep_offset)
@@ -191,11 +195,11 @@ svdq_status run_k2(const svdq_weights* w, int M, const void* qX, const void* sX,
   std::memset(&tmLR, 0, sizeof(tmLR));
   const bool nv = w->fmt == SVDQ_NVFP4;
   if (lowrank && !tmap_2d(&tmLR, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, LR, w->r_pad, M, (uint64_t)w->r_pad * 2,
-                          nv ? 64 : 32, 128, nv ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
+                          64, nv ? K2_NV_ROWS_A : K2_I4_ROWS))
     return SVDQ_ERR_CUDA;
   if (nv) {
     CUtensorMap tmA;
-    if (!tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, qX, w->K_pad / 2, M, w->K_pad / 2, 128, 128))
+    if (!tmap_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, qX, w->K_pad / 2, M, w->K_pad / 2, 128, K2_NV_ROWS_A))
       return SVDQ_ERR_CUDA;
     K2Params p;
     p.M = M;
@@ -217,9 +221,8 @@ svdq_status run_k2(const svdq_weights* w, int M, const void* qX, const void* sX,
     p.err = dev_err(d);
     return from_cuda(launch_gemm_nvfp4(tmA, w->tm_qR, tmLR, w->tm_L2a, p, d->num_sms, stream));
   }
-  CUtensorMap tmXp;
-  if (!tmap_2d(&tmXp, CU_TENSOR_MAP_DATA_TYPE_UINT8, qX, w->K_pad / 2, M, w->K_pad / 2, 64, 128,
-               CU_TENSOR_MAP_SWIZZLE_NONE))
+  CUtensorMap tmX8;
+  if (!tmap_2d(&tmX8, CU_TENSOR_MAP_DATA_TYPE_UINT8, qX, w->K_pad, M, w->K_pad, 128, K2_I4_ROWS))
     return SVDQ_ERR_CUDA;
   K2I8Params p;
   p.M = M;
@@ -231,20 +234,21 @@ svdq_status run_k2(const svdq_weights* w, int M, const void* qX, const void* sX,
   p.num_m_blocks = (M + 127) / 128;
   p.num_n_blocks = w->N_pad / 128;   // the INT4 kernel's tiles are 128 wide
   p.nk = w->K_pad / 128;
-  p.nl = lowrank ? (w->r_tot + 31) / 32 : 0;
+  p.nl = lowrank ? w->r_pad / 64 : 0;
   p.sX = static_cast<const float*>(sX);
   p.sR = reinterpret_cast<const float*>(w->sR);
   p.bias = w->bias_f;
   p.epi = (int)epi;
   p.Y = static_cast<__nv_bfloat16*>(Y);
   p.err = dev_err(d);
-  return from_cuda(launch_gemm_int4(tmXp, w->tm_qR_i4, tmLR, w->tm_L2a_i4, p, d->num_sms, stream));
+  return from_cuda(launch_gemm_int4(tmX8, w->tm_qR8, tmLR, w->tm_L2a_i4, p, d->num_sms, stream));
 }
 
 void free_buffers(svdq_weights* w) {
   cudaFree(w->qR);
   cudaFree(w->sR);
   cudaFree(w->sR_rep);
+  cudaFree(w->qR8);
   cudaFree(w->L1t);
   cudaFree(w->L2a);
   cudaFree(w->bias_f);
@@ -334,6 +338,7 @@ svdq_status svdq_prepare_weights(svdq_format fmt, int K, int N, int rank, const 
   unsigned* amax = nullptr;
   bool ok = cudaMalloc(&w->qR, qr_b) == cudaSuccess && cudaMalloc(&w->sR, sr_b) == cudaSuccess &&
             (fmt != SVDQ_NVFP4 || cudaMalloc(&w->sR_rep, 4 * sr_b) == cudaSuccess) &&
+            (fmt != SVDQ_INT4 || cudaMalloc(&w->qR8, 2 * qr_b) == cudaSuccess) &&
             cudaMalloc(&w->L1t, (size_t)r_tot * w->K_pad * 2) == cudaSuccess &&
             cudaMalloc(&w->L2a, (size_t)w->N_pad * w->r_pad * 2) == cudaSuccess &&
             cudaMalloc(&w->bias_f, (size_t)w->N_pad * 4) == cudaSuccess &&
@@ -370,6 +375,7 @@ svdq_status svdq_prepare_weights(svdq_format fmt, int K, int N, int rank, const 
   p.qR = w->qR;
   p.sR = w->sR;
   p.sR_rep = w->sR_rep;
+  p.qR8 = w->qR8;
   p.L1t = w->L1t;
   p.L2a = w->L2a;
   p.bias_f = w->bias_f;
@@ -406,13 +412,13 @@ svdq_status svdq_prepare_weights(svdq_format fmt, int K, int N, int rank, const 
   cudaFree(amax);
   bool maps = e == cudaSuccess &&
               tmap_2d(&w->tm_qR, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->qR, w->K_pad / 2, w->N_pad, w->K_pad / 2,
-                      128, 256) &&
+                      128, K2_NV_ROWS_B) &&
               tmap_2d(&w->tm_L2a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->L2a, w->r_pad, w->N_pad,
-                      (uint64_t)w->r_pad * 2, 64, 256) &&
-              tmap_2d(&w->tm_qR_i4, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->qR, w->K_pad / 2, w->N_pad, w->K_pad / 2,
-                      64, 128, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                      (uint64_t)w->r_pad * 2, 64, K2_NV_ROWS_B) &&
               tmap_2d(&w->tm_L2a_i4, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->L2a, w->r_pad, w->N_pad,
-                      (uint64_t)w->r_pad * 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B);
+                      (uint64_t)w->r_pad * 2, 64, K2_I4_ROWS) &&
+              (fmt != SVDQ_INT4 || tmap_2d(&w->tm_qR8, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->qR8, w->K_pad, w->N_pad,
+                                           w->K_pad, 128, K2_I4_ROWS));
   if (!maps) {
     free_buffers(w);
     delete w;

@@ -513,6 +513,30 @@ __device__ __forceinline__ void quant_int4_16of64(const float (&v)[16], uint2& c
   scale = sb;
 }
 
+// INT4 codes in FP8 E4M3 containers (E4M3 holds -8..7 exactly), the operand
+// form of the INT4 tensor-core product.  Table: E4M3 bytes of the two's
+// complement codes 0..7 (values 0..7) and 8..15 (values -8..-1), code c at
+// byte c % 4 of its word.
+constexpr uint32_t E4M3_POS_LO = 0x44403800u, E4M3_POS_HI = 0x4E4C4A48u;   // 0, 1, 2, 3 | 4, 5, 6, 7
+constexpr uint32_t E4M3_NEG_LO = 0xCACCCED0u, E4M3_NEG_HI = 0xB8C0C4C8u;   // -8, -7, -6, -5 | -4, -3, -2, -1
+__device__ __forceinline__ uint32_t prmt_b32(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+// The four codes in the low 16 bits of sel (k order, low nibble first) ->
+// four E4M3 bytes (k order): look up code & 7 in both halves of the table,
+// then pick per byte by bit 3 of the code.
+__device__ __forceinline__ uint32_t int4x4_to_e4m3(uint32_t sel) {
+  const uint32_t s7 = sel & 0x7777u;
+  const uint32_t pos = prmt_b32(E4M3_POS_LO, E4M3_POS_HI, s7), neg = prmt_b32(E4M3_NEG_LO, E4M3_NEG_HI, s7);
+  return prmt_b32(pos, neg, ((sel >> 1) & 0x4444u) | 0x3210u);
+}
+// 16 packed codes (8 bytes, element 2j in the low nibble of byte j) -> 16 E4M3 bytes.
+__device__ __forceinline__ uint4 int4x16_to_e4m3(uint2 c) {
+  return make_uint4(int4x4_to_e4m3(c.x), int4x4_to_e4m3(c.x >> 16), int4x4_to_e4m3(c.y), int4x4_to_e4m3(c.y >> 16));
+}
+
 // Byte offset of (row, 16-group) inside the tcgen05 scale-factor layout:
 // 512-byte atoms of 128 rows x 4 groups, ordered (row block, 64-k block).
 __host__ __device__ __forceinline__ size_t sf_atom_offset(int row, int g16, int kpad) {

@@ -1,28 +1,29 @@
 // gemm_int4.cu -- kernel 2 for INT4: the 4-bit GEMM fused with the low-rank up
 // projection ("Nunchaku engine design" figure (b), "svdq-int4-flux.1-dev" model
-// card), on the int8 tensor-core path.
+// card), on the FP8 tensor-core path.
 //
 // INT4 block scales are binary16 per 64 elements, which no block-scaled MMA
 // kind can take, so each 64-group is its own product:
 //     y[m,n] = sum_g sX[m,g] sR[n,g] (sum_{k in g} qX[m,k] qR[n,k]) + LR[m,:] L2[n,:] + b[n]
-// The int4 codes (-8..7) are unpacked in shared memory to FP8 E4M3, which
-// holds them exactly; every group runs as two tcgen05.mma.kind::f8f6f4
-// (K = 32) into a fresh fp32 TMEM tile, whose sums (|.| <= 64 * 64) are exact,
-// so the group product needs no integer-to-float conversion.  CUDA cores apply
-// sX sR and accumulate in fp32 registers with packed (f32x2) multiply and FMA:
-// one instruction per output element per group, the bound of this kernel.
+// The codes (-8..7) reach this kernel as FP8 E4M3 bytes, which hold them
+// exactly (kernel 1 writes the activations that way; the weights handle keeps
+// an E4M3 copy next to the packed codes), so TMA stages them straight into
+// the operand tiles.  Every group runs as two tcgen05.mma.kind::f8f6f4
+// (K = 32) into a fresh fp32 TMEM tile, whose sums (|.| <= 64 * 64) are exact;
+// CUDA cores apply sX sR and accumulate in fp32 registers with packed f32x2
+// multiply and FMA, one instruction per output element per group: the bound
+// of this kernel.  (A first version unpacked packed int4 tiles in shared
+// memory for every output tile; that byte shuffling set its pace.)
 //
 // One 128 x 128 output tile per CTA at a time, persistent over tiles:
-//   warp 0       TMA producer: packed int4 tiles of qX and qR (128 rows x 64 B
-//                per 128-wide k-tile) into a staging ring, the k-tile's scale
-//                chunks of both (1 KB each) into a scale ring, then the
-//                low-rank chunks (LR and L2, 32 columns, 64-byte swizzle).
-//   warps 1-4    unpack: staging int4 -> E4M3 operand tiles (128-byte
-//                swizzle) in the MMA ring, three byte permutes per 4 codes.
-//   warp 5       TMEM owner and MMA issuer (per group into one of four TMEM
-//                buffers; the low-rank chunks as kind::f16 straight from the
-//                staging ring into one more buffer use).
-//   warps 6-13   rescale + epilogue: 2 warps per TMEM sub-partition, 64 columns
+//   warp 0       TMA producer: per 128-wide k-tile the [128 x 128 B] E4M3
+//                tiles of qX and qR (128-byte swizzle) into the operand ring
+//                and the k-tile's scale chunks of both (1 KB each) into a
+//                scale ring; then the low-rank chunks (LR and L2, 64 columns).
+//   warp 1       TMEM owner and MMA issuer (per group into one of four TMEM
+//                buffers; the low-rank chunks as kind::f16 into one more
+//                buffer use).
+//   warps 2-9    rescale + epilogue: 2 warps per TMEM sub-partition, 64 columns
 //                each; fp32 accumulators in registers; bias, GELU, bf16 store.
 #include "common.cuh"
 #include "kernels.h"
@@ -31,18 +32,15 @@ namespace svdq {
 
 namespace {
 
-constexpr int BM = 128, BN = 128;
-constexpr int ST = 6;                    // staging ring (packed int4 / low-rank chunks)
-constexpr int MS = 3;                    // MMA ring (E4M3 tiles)
+constexpr int BM = K2_I4_ROWS, BN = K2_I4_ROWS;
+constexpr int MS = 6;                    // operand ring: E4M3 k-tiles / bf16 low-rank chunks
 constexpr int SC = 8;                    // scale ring (one k-tile's scales of qX and qR)
-constexpr int STG_HALF = 8192;           // packed [128 x 64 B] or bf16 [128 x 32]
-constexpr int STG_BYTES = 2 * STG_HALF;
-constexpr int OP_BYTES = 16384;          // E4M3 [128 x 128 B]
-constexpr int MMA_BYTES = 2 * OP_BYTES;
+constexpr int OP_BYTES = 16384;          // E4M3 [128 x 128 B] or bf16 [128 x 64]
+constexpr int STAGE_BYTES = 2 * OP_BYTES;
 constexpr int SC_HALF = 1024;            // float32 [2 groups][128 rows]
 constexpr int SC_BYTES = 2 * SC_HALF;
-constexpr int WARPS = 14, THREADS = WARPS * 32;
-constexpr int W_UNPACK = 1, W_MMA = 5, W_RESCALE = 6;
+constexpr int W_MMA = 1, W_RESCALE = 2;
+constexpr int THREADS = (W_RESCALE + 8) * 32;
 constexpr int NBUF = 4;                  // TMEM group buffers of BN columns
 constexpr uint32_t TMEM_COLS = NBUF * BN;
 // kind::f8f6f4: fp32 D, E4M3 A and B (format code 0), K-major
@@ -50,13 +48,11 @@ constexpr uint32_t IDESC_F8 = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32
 constexpr uint32_t IDESC_BF = idesc_bf16_f32(BM, BN);
 
 struct Ctl {
-  uint64_t sfull[ST], sempty[ST], mfull[MS], mempty[MS], cfull[SC], cempty[SC], dfull[NBUF], dempty[NBUF];
-  uint32_t unpack_done[ST];
+  uint64_t full[MS], empty[MS], cfull[SC], cempty[SC], dfull[NBUF], dempty[NBUF];
   uint32_t tmem_base;
   int abort;
 };
-constexpr size_t SMEM_BYTES =
-    (size_t)ST * STG_BYTES + (size_t)MS * MMA_BYTES + (size_t)SC * SC_BYTES + 1024 + sizeof(Ctl);
+constexpr size_t SMEM_BYTES = (size_t)MS * STAGE_BYTES + (size_t)SC * SC_BYTES + 1024 + sizeof(Ctl);
 
 __device__ __forceinline__ void mma_f8(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
   asm volatile(
@@ -66,9 +62,6 @@ __device__ __forceinline__ void mma_f8(uint32_t d, uint64_t a, uint64_t b, uint3
       "l"(a), "l"(b), "r"(idesc), "r"(acc)
       : "memory");
 }
-
-// K-major bf16 tile with 64-byte rows in the 64-byte swizzle (8-row groups 512 B apart).
-__device__ __forceinline__ uint64_t desc_k_sw64(uint32_t addr) { return smem_desc(addr, 16, 512, 4); }
 
 // Packed float32 pairs kept in 64-bit registers (element 0 in the low half).
 __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
@@ -91,40 +84,6 @@ __device__ __forceinline__ void lds2x64(uint32_t addr, uint64_t& a, uint64_t& b)
   asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "r"(addr));
 }
 
-__device__ __forceinline__ void sts128v(uint32_t addr, uint4 v) {
-  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-               : "memory");
-}
-
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t r;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
-  return r;
-}
-// E4M3 bytes of the int4 codes 0..7 (values 0..7) and 8..15 (values -8..-1),
-// four per word, code c at byte c % 4.
-constexpr uint32_t E4M3_POS_LO = 0x44403800u, E4M3_POS_HI = 0x4E4C4A48u;   // 0, 1, 2, 3 | 4, 5, 6, 7
-constexpr uint32_t E4M3_NEG_LO = 0xCACCCED0u, E4M3_NEG_HI = 0xB8C0C4C8u;   // -8, -7, -6, -5 | -4, -3, -2, -1
-// Four codes (the 4 nibbles of sel, in k order) -> four E4M3 bytes: look up
-// code & 7 in both halves of the table, then pick per byte by bit 3.
-__device__ __forceinline__ uint32_t e4m3x4(uint32_t sel) {
-  const uint32_t s7 = sel & 0x7777u;
-  const uint32_t pos = prmt(E4M3_POS_LO, E4M3_POS_HI, s7), neg = prmt(E4M3_NEG_LO, E4M3_NEG_HI, s7);
-  return prmt(pos, neg, ((sel >> 1) & 0x4444u) | 0x3210u);
-}
-// 16 packed bytes (32 int4, element 2j in the low nibble of byte j) -> 32 E4M3 bytes.
-__device__ __forceinline__ void unpack32(const uint4 p, uint4& o0, uint4& o1) {
-  const uint32_t w[4] = {p.x, p.y, p.z, p.w};
-  uint32_t o[8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    o[2 * i] = e4m3x4(w[i] & 0xFFFFu);
-    o[2 * i + 1] = e4m3x4(w[i] >> 16);
-  }
-  o0 = make_uint4(o[0], o[1], o[2], o[3]);
-  o1 = make_uint4(o[4], o[5], o[6], o[7]);
-}
-
 __device__ __forceinline__ float gelu_tanh(float y) {
   const float u = 0.7978845608028654f * (y + 0.044715f * y * y * y);
   return 0.5f * y * (1.f + tanhf(u));
@@ -138,33 +97,27 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }  // namespace
 
 __global__ void __launch_bounds__(THREADS, 1)
-    gemm_int4_kernel(const __grid_constant__ CUtensorMap tmXp, const __grid_constant__ CUtensorMap tmRp,
+    gemm_int4_kernel(const __grid_constant__ CUtensorMap tmX8, const __grid_constant__ CUtensorMap tmR8,
                      const __grid_constant__ CUtensorMap tmLR, const __grid_constant__ CUtensorMap tmL2,
                      K2I8Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* stg = base;                              // ST x 16 KB
-  uint8_t* mring = base + ST * STG_BYTES;           // MS x 32 KB
-  uint8_t* sring = mring + MS * MMA_BYTES;          // SC x 2 KB
+  uint8_t* ring = base;                             // MS x 32 KB
+  uint8_t* sring = ring + MS * STAGE_BYTES;         // SC x 2 KB
   Ctl* ctl = reinterpret_cast<Ctl*>(sring + SC * SC_BYTES);
   volatile int* abort_flag = &ctl->abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    tma_prefetch_desc(&tmXp);
-    tma_prefetch_desc(&tmRp);
+    tma_prefetch_desc(&tmX8);
+    tma_prefetch_desc(&tmR8);
     if (p.nl) {
       tma_prefetch_desc(&tmLR);
       tma_prefetch_desc(&tmL2);
     }
-    for (int s = 0; s < ST; ++s) {
-      mbar_init(smem_u32(&ctl->sfull[s]), 1);
-      mbar_init(smem_u32(&ctl->sempty[s]), 1);
-      ctl->unpack_done[s] = 0;
-    }
     for (int s = 0; s < MS; ++s) {
-      mbar_init(smem_u32(&ctl->mfull[s]), 4);
-      mbar_init(smem_u32(&ctl->mempty[s]), 1);
+      mbar_init(smem_u32(&ctl->full[s]), 1);
+      mbar_init(smem_u32(&ctl->empty[s]), 1);
     }
     for (int c = 0; c < SC; ++c) {
       mbar_init(smem_u32(&ctl->cfull[c]), 1);
@@ -198,15 +151,15 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
         const int mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
         for (int it = 0; it < nk + nl; ++it) {
-          if (!mbar_wait(smem_u32(&ctl->sempty[s]), ph ^ 1, abort_flag, p.err)) {
+          if (!mbar_wait(smem_u32(&ctl->empty[s]), ph ^ 1, abort_flag, p.err)) {
             ok = false;
             break;
           }
-          const uint32_t dst = smem_u32(stg + s * STG_BYTES), bar = smem_u32(&ctl->sfull[s]);
-          mbar_arrive_expect_tx(bar, STG_BYTES);
+          const uint32_t dst = smem_u32(ring + s * STAGE_BYTES), bar = smem_u32(&ctl->full[s]);
+          mbar_arrive_expect_tx(bar, STAGE_BYTES);
           if (it < nk) {
-            tma_load_2d(dst, &tmXp, it * 64, mb * BM, bar);
-            tma_load_2d(dst + STG_HALF, &tmRp, it * 64, nb * BN, bar);
+            tma_load_2d(dst, &tmX8, it * 128, mb * BM, bar);
+            tma_load_2d(dst + OP_BYTES, &tmR8, it * 128, nb * BN, bar);
             // the k-tile's scale chunks: 128 rows x 2 groups of float32 each
             if (!mbar_wait(smem_u32(&ctl->cempty[c]), cph ^ 1, abort_flag, p.err)) {
               ok = false;
@@ -221,88 +174,30 @@ __global__ void __launch_bounds__(THREADS, 1)
               cph ^= 1;
             }
           } else {
-            tma_load_2d(dst, &tmLR, (it - nk) * 32, mb * BM, bar);
-            tma_load_2d(dst + STG_HALF, &tmL2, (it - nk) * 32, nb * BN, bar);
+            tma_load_2d(dst, &tmLR, (it - nk) * 64, mb * BM, bar);
+            tma_load_2d(dst + OP_BYTES, &tmL2, (it - nk) * 64, nb * BN, bar);
           }
-          if (++s == ST) {
+          if (++s == MS) {
             s = 0;
             ph ^= 1;
           }
         }
       }
     }
-  } else if (warp >= W_UNPACK && warp < W_MMA) {
-    // ---------------------------------------------------------------- unpack
-    const int ut = threadIdx.x - W_UNPACK * 32;      // 0..127
-    int s = 0, t = 0;
-    uint32_t sph = 0, mph = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-      for (int it = 0; it < nk + nl; ++it) {
-        if (it < nk) {
-          if (!mbar_wait(smem_u32(&ctl->sfull[s]), sph, abort_flag, p.err) ||
-              !mbar_wait(smem_u32(&ctl->mempty[t]), mph ^ 1, abort_flag, p.err)) {
-            ok = false;
-            break;
-          }
-          const uint32_t src = smem_u32(stg + s * STG_BYTES);
-          const uint32_t dst = smem_u32(mring + t * MMA_BYTES);
-          // all loads first, then the permutes and stores (explicit shared-memory
-          // instructions: the generic path is several times slower here)
-          uint4 pk[8];
-#pragma unroll
-          for (int h = 0; h < 2; ++h)              // h = 0: A (activations), 1: B (weights)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int u = ut + 128 * j, row = u >> 2, c16 = u & 3;
-              pk[4 * h + j] = lds128(src + h * STG_HALF + row * 64 + c16 * 16);
-            }
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int u = ut + 128 * j, row = u >> 2, c16 = u & 3;
-              uint4 o0, o1;
-              unpack32(pk[4 * h + j], o0, o1);
-              const uint32_t rbase = dst + h * OP_BYTES + row * 128;
-              sts128v(rbase + (((2 * c16) ^ (row & 7)) << 4), o0);
-              sts128v(rbase + (((2 * c16 + 1) ^ (row & 7)) << 4), o1);
-            }
-          fence_proxy_async_smem();                // generic-proxy writes -> tensor core
-          __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(smem_u32(&ctl->mfull[t]));
-            // the last of the four unpack warps to finish releases the staging slot
-            if (atomicAdd(&ctl->unpack_done[s], 1u) == 3u) {
-              ctl->unpack_done[s] = 0;
-              mbar_arrive(smem_u32(&ctl->sempty[s]));
-            }
-          }
-          if (++t == MS) {
-            t = 0;
-            mph ^= 1;
-          }
-        }
-        if (++s == ST) {
-          s = 0;
-          sph ^= 1;
-        }
-      }
-    }
   } else if (warp == W_MMA) {
     if (lane == 0) {
       // -------------------------------------------------------------- MMA issuer
-      int s = 0, t = 0;
-      uint32_t sph = 0, mph = 0, uses = 0;
+      int s = 0;
+      uint32_t ph = 0, uses = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
         for (int it = 0; ok && it < nk; ++it) {
-          if (!mbar_wait(smem_u32(&ctl->mfull[t]), mph, abort_flag, p.err)) {
+          if (!mbar_wait(smem_u32(&ctl->full[s]), ph, abort_flag, p.err)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a = smem_u32(mring + t * MMA_BYTES), b = a + OP_BYTES;
+          const uint32_t a = smem_u32(ring + s * STAGE_BYTES), b = a + OP_BYTES;
           for (int j = 0; j < 2; ++j, ++uses) {
             const uint32_t buf = uses % NBUF, dph = (uses / NBUF) & 1;
             if (!mbar_wait(smem_u32(&ctl->dempty[buf]), dph ^ 1, abort_flag, p.err)) {
@@ -316,14 +211,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc_commit(smem_u32(&ctl->dfull[buf]));
           }
           if (!ok) break;
-          tc_commit(smem_u32(&ctl->mempty[t]));
-          if (++t == MS) {
-            t = 0;
-            mph ^= 1;
-          }
-          if (++s == ST) {
+          tc_commit(smem_u32(&ctl->empty[s]));
+          if (++s == MS) {
             s = 0;
-            sph ^= 1;
+            ph ^= 1;
           }
         }
         if (!ok) break;
@@ -331,20 +222,20 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t buf = uses % NBUF, dph = (uses / NBUF) & 1;
           if (!mbar_wait(smem_u32(&ctl->dempty[buf]), dph ^ 1, abort_flag, p.err)) break;
           for (int c = 0; c < nl; ++c) {
-            if (!mbar_wait(smem_u32(&ctl->sfull[s]), sph, abort_flag, p.err)) {
+            if (!mbar_wait(smem_u32(&ctl->full[s]), ph, abort_flag, p.err)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint32_t a = smem_u32(stg + s * STG_BYTES), b = a + STG_HALF;
-            const int steps = min(2, (p.r_tot - 32 * c) / 16);
+            const uint32_t a = smem_u32(ring + s * STAGE_BYTES), b = a + OP_BYTES;
+            const int steps = min(4, (p.r_tot - 64 * c) / 16);
             for (int j = 0; j < steps; ++j)
-              mma_bf16(tmem + buf * BN, desc_k_sw64(a + 32 * j), desc_k_sw64(b + 32 * j), IDESC_BF,
+              mma_bf16(tmem + buf * BN, desc_k_sw128(a + 32 * j), desc_k_sw128(b + 32 * j), IDESC_BF,
                        (c | j) != 0);
-            tc_commit(smem_u32(&ctl->sempty[s]));
-            if (++s == ST) {
+            tc_commit(smem_u32(&ctl->empty[s]));
+            if (++s == MS) {
               s = 0;
-              sph ^= 1;
+              ph ^= 1;
             }
           }
           if (!ok) break;
@@ -472,14 +363,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-cudaError_t launch_gemm_int4(const CUtensorMap& tmXp, const CUtensorMap& tmRp, const CUtensorMap& tmLR,
+cudaError_t launch_gemm_int4(const CUtensorMap& tmX8, const CUtensorMap& tmR8, const CUtensorMap& tmLR,
                              const CUtensorMap& tmL2, K2I8Params p, int num_sms, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int tiles = p.num_m_blocks * p.num_n_blocks;
   const int grid = tiles < num_sms ? tiles : num_sms;
-  gemm_int4_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tmXp, tmRp, tmLR, tmL2, p);
+  gemm_int4_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tmX8, tmR8, tmLR, tmL2, p);
   return cudaGetLastError();
 }
 

@@ -34,7 +34,7 @@ namespace svdq {
 
 namespace {
 
-constexpr int BLOCK_M = 128, BLOCK_N = 256, STAGES = 3;
+constexpr int BLOCK_M = K2_NV_ROWS_A, BLOCK_N = K2_NV_ROWS_B, STAGES = 3;
 constexpr int A_BYTES = BLOCK_M * 128;          // 16 KB
 constexpr int B_BYTES = BLOCK_N * 128;          // 32 KB
 constexpr int SF_BLOCK = 4096;                  // one replicated scale block (8 TMEM columns)

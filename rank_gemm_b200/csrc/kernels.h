@@ -44,6 +44,11 @@ struct K2Params {
   __nv_bfloat16* Y;        // [M][N]
   DeviceErr err;
 };
+// TMA box heights the host encodes for kernel 2's operands (rows of a tile):
+// NVFP4 stages 128 rows of qX / LR and 256 rows of qR / L2a per k-tile; INT4
+// stages 128 of each.
+constexpr int K2_NV_ROWS_A = 128, K2_NV_ROWS_B = 256;
+constexpr int K2_I4_ROWS = 128;
 cudaError_t launch_gemm_nvfp4(const CUtensorMap& tmA, const CUtensorMap& tmB,
                               const CUtensorMap& tmLR, const CUtensorMap& tmL2, K2Params p,
                               int num_sms, cudaStream_t stream);
@@ -51,8 +56,8 @@ cudaError_t launch_gemm_nvfp4(const CUtensorMap& tmA, const CUtensorMap& tmB,
 struct K2I8Params {
   int M, N, K_pad, r_tot, r_pad, N_pad;
   int num_m_blocks, num_n_blocks;
-  int nk;                  // K_pad / 128 int8 k-tiles (two 64-groups each)
-  int nl;                  // ceil(r_tot / 32) low-rank chunks (0: plain W4A4 GEMM)
+  int nk;                  // K_pad / 128 k-tiles (two 64-groups each)
+  int nl;                  // r_pad / 64 low-rank chunks (0: plain W4A4 GEMM)
   const float* sX;         // binary16 values widened to float32, chunked (int4_scale_offset)
   const float* sR;
   const float* bias;
@@ -60,7 +65,7 @@ struct K2I8Params {
   __nv_bfloat16* Y;
   DeviceErr err;
 };
-cudaError_t launch_gemm_int4(const CUtensorMap& tmXp, const CUtensorMap& tmRp, const CUtensorMap& tmLR,
+cudaError_t launch_gemm_int4(const CUtensorMap& tmX8, const CUtensorMap& tmR8, const CUtensorMap& tmLR,
                              const CUtensorMap& tmL2, K2I8Params p, int num_sms, cudaStream_t stream);
 
 // ---------------------------------------------------------------- unfused up projection
@@ -93,6 +98,7 @@ struct PrepParams {
   uint8_t* qR;                 // [N_pad][K_pad/2]
   uint8_t* sR;                 // scales
   uint8_t* sR_rep;             // NVFP4: kernel 2's replicated copy (sfw_rep_offset)
+  uint8_t* qR8;                // INT4: kernel 2's copy of the codes as E4M3 bytes [N_pad][K_pad]
   __nv_bfloat16* L1t;          // [K_pad/64][r_tot][64], 128-byte swizzled
   __nv_bfloat16* L2a;          // [N_pad][r_pad]
   float* bias_f;               // [N_pad]

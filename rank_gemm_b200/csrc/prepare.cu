@@ -155,6 +155,7 @@ __global__ void quantize_weights_kernel(PrepParams p, float s_tR, float six_st) 
     if ((g & 3) == 0) reinterpret_cast<float*>(p.sR)[int4_scale_offset(n, g / 4, p.K_pad)] = __half2float(sc);
   }
   *reinterpret_cast<uint2*>(p.qR + (size_t)n * (p.K_pad / 2) + k0 / 2) = codes;
+  if (p.qR8) *reinterpret_cast<uint4*>(p.qR8 + (size_t)n * p.K_pad + k0) = int4x16_to_e4m3(codes);
 }
 
 __global__ void factors_kernel(PrepParams p, float alpha) {

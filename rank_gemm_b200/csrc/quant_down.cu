@@ -191,7 +191,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int qw = warp - W_Q0;
     const int qb = qw & 1, qr = (qw >> 1) * 8 + (lane >> 2), qg = lane & 3;
     const int m = m0 + qr;
-    const size_t qx_row_bytes = (size_t)(p.K_pad / 2);
+    // NVFP4: packed codes (K_pad / 2 bytes a row); INT4: one E4M3 byte per code
+    const size_t qx_row_bytes = p.fmt == 0 ? (size_t)(p.K_pad / 2) : (size_t)p.K_pad;
     for (int it = 0; it < ns; ++it) {
       const int s = it % p.stages;
       if (!mbar_wait(smem_u32(&full[s]), (it / p.stages) & 1, abort_flag, p.err)) break;
@@ -235,7 +236,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         // stored widened to float32 (exact): kernel 2 multiplies in float32
         if (qg == 0) reinterpret_cast<float*>(p.sX)[int4_scale_offset(m, kb, p.K_pad)] = __half2float(sc);
       }
-      if (m < p.M) *reinterpret_cast<uint2*>(p.qX + (size_t)m * qx_row_bytes + (size_t)kb * 32 + qg * 8) = codes;
+      if (m < p.M) {
+        if (p.fmt == 0)
+          *reinterpret_cast<uint2*>(p.qX + (size_t)m * qx_row_bytes + (size_t)kb * 32 + qg * 8) = codes;
+        else
+          *reinterpret_cast<uint4*>(p.qX + (size_t)m * qx_row_bytes + (size_t)kb * 64 + qg * 16) = int4x16_to_e4m3(codes);
+      }
     }
   }
 

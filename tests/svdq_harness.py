@@ -52,9 +52,21 @@ def sfx_replicated_to_canonical(raw: np.ndarray, rows: int, K: int, K_pad: int) 
 
 
 def unpack_codes(raw: np.ndarray, rows: int, K: int, K_pad: int, fmt: str) -> np.ndarray:
+    """Weights (both formats) and NVFP4 activations: packed nibbles."""
     b = raw.reshape(-1)[: rows * (K_pad // 2)].reshape(rows, K_pad // 2)
     c = F.unpack_nibbles(b)[:, :K]
     return c if fmt == "nvfp4" else F.int4_from_nibble(c)
+
+
+def int4_act_codes(raw: np.ndarray, rows: int, K: int, K_pad: int) -> np.ndarray:
+    """INT4 activations as kernel 1 writes them: one E4M3 byte per code
+    [rows][K_pad] -> signed codes (rows, K).  Asserts every byte is an E4M3
+    integer in [-8, 7] and the pad columns hold code 0."""
+    b = raw.reshape(-1)[: rows * K_pad].reshape(rows, K_pad)
+    v = F.e4m3_decode(b)
+    assert np.all(v == np.rint(v)) and v.min() >= -8 and v.max() <= 7, "INT4 activation byte not a code"
+    assert np.all(v[:, K:] == 0)
+    return v[:, :K].astype(np.int8)
 
 
 def int4_scales(raw: np.ndarray, rows: int, K: int, K_pad: int) -> np.ndarray:
@@ -237,7 +249,10 @@ class GpuLayer:
 
     def decode_act(self, qX, sX, LR, M):
         i = self.info
-        q = unpack_codes(to_np(qX), M, self.K, i.K_pad, self.fmt)
+        if self.fmt == "nvfp4":
+            q = unpack_codes(to_np(qX), M, self.K, i.K_pad, self.fmt)
+        else:
+            q = int4_act_codes(to_np(qX), M, self.K, i.K_pad)
         if self.fmt == "nvfp4":
             s = sfx_replicated_to_canonical(to_np(sX), M, self.K, i.K_pad)
         else:
