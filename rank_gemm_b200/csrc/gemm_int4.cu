@@ -23,7 +23,7 @@
 //   warp 1       TMEM owner and MMA issuer (per group into one of four TMEM
 //                buffers; the low-rank chunks as kind::f16 into one more
 //                buffer use).
-//   warps 2-9    rescale + epilogue: 2 warps per TMEM sub-partition, 64 columns
+//   warps 2-17   rescale + epilogue: 4 warps per TMEM sub-partition, 32 columns
 //                each; fp32 accumulators in registers; bias, GELU, bf16 store.
 #include "common.cuh"
 #include "kernels.h"
@@ -40,7 +40,9 @@ constexpr int STAGE_BYTES = 2 * OP_BYTES;
 constexpr int SC_HALF = 1024;            // float32 [2 groups][128 rows]
 constexpr int SC_BYTES = 2 * SC_HALF;
 constexpr int W_MMA = 1, W_RESCALE = 2;
-constexpr int THREADS = (W_RESCALE + 8) * 32;
+constexpr int RS_WARPS = 16;             // four per TMEM sub-partition, 32 columns each
+constexpr int RS_COLS = BN / (RS_WARPS / 4);
+constexpr int THREADS = (W_RESCALE + RS_WARPS) * 32;
 constexpr int NBUF = 4;                  // TMEM group buffers of BN columns
 constexpr uint32_t TMEM_COLS = NBUF * BN;
 // kind::f8f6f4: fp32 D, E4M3 A and B (format code 0), K-major
@@ -121,11 +123,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int c = 0; c < SC; ++c) {
       mbar_init(smem_u32(&ctl->cfull[c]), 1);
-      mbar_init(smem_u32(&ctl->cempty[c]), 8);
+      mbar_init(smem_u32(&ctl->cempty[c]), RS_WARPS);
     }
     for (int b = 0; b < NBUF; ++b) {
       mbar_init(smem_u32(&ctl->dfull[b]), 1);
-      mbar_init(smem_u32(&ctl->dempty[b]), 8);
+      mbar_init(smem_u32(&ctl->dempty[b]), RS_WARPS);
     }
     ctl->abort = 0;
     fence_barrier_init();
@@ -246,18 +248,18 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // ---------------------------------------------------------------- rescale + epilogue
-    const int rw = warp - W_RESCALE;                 // 0..7
-    const int sub = warp & 3, half = rw >> 2;        // TMEM sub-partition, 64-column half
+    const int rw = warp - W_RESCALE;                 // 0..15
+    const int sub = warp & 3, quarter = rw >> 2;     // TMEM sub-partition, 32-column quarter
     const int row = sub * 32 + lane;
     uint32_t uses = 0;
     int c = 0;
     uint32_t cph = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const int mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
-      const int m = mb * BM + row, n0 = nb * BN + half * 64;
-      uint64_t acc[32];                            // 64 columns as float32 pairs
+      const int m = mb * BM + row, n0 = nb * BN + quarter * RS_COLS;
+      uint64_t acc[RS_COLS / 2];                   // 32 columns as float32 pairs
 #pragma unroll
-      for (int i = 0; i < 32; ++i) acc[i] = 0ull;
+      for (int i = 0; i < RS_COLS / 2; ++i) acc[i] = 0ull;
       bool ok = true;
       for (int kt = 0; ok && kt < nk; ++kt) {
         if (!mbar_wait(smem_u32(&ctl->cfull[c]), cph, abort_flag, p.err)) {
@@ -268,33 +270,27 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int j = 0; j < 2; ++j, ++uses) {        // the k-tile's two 64-groups
           const uint32_t sxb = __float_as_uint(sc[j * 128 + row]);
           const uint64_t sx2 = u2(sxb, sxb);
-          const uint32_t sra = smem_u32(sc + 256 + j * 128 + half * 64);
+          const uint32_t sra = smem_u32(sc + 256 + j * 128 + quarter * RS_COLS);
           const uint32_t buf = uses % NBUF, dph = (uses / NBUF) & 1;
           if (!mbar_wait(smem_u32(&ctl->dfull[buf]), dph, abort_flag, p.err)) {
             ok = false;
             break;
           }
           tc_fence_after();
+          uint32_t r[32];
+          tmem_ld32(tmem + ((uint32_t)(sub * 32) << 16) + buf * BN + quarter * RS_COLS, r);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&ctl->dempty[buf]));
+          // acc += (sx sr) d: the group's exact fp32 sum, rescaled by the
+          // product of two binary16 scales (exact in fp32), then one FMA
 #pragma unroll
-          for (int hc = 0; hc < 2; ++hc) {
-            uint32_t r[32];
-            tmem_ld32(tmem + ((uint32_t)(sub * 32) << 16) + buf * BN + half * 64 + hc * 32, r);
-            tmem_wait_ld();
-            if (hc == 1) {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(smem_u32(&ctl->dempty[buf]));
-            }
-            // acc += (sx sr) d: the group's exact fp32 sum, rescaled by the
-            // product of two binary16 scales (exact in fp32), then one FMA
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              uint64_t sr01, sr23;
-              lds2x64(sra + (hc * 8 + q) * 16, sr01, sr23);
-              const int i = hc * 16 + 2 * q;
-              acc[i] = f2_fma(f2_mul(sx2, sr01), u2(r[4 * q], r[4 * q + 1]), acc[i]);
-              acc[i + 1] = f2_fma(f2_mul(sx2, sr23), u2(r[4 * q + 2], r[4 * q + 3]), acc[i + 1]);
-            }
+          for (int q = 0; q < 8; ++q) {
+            uint64_t sr01, sr23;
+            lds2x64(sra + q * 16, sr01, sr23);
+            acc[2 * q] = f2_fma(f2_mul(sx2, sr01), u2(r[4 * q], r[4 * q + 1]), acc[2 * q]);
+            acc[2 * q + 1] = f2_fma(f2_mul(sx2, sr23), u2(r[4 * q + 2], r[4 * q + 3]), acc[2 * q + 1]);
           }
         }
         __syncwarp();
@@ -312,25 +308,20 @@ __global__ void __launch_bounds__(THREADS, 1)
           ok = false;
         } else {
           tc_fence_after();
+          uint32_t r[32];
+          tmem_ld32(tmem + ((uint32_t)(sub * 32) << 16) + buf * BN + quarter * RS_COLS, r);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&ctl->dempty[buf]));
 #pragma unroll
-          for (int hc = 0; hc < 2; ++hc) {
-            uint32_t r[32];
-            tmem_ld32(tmem + ((uint32_t)(sub * 32) << 16) + buf * BN + half * 64 + hc * 32, r);
-            tmem_wait_ld();
-            if (hc == 1) {
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(smem_u32(&ctl->dempty[buf]));
-            }
-#pragma unroll
-            for (int i = 0; i < 16; ++i) acc[hc * 16 + i] = f2_add(acc[hc * 16 + i], u2(r[2 * i], r[2 * i + 1]));
-          }
+          for (int i = 0; i < 16; ++i) acc[i] = f2_add(acc[i], u2(r[2 * i], r[2 * i + 1]));
         }
       }
       if (!ok) break;
       if (m < p.M) {
 #pragma unroll
-        for (int c8 = 0; c8 < 64; c8 += 8) {
+        for (int c8 = 0; c8 < RS_COLS; c8 += 8) {
           const int n = n0 + c8;
           if (n < p.N) {
             const float4 b0 = __ldg(reinterpret_cast<const float4*>(p.bias + n));
