@@ -320,26 +320,29 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (!ok) break;
       if (m < p.M) {
+        // 16 columns (32 bytes, one full sector) per store
 #pragma unroll
-        for (int c8 = 0; c8 < RS_COLS; c8 += 8) {
-          const int n = n0 + c8;
+        for (int c16 = 0; c16 < RS_COLS; c16 += 16) {
+          const int n = n0 + c16;
           if (n < p.N) {
-            const float4 b0 = __ldg(reinterpret_cast<const float4*>(p.bias + n));
-            const float4 b1 = __ldg(reinterpret_cast<const float4*>(p.bias + n + 4));
-            const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-            float y[8];
+            float y[16];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const uint64_t a2 = acc[(c8 + e) >> 1];
-              y[e] = __uint_as_float((e & 1) ? (uint32_t)(a2 >> 32) : (uint32_t)a2) + bb[e];
-              if (p.epi == 1) y[e] = gelu_tanh(y[e]);
+            for (int q = 0; q < 4; ++q) {
+              const float4 bq = __ldg(reinterpret_cast<const float4*>(p.bias + n) + q);
+              const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const uint64_t a2 = acc[(c16 + 4 * q + e) >> 1];
+                y[4 * q + e] = __uint_as_float((e & 1) ? (uint32_t)(a2 >> 32) : (uint32_t)a2) + bb[e];
+                if (p.epi == 1) y[4 * q + e] = gelu_tanh(y[4 * q + e]);
+              }
             }
-            uint4 o;
-            o.x = pack_bf16x2(y[0], y[1]);
-            o.y = pack_bf16x2(y[2], y[3]);
-            o.z = pack_bf16x2(y[4], y[5]);
-            o.w = pack_bf16x2(y[6], y[7]);
-            *reinterpret_cast<uint4*>(p.Y + (size_t)m * p.N + n) = o;
+            uint32_t o[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) o[j] = pack_bf16x2(y[2 * j], y[2 * j + 1]);
+            asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p.Y + (size_t)m * p.N + n),
+                         "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3]), "r"(o[4]), "r"(o[5]), "r"(o[6]), "r"(o[7])
+                         : "memory");
           }
         }
       }

@@ -75,6 +75,14 @@ __device__ __forceinline__ float gelu_tanh(float y) {
   return 0.5f * y * (1.f + tanhf(u));
 }
 
+// 32 bytes in one store (16-byte stores would leave every 32-byte sector
+// half written by each of two instructions).  p must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&o)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(o[0]), "r"(o[1]), "r"(o[2]),
+               "r"(o[3]), "r"(o[4]), "r"(o[5]), "r"(o[6]), "r"(o[7])
+               : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
@@ -239,25 +247,24 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int m = mb * BLOCK_M + row;
       if (m < p.M) {
         __nv_bfloat16* yrow = p.Y + (size_t)m * p.N;
+        // 16 columns (32 bytes, one full sector) per store
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int col = c * 32 + q * 8;
+          for (int q = 0; q < 2; ++q) {
+            const int col = c * 32 + q * 16;
             const int n = n0 + col;
             if (n < p.N) {
-              float y[8];
+              float y[16];
 #pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                y[j] = fmaf(p.alpha, __uint_as_float(r[c][q * 8 + j]), bslice[col + j]);
+              for (int j = 0; j < 16; ++j) {
+                y[j] = fmaf(p.alpha, __uint_as_float(r[c][q * 16 + j]), bslice[col + j]);
                 if (p.epi == 1) y[j] = gelu_tanh(y[j]);
               }
-              uint4 o;
-              o.x = pack_bf16x2(y[0], y[1]);
-              o.y = pack_bf16x2(y[2], y[3]);
-              o.z = pack_bf16x2(y[4], y[5]);
-              o.w = pack_bf16x2(y[6], y[7]);
-              *reinterpret_cast<uint4*>(yrow + n) = o;
+              uint32_t o[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) o[j] = pack_bf16x2(y[2 * j], y[2 * j + 1]);
+              st_global_v8(yrow + n, o);
             }
           }
         }
