@@ -4,13 +4,14 @@
 // so they are fused and X is read from HBM once).
 //
 // A cluster of two CTAs owns 64 rows of X; CTA c of the cluster walks the
-// c-th half of K in 128-column stages.  A producer warp keeps a TMA ring of
-// stages in flight; a stage holds the [64 x 128] bf16 tile of X (two
-// 128-byte-swizzled [64 x 64] boxes), the matching [r_tot x 128] tile of
-// L1f^T (stored pre-swizzled, one contiguous bulk copy) and the 128 values of
+// c-th half of K in 256-column stages.  A producer warp keeps a TMA ring of
+// stages in flight; a stage holds the [64 x 256] bf16 tile of X (four
+// 128-byte-swizzled [64 x 64] boxes: 512 contiguous bytes of every row, which
+// HBM streams faster than 256), the matching [r_tot x 256] tile of L1f^T
+// (stored pre-swizzled, one contiguous bulk copy) and the 256 values of
 // 1/lambda.
 // From the same staged tile:
-//   * 16 quantizer warps: every thread one 16-element group of one row
+//   * 16 quantizer warps: every thread two 16-element groups of one row
 //     (x^ = x / lambda, amax, block scale, 4-bit codes), written packed with
 //     scales in the layout kernel 2's tensor-core MMA consumes;
 //   * one thread issues the down projection on the 5th-generation tensor core:
@@ -36,12 +37,12 @@ namespace svdq {
 namespace {
 
 constexpr int BM = K1_BOX_ROWS;              // rows per cluster (= MMA M = TMA box rows)
-constexpr int BK = 128;                      // K columns per stage (two 64-column swizzled boxes)
+constexpr int BK = 256;                      // K columns per stage (four 64-column swizzled boxes)
 constexpr int KSPLIT = 2;                    // CTAs per cluster, each half of K
 constexpr int QWARPS = 16;                   // quantizer warps: 64 rows x 8 groups
 constexpr int THREADS = 32 * (QWARPS + 2);   // + producer warp + MMA warp
 constexpr int X_BOX = BM * 128;              // one [64 x 64] bf16 box, 8 KB
-constexpr int X_BYTES = 2 * X_BOX;           // 16 KB
+constexpr int X_BYTES = 4 * X_BOX;           // 32 KB
 constexpr int IL_BYTES = BK * 4;             // 1/lambda for the stage
 constexpr int W_PROD = 0, W_MMA = 1, W_Q0 = 2;
 constexpr int MAX_STAGES = 8;
@@ -79,7 +80,7 @@ struct Layout {
 __host__ __device__ inline Layout make_layout(int stages, int r_tot, bool do_lr) {
   Layout L;
   L.stages = stages;
-  L.l_bytes = do_lr ? 2 * r_tot * 128 : 0;  // r_tot % 16 == 0: 2 KB multiples keep the 1 KB swizzle atoms aligned
+  L.l_bytes = do_lr ? 4 * r_tot * 128 : 0;  // r_tot % 16 == 0: 2 KB multiples keep the 1 KB swizzle atoms aligned
   L.x_ring = 0;
   L.l_ring = stages * X_BYTES;
   L.il_ring = L.l_ring + stages * L.l_bytes;
@@ -104,8 +105,11 @@ __global__ void __launch_bounds__(THREADS, 1)
   // cluster, and the cluster rank equals this index
   const int split = blockIdx.x % KSPLIT;
   const int m0 = (blockIdx.x / KSPLIT) * BM;
-  const int ns = p.K_pad / BK / KSPLIT;                  // stages per CTA (K_pad % 256 == 0)
-  const int kb0 = split * ns;                            // first 128-column block of this CTA
+  // stages of 256 columns: the first CTA of the pair takes ceil(nk / 2), the
+  // second the rest (possibly none: then its partial LR is zero)
+  const int nk = p.K_pad / BK, nk0 = (nk + 1) / 2;
+  const int ns = split == 0 ? nk0 : nk - nk0;
+  const int kb0 = split * nk0;                           // first 256-column block of this CTA
 
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const Layout L = make_layout(p.stages, p.r_tot, p.do_lr != 0);
@@ -148,8 +152,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int kb = kb0 + it;
         const uint32_t bar = smem_u32(&full[s]);
         mbar_arrive_expect_tx(bar, X_BYTES + L.l_bytes + IL_BYTES);
-        tma_load_2d(smem_u32(base + L.x_ring + s * X_BYTES), &tmX, kb * BK, m0, bar);
-        tma_load_2d(smem_u32(base + L.x_ring + s * X_BYTES + X_BOX), &tmX, kb * BK + 64, m0, bar);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) tma_load_2d(smem_u32(base + L.x_ring + s * X_BYTES + b * X_BOX), &tmX, kb * BK + 64 * b, m0, bar);
         if (p.do_lr)   // the stage's L1f^T tile is stored contiguous and pre-swizzled: one bulk copy
           bulk_load(smem_u32(base + L.l_ring + s * L.l_bytes), p.L1t + (size_t)kb * p.r_tot * BK, L.l_bytes, bar);
         bulk_load(smem_u32(base + L.il_ring + s * IL_BYTES), p.inv_lambda + kb * BK, IL_BYTES, bar);
@@ -196,51 +200,63 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int it = 0; it < ns; ++it) {
       const int s = it % p.stages;
       if (!mbar_wait(smem_u32(&full[s]), (it / p.stages) & 1, abort_flag, p.err)) break;
-      const int kb = 2 * (kb0 + it) + qb;                // 64-column block
-      const uint32_t box = smem_u32(base + L.x_ring + s * X_BYTES + qb * X_BOX);
-      const uint4 u0 = lds128(sw128_chunk(box, qr, 2 * qg));
-      const uint4 u1 = lds128(sw128_chunk(box, qr, 2 * qg + 1));
-      const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-      // 1/lambda of this group: chunk q at position 4 q + qg of the permuted
-      // stage copy (zeros past K, where TMA also filled x with zeros)
-      const uint32_t ila = smem_u32(base + L.il_ring + s * IL_BYTES) + qb * 256 + qg * 16;
-      float il[16];
+      // this thread's two groups of the stage: boxes qb and qb + 2; read both,
+      // release the stage, then quantize
+      uint32_t w[2][8];
+      float il[2][16];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 f = lds128(ila + 64 * q);
-        il[4 * q] = __uint_as_float(f.x);
-        il[4 * q + 1] = __uint_as_float(f.y);
-        il[4 * q + 2] = __uint_as_float(f.z);
-        il[4 * q + 3] = __uint_as_float(f.w);
+      for (int h = 0; h < 2; ++h) {
+        const int b = qb + 2 * h;
+        const uint32_t box = smem_u32(base + L.x_ring + s * X_BYTES + b * X_BOX);
+        const uint4 u0 = lds128(sw128_chunk(box, qr, 2 * qg));
+        const uint4 u1 = lds128(sw128_chunk(box, qr, 2 * qg + 1));
+        w[h][0] = u0.x; w[h][1] = u0.y; w[h][2] = u0.z; w[h][3] = u0.w;
+        w[h][4] = u1.x; w[h][5] = u1.y; w[h][6] = u1.z; w[h][7] = u1.w;
+        // 1/lambda of this group: chunk q at position 4 q + qg of the 64-column
+        // block's permuted copy (zeros past K, where TMA also filled x with zeros)
+        const uint32_t ila = smem_u32(base + L.il_ring + s * IL_BYTES) + b * 256 + qg * 16;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 f = lds128(ila + 64 * q);
+          il[h][4 * q] = __uint_as_float(f.x);
+          il[h][4 * q + 1] = __uint_as_float(f.y);
+          il[h][4 * q + 2] = __uint_as_float(f.z);
+          il[h][4 * q + 3] = __uint_as_float(f.w);
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&empty[s]));   // shared-memory reads of stage s are done
-      float v[16];
 #pragma unroll
-      for (int j = 0; j < 16; j += 2)   // bf16 pair -> two floats, times 1/lambda
-        mul2_rn(__uint_as_float(w[j >> 1] << 16), __uint_as_float(w[j >> 1] & 0xFFFF0000u), il[j], il[j + 1],
-                v[j], v[j + 1]);
-      uint2 codes;
-      if (p.fmt == 0) {
-        uint32_t sc;
-        quant_nvfp4_16_tab(v, p.six_st, inv_tab, codes, sc);
-        // the row's four scale bytes form one word; kernel 2 wants it in four
-        // replicas (one per TMEM sub-partition): lane qg of the quad writes replica qg
-        uint32_t sw = sc << (8 * qg);
-        sw |= __shfl_xor_sync(0xffffffffu, sw, 1);
-        sw |= __shfl_xor_sync(0xffffffffu, sw, 2);
-        *reinterpret_cast<uint32_t*>(p.sX + sfx_rep_offset(m, kb, qg, p.K_pad)) = sw;
-      } else {
-        __half sc;
-        quant_int4_16of64(v, codes, sc);
-        // stored widened to float32 (exact): kernel 2 multiplies in float32
-        if (qg == 0) reinterpret_cast<float*>(p.sX)[int4_scale_offset(m, kb, p.K_pad)] = __half2float(sc);
-      }
-      if (m < p.M) {
-        if (p.fmt == 0)
-          *reinterpret_cast<uint2*>(p.qX + (size_t)m * qx_row_bytes + (size_t)kb * 32 + qg * 8) = codes;
-        else
-          *reinterpret_cast<uint4*>(p.qX + (size_t)m * qx_row_bytes + (size_t)kb * 64 + qg * 16) = int4x16_to_e4m3(codes);
+      for (int h = 0; h < 2; ++h) {
+        const int kb = 4 * (kb0 + it) + qb + 2 * h;      // 64-column block
+        float v[16];
+#pragma unroll
+        for (int j = 0; j < 16; j += 2)   // bf16 pair -> two floats, times 1/lambda
+          mul2_rn(__uint_as_float(w[h][j >> 1] << 16), __uint_as_float(w[h][j >> 1] & 0xFFFF0000u), il[h][j],
+                  il[h][j + 1], v[j], v[j + 1]);
+        uint2 codes;
+        if (p.fmt == 0) {
+          uint32_t sc;
+          quant_nvfp4_16_tab(v, p.six_st, inv_tab, codes, sc);
+          // the row's four scale bytes form one word; kernel 2 wants it in four
+          // replicas (one per TMEM sub-partition): lane qg of the quad writes replica qg
+          uint32_t sw = sc << (8 * qg);
+          sw |= __shfl_xor_sync(0xffffffffu, sw, 1);
+          sw |= __shfl_xor_sync(0xffffffffu, sw, 2);
+          *reinterpret_cast<uint32_t*>(p.sX + sfx_rep_offset(m, kb, qg, p.K_pad)) = sw;
+        } else {
+          __half sc;
+          quant_int4_16of64(v, codes, sc);
+          // stored widened to float32 (exact): kernel 2 multiplies in float32
+          if (qg == 0) reinterpret_cast<float*>(p.sX)[int4_scale_offset(m, kb, p.K_pad)] = __half2float(sc);
+        }
+        if (m < p.M) {
+          if (p.fmt == 0)
+            *reinterpret_cast<uint2*>(p.qX + (size_t)m * qx_row_bytes + (size_t)kb * 32 + qg * 8) = codes;
+          else
+            *reinterpret_cast<uint4*>(p.qX + (size_t)m * qx_row_bytes + (size_t)kb * 64 + qg * 16) =
+                int4x16_to_e4m3(codes);
+        }
       }
     }
   }
@@ -315,9 +331,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 size_t quant_down_smem_bytes(int r_tot, bool do_lr, int* stages_out, int ns) {
-  const int stage_bytes = X_BYTES + IL_BYTES + (do_lr ? 2 * r_tot * 128 : 0);
-  int stages = (200 * 1024) / stage_bytes;
-  stages = stages < 2 ? 2 : (stages > MAX_STAGES ? MAX_STAGES : stages);
+  // as many stages as fit in 216 KB (large ranks get a single stage)
+  const int stage_bytes = X_BYTES + IL_BYTES + (do_lr ? 4 * r_tot * 128 : 0);
+  int stages = (216 * 1024) / stage_bytes;
+  stages = stages < 1 ? 1 : (stages > MAX_STAGES ? MAX_STAGES : stages);
   if (stages > ns) stages = ns < 1 ? 1 : ns;
   *stages_out = stages;
   const Layout L = make_layout(stages, r_tot, do_lr);
@@ -325,8 +342,9 @@ size_t quant_down_smem_bytes(int r_tot, bool do_lr, int* stages_out, int ns) {
 }
 
 cudaError_t launch_quant_down(const CUtensorMap& tmX, K1Params p, cudaStream_t stream) {
-  const int ns = p.K_pad / BK / KSPLIT;
+  const int ns = (p.K_pad / BK + 1) / 2;   // the larger of the two CTAs' stage counts
   const size_t smem = quant_down_smem_bytes(p.r_tot, p.do_lr != 0, &p.stages, ns);
+  if (smem > 227 * 1024) return cudaErrorInvalidValue;   // never launch past the shared-memory limit
   cudaError_t e = cudaFuncSetAttribute(quant_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
