@@ -41,7 +41,8 @@ Readings where the pages are silent (each one is a choice of this build):
     Per block of 16: a = max|v|, sb = E4M3(a / fp32(6 s_t)),
     d = fp32(f32(sb) s_t), inv = fp32(1/d) (0 if d = 0),
     code = E2M1(fp32(v inv)).  The activation tensor scale is static (an
-    offline calibration: amax of X^ / 2688).
+    offline calibration: amax of X^ / 2688) or, per call, the batch's own
+    (dynamic_act_scale: the batch's amax paired with s_tR to a power of two).
   * INT4: per block of 64: sb = fp16(fp32(a / 7)), d = f32(sb),
     inv = fp32(1/d) (0 if d = 0), code = clamp(rint(fp32(v inv)), -8, 7).
   * The low-rank down-projection output LR is rounded to bf16 (it is the
@@ -51,7 +52,7 @@ Readings where the pages are silent (each one is a choice of this build):
 """
 from __future__ import annotations
 
-from dataclasses import dataclass
+from dataclasses import dataclass, replace
 from typing import Optional
 
 import numpy as np
@@ -286,6 +287,27 @@ def quantize_activation(pw: PreparedWeights, X):
     return quantize_int4(Xh)
 
 
+def dynamic_act_scale(pw: PreparedWeights, X):
+    """Per-call NVFP4 activation tensor scale (a reading: the pages fix only
+    the FP32 tensor scale, not how it is chosen).  The batch's own
+    a = amax(|X^|) takes the place of the calibration value, paired with the
+    residual's tensor scale the way weight_tensor_scale pairs it the other
+    way round: j is the smallest integer with 2^j >= s_tR a / 2688 (float64;
+    a = 0 counts as 2688) and s_tX = fl32(2^j / s_tR), so no block scale needs
+    more than 448 and s_tX s_tR is the power of two 2^j.  Returns (s_tX, j)."""
+    Xh = smooth_activation(X, pw.inv_lam)
+    a = float(np.max(np.abs(Xh))) if np.size(Xh) else 0.0
+    x = (a if a > 0 else NVFP4_TENSOR_DIVISOR) * float(np.float32(pw.s_tR)) / float(NVFP4_TENSOR_DIVISOR)
+    m, e = np.frexp(x)
+    j = int(e - 1) if m == 0.5 else int(e)
+    return np.float32(np.float32(np.ldexp(1.0, j)) / np.float32(pw.s_tR)), j
+
+
+def with_act_scale(pw: PreparedWeights, s_tX) -> PreparedWeights:
+    """The same prepared layer with another NVFP4 activation tensor scale."""
+    return replace(pw, s_tX=np.float32(s_tX))
+
+
 def main_product(pw: PreparedWeights, qX, sX) -> np.ndarray:
     """Q(X^) Q(R) in float64 from the codes and scales."""
     if pw.fmt == "nvfp4":
@@ -301,13 +323,18 @@ def epilogue(y, bias, gelu: bool) -> np.ndarray:
     return F.bf16_round(y)
 
 
-def forward(pw: PreparedWeights, X, gelu: bool = False, quantize: bool = True):
+def forward(pw: PreparedWeights, X, gelu: bool = False, quantize: bool = True, dynamic: bool = False):
     """Y for activation X (M, K).  Returns dict with the intermediates.
+
+    dynamic=True (NVFP4) quantizes X^ with its own tensor scale
+    (dynamic_act_scale) instead of the calibrated one.
 
     quantize=False replaces every rounding of the layer's data path (the two
     4-bit quantizers, the bf16 LR and the bf16 output) by the identity, which
     leaves X^ R + X L1f L2 + b: equal to X W + b up to float32 rounding."""
     X = np.asarray(X, np.float32)
+    if dynamic and pw.fmt == "nvfp4":
+        pw = with_act_scale(pw, dynamic_act_scale(pw, X)[0])
     if quantize:
         qX, sX = quantize_activation(pw, X)
         LR = lowrank_down(X, pw.L1f)

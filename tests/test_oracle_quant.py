@@ -118,3 +118,52 @@ def test_weight_tensor_scale_pairs_to_a_power_of_two():
         _, sc = S.quantize_nvfp4(R, s_tR)
         top = F.e4m3_decode(sc).max()
         assert 224 <= top <= 448
+
+
+# ------------------------------------------------------------ per-call (dynamic) activation tensor scale
+def _prepared_small():
+    import workloads
+    L = workloads.draw_layer("dyn", "nvfp4", 48, 128, 64, 8, seed=31, n_out=3)
+    return L, S.calibrate_and_prepare("nvfp4", L.X, L.W, L.bias, L.rank)
+
+
+def test_dynamic_scale_pairs_to_a_power_of_two_and_covers_the_batch():
+    L, pw = _prepared_small()
+    for f in (1.0, 3.0, 0.01, 250.0):
+        X = (L.X * np.float32(f)).astype(np.float32)
+        s, j = S.dynamic_act_scale(pw, X)
+        a = float(np.max(np.abs(S.smooth_activation(X, pw.inv_lam))))
+        # alpha = s s_tR is 2^j up to the one float32 rounding of s
+        assert abs(float(s) * float(pw.s_tR) / 2.0 ** j - 1.0) < 2.0 ** -23
+        # the scale covers the batch (no block scale above 448) and is within a factor 2 of the tight one
+        assert float(s) * 2688.0 >= a * (1 - 2.0 ** -23)
+        assert float(s) * 2688.0 < 2.0 * a * (1 + 2.0 ** -23)
+        qX, sX = S.quantize_nvfp4(S.smooth_activation(X, pw.inv_lam), s)
+        assert F.e4m3_decode(sX).max() <= 448.0
+
+
+def test_dynamic_scale_is_equivariant_under_powers_of_two():
+    # scaling X by 2^p scales the dynamic tensor scale by 2^p exactly and leaves every code and block scale
+    L, pw = _prepared_small()
+    s0, j0 = S.dynamic_act_scale(pw, L.X)
+    q0, b0 = S.quantize_nvfp4(S.smooth_activation(L.X, pw.inv_lam), s0)
+    for p in (-3, 2, 5):
+        X = (L.X * np.float32(2.0 ** p)).astype(np.float32)
+        s, j = S.dynamic_act_scale(pw, X)
+        assert j == j0 + p and float(s) == float(s0) * 2.0 ** p
+        q, b = S.quantize_nvfp4(S.smooth_activation(X, pw.inv_lam), s)
+        assert np.array_equal(q, q0) and np.array_equal(b, b0)
+
+
+def test_dynamic_forward_tracks_the_batch_where_the_static_scale_saturates():
+    # a batch 1000x larger than the calibration one: the static scale clips every block above
+    # 6 * 448 * s_tX, the dynamic one follows the batch and keeps the calibration-level error
+    L, pw = _prepared_small()
+    rel = lambda Y, X: float(np.sqrt(np.mean((Y - (X.astype(np.float64) @ L.W.astype(np.float64) + L.bias[None, :])) ** 2))
+                             / np.sqrt(np.mean((X.astype(np.float64) @ L.W.astype(np.float64) + L.bias[None, :]) ** 2)))
+    e_calib = rel(S.forward(pw, L.X)["Y"], L.X)
+    X = (L.X * np.float32(1000.0)).astype(np.float32)
+    e_static = rel(S.forward(pw, X)["Y"], X)
+    e_dynamic = rel(S.forward(pw, X, dynamic=True)["Y"], X)
+    assert e_dynamic < 1.05 * e_calib + 1e-4
+    assert e_static > 3 * e_dynamic
