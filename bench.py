@@ -446,6 +446,15 @@ def run_ours(args, world, rank, local):
                                B.svdq_w4a4_gemm_lowrank_up(h, M, *acts[i % sets], epi,
                                                            Ys[i % sets], stream)), n_ov)
     t_unfused = timed(unfused, n_ov)
+    # the per-call NVFP4 activation tensor scale (svdq_linear_dynamic: one
+    # extra pass over X for its amax) against the static-scale public call
+    wss = [torch.empty(B.svdq_linear_dynamic_workspace_bytes(h, M), dtype=torch.uint8, device=dev)
+           for _ in range(sets)]
+    t_linear = timed(lambda i: B.svdq_linear(h, M, Xs[i % sets], epi, Ys[i % sets], wss[i % sets], None, stream),
+                     n_ov)
+    t_dyn = timed(lambda i: B.svdq_linear_dynamic(h, M, Xs[i % sets], epi, Ys[i % sets], wss[i % sets], None,
+                                                  stream), n_ov) if nv else None
+    del wss
 
     # end to end through the public call with host buffers
     e2e_steps = min(K_steps, 50)
@@ -498,6 +507,9 @@ def run_ours(args, world, rank, local):
                                     "unfused_us": round(t_unfused * 1e3, 2),
                                     "fused_over_plain": round(t_fused / t_plain - 1, 4),
                                     "unfused_over_plain": round(t_unfused / t_plain - 1, 4)},
+               "dynamic_scale": None if t_dyn is None else
+               {"linear_us": round(t_linear * 1e3, 2), "linear_dynamic_us": round(t_dyn * 1e3, 2),
+                "overhead": round(t_dyn / t_linear - 1, 4)},
                "gpu_launches": 2 * K_steps,
                "device_status": status,
                "clocks": clocks.summary()}

@@ -226,6 +226,37 @@ svdq_status svdq_linear(const svdq_weights* w, int M, const void* X, svdq_epilog
                         void* workspace, size_t ws_bytes, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * The whole layer with a per-call NVFP4 activation tensor scale.
+ * The "SVDQuant" paper's NVFP4 setting gives the activation an FP32 tensor
+ * scale on top of the E4M3 scales per 16 elements, but does not say how it
+ * is chosen.  svdq_linear uses the one fixed at preparation (act_scale);
+ * this entry point takes it from the call's own X^ = X diag(lambda)^-1:
+ *   a    = amax |X^| over all M x K elements (X^ rounded to float32 as in
+ *          kernel 1; a = 0 counts as 2688),
+ *   j    = the smallest integer with 2^j >= s_tR a / 2688 (float64),
+ *   s_tX = fl32(2^j / s_tR),
+ * so s_tX s_tR is the power of two 2^j, as alpha is at preparation, and no
+ * activation block scale exceeds 448 however X is distributed.  Kernel 2
+ * multiplies by 2^j; kernel 1 stores LR times 2^(k - j), where 2^k is the
+ * prepared alpha (svdq_weights_view), so LR L2a keeps its weight.
+ * Launches: one streaming pass over X (amax per CTA into the workspace, no
+ * atomics), then kernels 1 and 2, which read the partial maxima after their
+ * grid-dependency wait (no host round trip; stream capture works).
+ * INT4 has no tensor scale: for INT4 weights this is svdq_linear.
+ *   X  dev bf16 [M][K];  Y  dev bf16 [M][N]
+ *   workspace  dev, at least svdq_linear_dynamic_workspace_bytes(w, M):
+ *     bytes [0, svdq_linear_workspace_bytes(w, M)) hold qX, sX and LR as
+ *     svdq_linear places them (each at a 256-byte aligned offset, in that
+ *     order, sizes svdq_act_buffer_sizes); then 16 bytes written by the call
+ *     (NVFP4 only): float s_tX, int32 j, float 2^j, unused; then the amax
+ *     slots.  Every byte read is written first by the same call.
+ * Errors: as svdq_linear.
+ * ------------------------------------------------------------------------ */
+size_t svdq_linear_dynamic_workspace_bytes(const svdq_weights* w, int M);
+svdq_status svdq_linear_dynamic(const svdq_weights* w, int M, const void* X, svdq_epilogue epi, void* Y,
+                                void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * svdq_linear without a workspace argument (no counterpart in the paper: it
  * is an integration convenience, not part of the method).
  *

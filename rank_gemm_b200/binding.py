@@ -63,6 +63,8 @@ _SIGS = {
     "svdq_w4a4_gemm_lowrank_up": (_i, [_vp, _i, _vp, _vp, _vp, _i, _vp, _vp]),
     "svdq_linear_workspace_bytes": (_sz, [_vp, _i]),
     "svdq_linear": (_i, [_vp, _i, _vp, _i, _vp, _vp, _sz, _vp]),
+    "svdq_linear_dynamic_workspace_bytes": (_sz, [_vp, _i]),
+    "svdq_linear_dynamic": (_i, [_vp, _i, _vp, _i, _vp, _vp, _sz, _vp]),
     "svdq_quantize_act": (_i, [_vp, _i, _vp, _vp, _vp, _vp]),
     "svdq_lowrank_down": (_i, [_vp, _i, _vp, _vp, _vp]),
     "svdq_w4a4_gemm": (_i, [_vp, _i, _vp, _vp, _vp, _vp]),
@@ -161,6 +163,16 @@ def svdq_linear(w, M, X, epi, Y, workspace, ws_bytes=None, stream=None):
     ws_bytes = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
     _check(lib.svdq_linear(w, M, _ptr(X), epi, _ptr(Y), _ptr(workspace), ws_bytes, _stream(stream)),
            "svdq_linear")
+
+
+def svdq_linear_dynamic_workspace_bytes(w, M) -> int:
+    return lib.svdq_linear_dynamic_workspace_bytes(w, M)
+
+
+def svdq_linear_dynamic(w, M, X, epi, Y, workspace, ws_bytes=None, stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
+    _check(lib.svdq_linear_dynamic(w, M, _ptr(X), epi, _ptr(Y), _ptr(workspace), ws_bytes, _stream(stream)),
+           "svdq_linear_dynamic")
 
 
 def svdq_quantize_act(w, M, X, qX, sX, stream=None):

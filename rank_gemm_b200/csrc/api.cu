@@ -152,8 +152,16 @@ svdq_status check_handle_device(const svdq_weights* w, DevState** d) {
   return dev == w->dev ? SVDQ_OK : SVDQ_ERR_INVALID_ARG;
 }
 
+// Per-call NVFP4 activation tensor scale: where the amax slots are and where
+// kernel 1 reports the scale it chose.
+struct DynScale {
+  const uint32_t* parts;
+  int n_parts;
+  float* record;
+};
+
 K1Params k1_params(const svdq_weights* w, const DevState* d, int M, void* qX, void* sX, void* LR,
-                   int do_quant, int do_lr) {
+                   int do_quant, int do_lr, const DynScale* dyn) {
   K1Params p;
   p.M = M;
   p.K = w->K;
@@ -168,6 +176,11 @@ K1Params k1_params(const svdq_weights* w, const DevState* d, int M, void* qX, vo
   p.L1t = w->L1t;
   p.s_t = w->s_tX;
   p.six_st = 6.0f * w->s_tX;   // one IEEE float32 multiply on the host
+  p.amax_parts = dyn ? dyn->parts : nullptr;
+  p.n_parts = dyn ? dyn->n_parts : 0;
+  p.k_alpha = std::ilogb(w->alpha);   // the prepared alpha is a power of two
+  p.s_tR = w->s_tR;
+  p.dyn_record = dyn ? dyn->record : nullptr;
   p.qX = static_cast<uint8_t*>(qX);
   p.sX = static_cast<uint8_t*>(sX);
   p.LR = static_cast<__nv_bfloat16*>(LR);
@@ -176,18 +189,19 @@ K1Params k1_params(const svdq_weights* w, const DevState* d, int M, void* qX, vo
 }
 
 svdq_status run_k1(const svdq_weights* w, int M, const void* X, void* qX, void* sX, void* LR,
-                   int do_quant, int do_lr, cudaStream_t stream) {
+                   int do_quant, int do_lr, cudaStream_t stream, const DynScale* dyn = nullptr) {
   DevState* d = nullptr;
   svdq_status s = check_handle_device(w, &d);
   if (s != SVDQ_OK) return s;
   CUtensorMap tmX;
   if (!tmap_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, w->K, M, (uint64_t)w->K * 2, 64, K1_BOX_ROWS))
     return SVDQ_ERR_CUDA;
-  return from_cuda(launch_quant_down(tmX, k1_params(w, d, M, qX, sX, LR, do_quant, do_lr), stream));
+  return from_cuda(launch_quant_down(tmX, k1_params(w, d, M, qX, sX, LR, do_quant, do_lr, dyn), stream));
 }
 
 svdq_status run_k2(const svdq_weights* w, int M, const void* qX, const void* sX, const void* LR,
-                   svdq_epilogue epi, void* Y, bool lowrank, cudaStream_t stream) {
+                   svdq_epilogue epi, void* Y, bool lowrank, cudaStream_t stream,
+                   const DynScale* dyn = nullptr) {
   DevState* d = nullptr;
   svdq_status s = check_handle_device(w, &d);
   if (s != SVDQ_OK) return s;
@@ -216,6 +230,9 @@ svdq_status run_k2(const svdq_weights* w, int M, const void* qX, const void* sX,
     p.sR = w->sR_rep;
     p.bias = w->bias_f;
     p.alpha = w->alpha;
+    p.amax_parts = dyn ? dyn->parts : nullptr;
+    p.n_parts = dyn ? dyn->n_parts : 0;
+    p.s_tR = w->s_tR;
     p.epi = (int)epi;
     p.Y = static_cast<__nv_bfloat16*>(Y);
     p.err = dev_err(d);
@@ -521,6 +538,42 @@ svdq_status svdq_linear(const svdq_weights* w, int M, const void* X, svdq_epilog
   s = run_k1(w, M, X, qX, sX, LR, 1, 1, stream);
   if (s != SVDQ_OK) return s;
   return run_k2(w, M, qX, sX, LR, epi, Y, true, stream);
+}
+
+// [svdq_linear's workspace | 256-byte record | amax slots]
+size_t svdq_linear_dynamic_workspace_bytes(const svdq_weights* w, int M) {
+  if (!w || M < 0) return 0;
+  return svdq_linear_workspace_bytes(w, M) + 256 + align256((size_t)AMAX_MAX_PARTS * 4);
+}
+
+svdq_status svdq_linear_dynamic(const svdq_weights* w, int M, const void* X, svdq_epilogue epi, void* Y,
+                                void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  if (!w || (M > 0 && (!X || !Y))) return SVDQ_ERR_INVALID_ARG;
+  if (epi != SVDQ_EPI_NONE && epi != SVDQ_EPI_GELU_TANH) return SVDQ_ERR_INVALID_ARG;
+  if (M < 0) return SVDQ_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(Y)) return SVDQ_ERR_ALIGNMENT;
+  if (M == 0) return SVDQ_OK;
+  if (!workspace || ws_bytes < svdq_linear_dynamic_workspace_bytes(w, M)) return SVDQ_ERR_WORKSPACE;
+  void *qX, *sX, *LR;
+  svdq_status s = carve(w, M, workspace, ws_bytes, &qX, &sX, &LR);
+  if (s != SVDQ_OK) return s;
+  if (w->fmt != SVDQ_NVFP4) {   // INT4 has no tensor scale: the static layer
+    if ((s = run_k1(w, M, X, qX, sX, LR, 1, 1, stream)) != SVDQ_OK) return s;
+    return run_k2(w, M, qX, sX, LR, epi, Y, true, stream);
+  }
+  DevState* d = nullptr;
+  if ((s = check_handle_device(w, &d)) != SVDQ_OK) return s;
+  uint8_t* tail = static_cast<uint8_t*>(workspace) + svdq_linear_workspace_bytes(w, M);
+  DynScale dyn;
+  dyn.record = reinterpret_cast<float*>(tail);
+  dyn.parts = reinterpret_cast<const uint32_t*>(tail + 256);
+  dyn.n_parts = act_amax_num_parts(w->K, d->num_sms);
+  if (dyn.n_parts <= 0) return SVDQ_ERR_SHAPE;
+  s = from_cuda(launch_act_amax(static_cast<const __nv_bfloat16*>(X), M, w->K, w->lambda_inv,
+                                reinterpret_cast<uint32_t*>(tail + 256), d->num_sms, stream));
+  if (s != SVDQ_OK) return s;
+  if ((s = run_k1(w, M, X, qX, sX, LR, 1, 1, stream, &dyn)) != SVDQ_OK) return s;
+  return run_k2(w, M, qX, sX, LR, epi, Y, true, stream, &dyn);
 }
 
 svdq_status svdq_quantize_act(const svdq_weights* w, int M, const void* X, void* qX, void* sX,

@@ -169,6 +169,12 @@ __device__ __forceinline__ void grid_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Named barrier `id` (1..15; 0 is __syncthreads) over `threads` threads of
+// the CTA (a multiple of 32; whole warps).
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 // ----------------------------------------------------------------- thread-block clusters
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
@@ -579,5 +585,45 @@ __host__ __device__ __forceinline__ size_t int4_scale_offset(int row, int g64, i
 }
 
 __host__ __device__ constexpr int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+// ----------------------------------------------------------------- per-call NVFP4 activation tensor scale
+// (the FP32 tensor scale of the "SVDQuant" paper's NVFP4 setting, chosen from
+// the call's own amax(|X^|) instead of the calibrated value)
+//
+// Largest of n <= 1024 non-negative float32 values kept as their bit
+// patterns (for those the integer order is the float order), reduced by one
+// warp.  The values were written by an earlier kernel: read through L2, all
+// loads issued before the first is used (one L2 round trip, not n / 32).
+__device__ __forceinline__ uint32_t warp_amax_bits(const uint32_t* parts, int n, int lane) {
+  uint32_t v[32];
+#pragma unroll
+  for (int t = 0; t < 32; ++t) v[t] = (lane + 32 * t < n) ? __ldcg(parts + lane + 32 * t) : 0u;
+  uint32_t m = 0;
+#pragma unroll
+  for (int t = 0; t < 32; ++t) m = max(m, v[t]);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+  return m;
+}
+
+// j = the smallest integer with 2^j >= s_tR a / 2688 (a = 0 counts as 2688),
+// evaluated in float64, where a s_tR is exact and the division is IEEE
+// round-to-nearest; then s_tX = fl32(2^j / s_tR) and s_tX s_tR is 2^j up to
+// one float32 rounding, so no activation block scale exceeds 448.
+__device__ __forceinline__ int dyn_scale_exponent(uint32_t amax_bits, float s_tR) {
+  const float a = __uint_as_float(amax_bits);
+  const double x = (a > 0.f ? (double)a : 2688.0) * (double)s_tR / 2688.0;
+  const unsigned long long b = (unsigned long long)__double_as_longlong(x);
+  const int e = (int)((b >> 52) & 0x7FF) - 1023;   // x is a normal float64: x >= 2^-298
+  return (b & 0xFFFFFFFFFFFFFull) ? e + 1 : e;     // x = 2^e exactly, else round up
+}
+
+// fl32(2^j): exact for -149 <= j <= 127, infinity above, zero below.
+__device__ __forceinline__ float exp2i_f32(int j) {
+  if (j > 127) return __uint_as_float(0x7F800000u);
+  if (j >= -126) return __uint_as_float((uint32_t)(j + 127) << 23);
+  if (j >= -149) return __uint_as_float(1u << (j + 149));
+  return 0.f;
+}
 
 }  // namespace svdq

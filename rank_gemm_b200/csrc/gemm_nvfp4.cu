@@ -221,6 +221,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int e = warp - 2, sub = warp & 3, ch = e >> 2;
     const int row = sub * 32 + lane;
     float* bslice = bias_s + e * 128;
+    // per-call activation tensor scale: alpha = s_tX s_tR = 2^j from the amax
+    // partials (kernel 1 scaled LR to match)
+    const float alpha =
+        p.amax_parts ? exp2i_f32(dyn_scale_exponent(warp_amax_bits(p.amax_parts, p.n_parts, lane), p.s_tR))
+                     : p.alpha;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       int mb, nb;
@@ -258,7 +263,7 @@ __global__ void __launch_bounds__(THREADS, 1)
               float y[16];
 #pragma unroll
               for (int j = 0; j < 16; ++j) {
-                y[j] = fmaf(p.alpha, __uint_as_float(r[c][q * 16 + j]), bslice[col + j]);
+                y[j] = fmaf(alpha, __uint_as_float(r[c][q * 16 + j]), bslice[col + j]);
                 if (p.epi == 1) y[j] = gelu_tanh(y[j]);
               }
               uint32_t o[8];

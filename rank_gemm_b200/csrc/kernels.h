@@ -20,6 +20,13 @@ struct K1Params {
   const float* inv_lambda; // [K_pad], permuted per 64-wide stage (see prepare.cu)
   const __nv_bfloat16* L1t; // L1f^T in the staged layout (one contiguous tile per stage)
   float s_t, six_st;       // NVFP4 activation tensor scale and fl32(6 s_t)
+  // per-call NVFP4 tensor scale (null: s_t above): the amax partials of X^,
+  // reduced after the grid-dependency wait; s_t = fl32(2^j / s_tR) and LR
+  // leaves scaled by 2^(k_alpha - j), where 2^k_alpha is the prepared alpha
+  const uint32_t* amax_parts;
+  int n_parts, k_alpha;
+  float s_tR;
+  float* dyn_record;       // if set, CTA 0 writes {s_t, j as int32 bits, 2^j}
   uint8_t* qX;             // [M][K_pad/2]
   uint8_t* sX;             // scale layout (see svdq.h)
   __nv_bfloat16* LR;       // [M][r_pad]
@@ -40,6 +47,9 @@ struct K2Params {
   const uint8_t* sR;       // weight scales, replicated layout (sfw_rep_offset)
   const float* bias;       // [N_pad]
   float alpha;             // s_tX * s_tR
+  const uint32_t* amax_parts;  // per-call tensor scale: alpha = 2^j from these (null: alpha above)
+  int n_parts;
+  float s_tR;
   int epi;                 // 0 none, 1 GELU (tanh form)
   __nv_bfloat16* Y;        // [M][N]
   DeviceErr err;
@@ -67,6 +77,15 @@ struct K2I8Params {
 };
 cudaError_t launch_gemm_int4(const CUtensorMap& tmX8, const CUtensorMap& tmR8, const CUtensorMap& tmLR,
                              const CUtensorMap& tmL2, K2I8Params p, int num_sms, cudaStream_t stream);
+
+// ---------------------------------------------------------------- per-call activation amax
+// One uint32 slot per CTA (the bits of that CTA's amax(|X^|)); at most
+// AMAX_MAX_PARTS slots.
+constexpr int AMAX_MAX_PARTS = 1024;
+static_assert(AMAX_MAX_PARTS <= 1024, "warp_amax_bits reads at most 32 slots a lane");
+int act_amax_num_parts(int K, int num_sms);   // slots the pass writes (0: K too large)
+cudaError_t launch_act_amax(const __nv_bfloat16* X, int M, int K, const float* inv_lambda, uint32_t* parts,
+                            int num_sms, cudaStream_t stream);
 
 // ---------------------------------------------------------------- unfused up projection
 struct UpParams {

@@ -131,7 +131,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (p.fmt == 0 && tid < 128) inv_tab[tid] = nvfp4_inv_entry((uint32_t)tid, p.s_t);
+  float* lr_scale_s = inv_tab + 128;                                 // per-call scale only
+  if (p.fmt == 0 && !p.amax_parts && tid < 128) inv_tab[tid] = nvfp4_inv_entry((uint32_t)tid, p.s_t);
   if (p.do_lr && warp == W_MMA) {
     tmem_alloc(smem_u32(tmem_slot), tmem_cols);
     tmem_relinquish();
@@ -195,6 +196,26 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int qw = warp - W_Q0;
     const int qb = qw & 1, qr = (qw >> 1) * 8 + (lane >> 2), qg = lane & 3;
     const int m = m0 + qr;
+    float six_st = p.six_st;
+    if (p.amax_parts) {
+      // per-call tensor scale: every quantizer warp reduces the amax partials
+      // (written by the amax pass, visible after the dependency wait), the
+      // first four build the 1/scale table, then the 16 warps meet
+      const int j = dyn_scale_exponent(warp_amax_bits(p.amax_parts, p.n_parts, lane), p.s_tR);
+      const float s_t = __fdiv_rn(exp2i_f32(j), p.s_tR);
+      six_st = __fmul_rn(6.f, s_t);
+      const int qt = tid - 32 * W_Q0;
+      if (qt < 128) inv_tab[qt] = nvfp4_inv_entry((uint32_t)qt, s_t);
+      if (qt == 0) {
+        *lr_scale_s = exp2i_f32(p.k_alpha - j);
+        if (blockIdx.x == 0 && p.dyn_record) {
+          p.dyn_record[0] = s_t;
+          p.dyn_record[1] = __int_as_float(j);
+          p.dyn_record[2] = exp2i_f32(j);
+        }
+      }
+      named_bar_sync(1, 32 * QWARPS);
+    }
     // NVFP4: packed codes (K_pad / 2 bytes a row); INT4: one E4M3 byte per code
     const size_t qx_row_bytes = p.fmt == 0 ? (size_t)(p.K_pad / 2) : (size_t)p.K_pad;
     for (int it = 0; it < ns; ++it) {
@@ -237,7 +258,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         uint2 codes;
         if (p.fmt == 0) {
           uint32_t sc;
-          quant_nvfp4_16_tab(v, p.six_st, inv_tab, codes, sc);
+          quant_nvfp4_16_tab(v, six_st, inv_tab, codes, sc);
           // the row's four scale bytes form one word; kernel 2 wants it in four
           // replicas (one per TMEM sub-partition): lane qg of the quad writes replica qg
           uint32_t sw = sc << (8 * qg);
@@ -294,6 +315,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ---------------------------------------------------------------- cluster reduction
     // this CTA's 32 rows; four consecutive columns per task; pad columns -> 0
     const int rows_per = BM / KSPLIT, quads = p.r_pad / 4;
+    // per-call scale: LR carries 2^(k_alpha - j) so that kernel 2's single
+    // factor 2^j restores it (a power of two: exact before the bf16 rounding)
+    const float lrs = p.amax_parts ? *lr_scale_s : 1.f;
     for (int i = tid; i < rows_per * quads; i += THREADS) {
       const int rr = split * rows_per + i / quads, c = (i % quads) * 4;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -306,6 +330,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           acc.y += v.y;
           acc.z += v.z;
           acc.w += v.w;
+        }
+        if (p.amax_parts) {
+          acc.x *= lrs;
+          acc.y *= lrs;
+          acc.z *= lrs;
+          acc.w *= lrs;
         }
       }
       const int m = m0 + rr;

@@ -267,3 +267,21 @@ class GpuLayer:
         (self.B.svdq_linear_unfused if unfused else self.B.svdq_linear)(self.h, M, Xd, epi, Y, ws)
         torch.cuda.synchronize()
         return Y
+
+    def linear_dynamic(self, Xd, M, gelu=False):
+        """svdq_linear_dynamic.  Returns (Y, qX, sX, LR, record): the
+        intermediates are sliced out of the workspace at the offsets
+        include/svdq.h gives, record = (s_tX, j, 2^j) as the call wrote it."""
+        B = self.B
+        ws = torch.empty(max(B.svdq_linear_dynamic_workspace_bytes(self.h, M), 16), dtype=torch.uint8,
+                         device="cuda").fill_(0xA5)
+        Y = torch.empty(M, self.N, dtype=torch.bfloat16, device="cuda")
+        B.svdq_linear_dynamic(self.h, M, Xd, B.SVDQ_EPI_GELU_TANH if gelu else B.SVDQ_EPI_NONE, Y, ws)
+        torch.cuda.synchronize()
+        qb, sb, lb = B.svdq_act_buffer_sizes(self.h, M)
+        o_s = rup(qb, 256)
+        o_l = o_s + rup(sb, 256)
+        o_r = B.svdq_linear_workspace_bytes(self.h, M)
+        rec = to_np(ws[o_r:o_r + 16])
+        record = (rec[0:4].view(np.float32)[0], int(rec[4:8].view(np.int32)[0]), rec[8:12].view(np.float32)[0])
+        return Y, ws[:qb], ws[o_s:o_s + sb], ws[o_l:o_l + lb], record
