@@ -190,12 +190,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (p.do_quant) {
     // ---------------------------------------------------------------- quantizers
-    // box qb, row qr, 16-column group qg of the stage: a warp covers 8 rows
-    // of one box (conflict-free swizzled reads), the four groups of a row
-    // sit in one quad of lanes
+    // box qb, rows qr and qr + 32, 16-column group qg of the stage: both of a
+    // thread's groups use the same 16 values of 1/lambda (read once); a warp
+    // covers 8 rows of one box (conflict-free swizzled reads), the four groups
+    // of a row sit in one quad of lanes
     const int qw = warp - W_Q0;
-    const int qb = qw & 1, qr = (qw >> 1) * 8 + (lane >> 2), qg = lane & 3;
-    const int m = m0 + qr;
+    const int qb = qw & 3, qr = (qw >> 2) * 8 + (lane >> 2), qg = lane & 3;
     float six_st = p.six_st;
     if (p.amax_parts) {
       // per-call tensor scale: every quantizer warp reduces the amax partials
@@ -221,44 +221,46 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int it = 0; it < ns; ++it) {
       const int s = it % p.stages;
       if (!mbar_wait(smem_u32(&full[s]), (it / p.stages) & 1, abort_flag, p.err)) break;
-      // this thread's two groups of the stage: boxes qb and qb + 2; read both,
-      // release the stage, then quantize
+      // this thread's two groups of the stage: rows qr and qr + 32 of box qb;
+      // read both and form x^ = x * (1/lambda) in registers, release the
+      // stage, then quantize and store
+      float v[2][16];
+      const uint32_t box = smem_u32(base + L.x_ring + s * X_BYTES + qb * X_BOX);
       uint32_t w[2][8];
-      float il[2][16];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int b = qb + 2 * h;
-        const uint32_t box = smem_u32(base + L.x_ring + s * X_BYTES + b * X_BOX);
-        const uint4 u0 = lds128(sw128_chunk(box, qr, 2 * qg));
-        const uint4 u1 = lds128(sw128_chunk(box, qr, 2 * qg + 1));
+        const uint4 u0 = lds128(sw128_chunk(box, qr + 32 * h, 2 * qg));
+        const uint4 u1 = lds128(sw128_chunk(box, qr + 32 * h, 2 * qg + 1));
         w[h][0] = u0.x; w[h][1] = u0.y; w[h][2] = u0.z; w[h][3] = u0.w;
         w[h][4] = u1.x; w[h][5] = u1.y; w[h][6] = u1.z; w[h][7] = u1.w;
-        // 1/lambda of this group: chunk q at position 4 q + qg of the 64-column
-        // block's permuted copy (zeros past K, where TMA also filled x with zeros)
-        const uint32_t ila = smem_u32(base + L.il_ring + s * IL_BYTES) + b * 256 + qg * 16;
+      }
+      // 1/lambda of this group: chunk q at position 4 q + qg of the 64-column
+      // block's permuted copy (zeros past K, where TMA also filled x with zeros)
+      const uint32_t ila = smem_u32(base + L.il_ring + s * IL_BYTES) + qb * 256 + qg * 16;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint4 f = lds128(ila + 64 * q);
-          il[h][4 * q] = __uint_as_float(f.x);
-          il[h][4 * q + 1] = __uint_as_float(f.y);
-          il[h][4 * q + 2] = __uint_as_float(f.z);
-          il[h][4 * q + 3] = __uint_as_float(f.w);
+      for (int q = 0; q < 4; ++q) {
+        const uint4 f = lds128(ila + 64 * q);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {   // bf16 pair -> two floats, times 1/lambda
+          mul2_rn(__uint_as_float(w[h][2 * q] << 16), __uint_as_float(w[h][2 * q] & 0xFFFF0000u),
+                  __uint_as_float(f.x), __uint_as_float(f.y), v[h][4 * q], v[h][4 * q + 1]);
+          mul2_rn(__uint_as_float(w[h][2 * q + 1] << 16), __uint_as_float(w[h][2 * q + 1] & 0xFFFF0000u),
+                  __uint_as_float(f.z), __uint_as_float(f.w), v[h][4 * q + 2], v[h][4 * q + 3]);
         }
       }
+      // every lane has consumed its shared-memory loads of stage s (the products
+      // above used them): the slot may be refilled.  A relaxed arrival, so that
+      // it does not wait for the previous stage's global stores.
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&empty[s]));   // shared-memory reads of stage s are done
+      if (lane == 0) mbar_arrive_relaxed(smem_u32(&empty[s]));
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int kb = 4 * (kb0 + it) + qb + 2 * h;      // 64-column block
-        float v[16];
-#pragma unroll
-        for (int j = 0; j < 16; j += 2)   // bf16 pair -> two floats, times 1/lambda
-          mul2_rn(__uint_as_float(w[h][j >> 1] << 16), __uint_as_float(w[h][j >> 1] & 0xFFFF0000u), il[h][j],
-                  il[h][j + 1], v[j], v[j + 1]);
+        const int kb = 4 * (kb0 + it) + qb;              // 64-column block
+        const int m = m0 + qr + 32 * h;
         uint2 codes;
         if (p.fmt == 0) {
           uint32_t sc;
-          quant_nvfp4_16_tab(v, six_st, inv_tab, codes, sc);
+          quant_nvfp4_16_tab(v[h], six_st, inv_tab, codes, sc);
           // the row's four scale bytes form one word; kernel 2 wants it in four
           // replicas (one per TMEM sub-partition): lane qg of the quad writes replica qg
           uint32_t sw = sc << (8 * qg);
@@ -267,7 +269,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           *reinterpret_cast<uint32_t*>(p.sX + sfx_rep_offset(m, kb, qg, p.K_pad)) = sw;
         } else {
           __half sc;
-          quant_int4_16of64(v, codes, sc);
+          quant_int4_16of64(v[h], codes, sc);
           // stored widened to float32 (exact): kernel 2 multiplies in float32
           if (qg == 0) reinterpret_cast<float*>(p.sX)[int4_scale_offset(m, kb, p.K_pad)] = __half2float(sc);
         }
