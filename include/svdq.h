@@ -204,8 +204,10 @@ svdq_status svdq_quantize_act_lowrank_down(const svdq_weights* w, int M, const v
  * write the same output, so the 16-bit branch adds no HBM round trip).
  *   y[m,n] = alpha * ( sum_k dq(qX)[m,k] dq(qR)[n,k] + sum_i LR[m,i] L2a[n,i] ) + b[n]
  *   (NVFP4: block-scaled tensor-core MMA with E4M3 scales per 16; INT4:
- *   int8 MMA per 64-group, rescaled by sX[m,g] sR[n,g]); optional GELU (tanh
- *   form); Y = bf16(y).
+ *   an exact tensor-core product per 64-group on the codes held as E4M3,
+ *   rescaled by sX[m,g] sR[n,g]); optional GELU (tanh form, evaluated as
+ *   y / (1 + e^(-2u)) with the hardware exp2 and reciprocal approximations,
+ *   relative error near 1e-6); Y = bf16(y).
  *   qX, sX, LR  dev, as written by kernel 1 (or by an equivalent producer)
  *   Y   dev bf16 [M][N] row-major
  * Errors: INVALID_ARG, SHAPE, ALIGNMENT, UNSUPPORTED_DEVICE, CUDA.

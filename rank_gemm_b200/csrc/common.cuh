@@ -452,6 +452,21 @@ __device__ __forceinline__ float absmax16(const float (&v)[16]) {
   return fmaxf(a, fabsf(v[15]));
 }
 
+// GELU, tanh form: 0.5 y (1 + tanh(u)) with u = sqrt(2/pi) (y + 0.044715 y^3),
+// evaluated as the equal y / (1 + e^(-2u)), e^(-2u) = 2^(-2u log2 e), with
+// the hardware base-2 exponential and reciprocal approximations (relative
+// error near 1e-6, far inside the layer's bf16 output): two special-function
+// instructions instead of a full-precision tanh.  Large negative y: the
+// exponential overflows to +inf and the result is -0.
+__device__ __forceinline__ float gelu_tanh(float y) {
+  constexpr float kTwoULog2e = 2.302208198144325f;   // 2 sqrt(2/pi) log2(e)
+  const float z = y * fmaf(0.044715f * y, y, 1.0f);   // y + 0.044715 y^3
+  float t, r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(t) : "f"(-kTwoULog2e * z));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + t));
+  return y * r;
+}
+
 // ----------------------------------------------------------------- 4-bit group quantizers
 // NVFP4, one 16-element group: a = max|v|; sb = E4M3(a / six_st) with six_st
 // = fl32(6 s_t); d = fl32(f32(sb) s_t); inv = fl32(1/d) (0 if d == 0);

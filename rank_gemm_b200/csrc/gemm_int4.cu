@@ -86,11 +86,6 @@ __device__ __forceinline__ void lds2x64(uint32_t addr, uint64_t& a, uint64_t& b)
   asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "r"(addr));
 }
 
-__device__ __forceinline__ float gelu_tanh(float y) {
-  const float u = 0.7978845608028654f * (y + 0.044715f * y * y * y);
-  return 0.5f * y * (1.f + tanhf(u));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);

@@ -70,11 +70,6 @@ __device__ __forceinline__ void tile_coords(int tile, int nmb, int nnb, int& mb,
   nb = rr / gs;
 }
 
-__device__ __forceinline__ float gelu_tanh(float y) {
-  const float u = 0.7978845608028654f * (y + 0.044715f * y * y * y);
-  return 0.5f * y * (1.f + tanhf(u));
-}
-
 // 32 bytes in one store (16-byte stores would leave every 32-byte sector
 // half written by each of two instructions).  p must be 32-byte aligned.
 __device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&o)[8]) {

@@ -86,8 +86,8 @@ __global__ void __launch_bounds__(THREADS) lowrank_up_kernel(UpParams p) {
           const float2 old = __bfloat1622float2(*y);
           float v0 = old.x + p.alpha * acc[a][b][2 * h], v1 = old.y + p.alpha * acc[a][b][2 * h + 1];
           if (p.epi == 1) {
-            v0 = 0.5f * v0 * (1.f + tanhf(0.7978845608028654f * (v0 + 0.044715f * v0 * v0 * v0)));
-            v1 = 0.5f * v1 * (1.f + tanhf(0.7978845608028654f * (v1 + 0.044715f * v1 * v1 * v1)));
+            v0 = gelu_tanh(v0);
+            v1 = gelu_tanh(v1);
           }
           *y = __floats2bfloat162_rn(v0, v1);
         }
