@@ -42,7 +42,7 @@ sys.path.insert(0, ROOT)
 WORKLOAD = dict(name="nvfp4_qkv_M4608_K3072_N9216_r32", fmt="nvfp4", M=4608, K=3072, N=9216, rank=32)
 # --workload: the QKV projection is the bench line; the others are the
 # remaining parity configurations, timed the same way for their profiles.
-WORKLOADS = ("qkv", "int4_qkv", "mlp_fc1", "mlp_fc2", "lora")
+WORKLOADS = ("qkv", "int4_qkv", "mlp_fc1", "mlp_fc2", "lora", "awq_adaln")
 INT8_PER_BF16 = 2.0         # nominal dense INT8 : BF16 tensor throughput (4.5 : 2.25)
 METRIC = "SVDQuant W4A4 linear effective TFLOPS & % of FP4 tensor peak; µs/layer"
 UNIT = "TFLOP/s"
@@ -524,6 +524,124 @@ def run_ours(args, world, rank, local):
         print(json.dumps(out), flush=True)
 
 
+# ------------------------------------------------------------------ AWQ W4A16 arm
+AWQ_METRIC = "AWQ W4A16 linear effective TFLOPS & % of HBM bandwidth; µs/layer"
+
+
+def run_awq(args, world, rank, local):
+    """The awq_w4a16 modulation projection (workloads.awq_adaln): one
+    svdq_awq_linear call per step.  Five prepared weight sets (32 MB each,
+    160 MB together > the 126 MB L2) rotate, so the weights stream from HBM
+    on every call, as in a model where the layer runs once per block."""
+    import numpy as np
+    import torch
+    import workloads
+    from rank_gemm_b200 import build as _b
+    if rank == 0:
+        _b.build()
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", init_method="env://", world_size=world, rank=rank,
+                                timeout=__import__("datetime").timedelta(seconds=120))
+        dist.barrier()
+    from rank_gemm_b200 import binding as B
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    L = workloads.awq_adaln()
+    M, K, N = L.M, L.K, L.N
+    sets = 5
+    Wt = torch.from_numpy(np.ascontiguousarray(L.W.T)).to(torch.bfloat16).to(dev)
+    bias = torch.from_numpy(L.bias).to(torch.bfloat16).to(dev)
+    hs = [B.svdq_awq_prepare(K, N, Wt, None, bias) for _ in range(sets)]
+    del Wt
+    X = torch.from_numpy(L.X).to(torch.bfloat16).to(dev)
+    Ys = [torch.empty(M, N, dtype=torch.bfloat16, device=dev) for _ in range(sets)]
+    stream = torch.cuda.current_stream(dev)
+    for i in range(args.warmup):
+        B.svdq_awq_linear(hs[i % sets], M, X, Ys[i % sets], stream)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t0.record(stream)
+        for i in range(args.steps):
+            B.svdq_awq_linear(hs[i % sets], M, X, Ys[i % sets], stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    max_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+    status = B.svdq_poll_device_error(stream)
+    us = max_ms / args.steps * 1e3
+    flops = 2.0 * M * N * K
+    value = weak_scaling_value(flops, args.steps, world, max_ms)
+    peaks = measured_peaks()
+    G = K // 64
+    # algorithmic bytes: codes, scales and zero points once, X, 1/s, bias, Y
+    nbytes = N * K // 2 + G * N * 3 + M * K * 2 + K * 4 + N * 4 + M * N * 2
+    gbs = nbytes / (us * 1e-6) / 1e9
+    traffic = profiled_traffic("awq_gemv_%s.md" % "adaln", kernel_sources("awq.cu"))
+    # end to end through the public call with host buffers
+    Xh = torch.empty(M, K, dtype=torch.bfloat16, pin_memory=True)
+    Xh.copy_(X.cpu())
+    Yh = torch.empty(M, N, dtype=torch.bfloat16, pin_memory=True)
+    Xd = torch.empty_like(X)
+    e2e_steps = min(args.steps, 200)
+    for i in range(3):
+        Xd.copy_(Xh, non_blocking=True)
+        B.svdq_awq_linear(hs[i % sets], M, Xd, Ys[0], stream)
+        Yh.copy_(Ys[0], non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        Xd.copy_(Xh, non_blocking=True)
+        B.svdq_awq_linear(hs[i % sets], M, Xd, Ys[0], stream)
+        Yh.copy_(Ys[0], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / e2e_steps
+    out = None
+    if rank == 0:
+        out = {"metric": AWQ_METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+               "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 6), "us_per_layer": round(us, 3),
+               "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 x int4 -> f32",
+               "data": "synthetic (seeded: SiLU(randn) activation, randn*0.02 weight), random-init weights",
+               "config": {"workload": L.name, "M": M, "K": K, "N": N, "group": 64, "awq_scale": "none",
+                          "parallelism": "replicas x%d (each rank its own batch)" % world,
+                          "l2": "%d rotating weight sets (%.0f MB) > 126 MB L2" % (sets, sets * nbytes / 1e6)},
+               "roofline": {"kernel": "awq_gemv", "bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm"],
+                            "unit": "GB/s", "frac": round(gbs / peaks["hbm"], 4), "traffic": traffic,
+                            "algorithmic_bytes": nbytes, "us": round(us, 3),
+                            "peak_source": "%s HBM copy bandwidth" % peaks["source"]},
+               "e2e": {"value": round(flops * world / (e2e_ms * 1e-3) / 1e12, 4), "unit": UNIT,
+                       "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2,
+                       "ms_per_step": round(e2e_ms, 5)},
+               "gpu_launches": args.steps, "device_status": status, "clocks": clocks.summary()}
+    for h in hs:
+        B.svdq_awq_free(h)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            from oracle import awq as A
+            aw = A.prepare(L.W, L.bias)
+            ts = []
+            for _ in range(3):
+                c0 = time.perf_counter()
+                A.forward(aw, L.X)
+                ts.append(time.perf_counter() - c0)
+            t = statistics.median(ts)
+            out["cpu_baseline"] = {"value": round(flops / t / 1e12, 6), "unit": UNIT, "cores": oracle_threads(),
+                                   "kind": "oracle",
+                                   "sample": "float64 numpy oracle forward of the whole layer (dequantize, "
+                                             "matmul, bias); median of 3", "seconds_per_sample": round(t, 4)}
+        print(json.dumps(out), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -538,6 +656,8 @@ def main():
     world, rank, local = dist_setup()
     if args.impl == "reference":
         run_reference(args, world, rank)
+    elif args.workload == "awq_adaln":
+        run_awq(args, world, rank, local)
     else:
         run_ours(args, world, rank, local)
 

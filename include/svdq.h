@@ -314,6 +314,59 @@ svdq_status svdq_linear_unfused(const svdq_weights* w, int M, const void* X, svd
                                 void* Y, void* workspace, size_t ws_bytes, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * AWQ W4A16 linear layer: 4-bit weights, 16-bit activations.
+ * The second kernel family of the Diffusers blog "Integrating Nunchaku 4-bit
+ * diffusion inference into Diffusers" ("Introducing Nunchaku Lite":
+ * awq_w4a16, for the adaptive-normalization and modulation projections,
+ * which are memory-bound and sensitive to precision; "Native loading in
+ * Diffusers": precision int4, group_size 64).
+ *
+ *   prepare:  W' = fl32(w * s_k) with AWQ's per-input-channel scale s (all
+ *             ones if NULL); per group g of 64 input features and output
+ *             feature n: lo, hi = min, max of W'; d = binary16 of
+ *             fl32(max(hi - lo, 1e-5) / 15), round to nearest even,
+ *             saturating at 65504; zero = clamp(rint(-lo / d), 0, 15);
+ *             code = clamp(rint(w' / d) + zero, 0, 15) (IEEE float32
+ *             divisions, rint = round half to even).
+ *   layer:    y[m,n] = sum_g d[g,n] sum_{k in g} (code[k,n] - zero[g,n]) x'[m,k]
+ *             + b[n], x' = fl32(x * fl32(1/s_k)); float32 accumulation;
+ *             Y = bf16(y).
+ * The layer reads every weight byte once per call and is sized for small M
+ * (the rows of a modulation projection: a few per image); it stages up to
+ * 4 activation rows at a time (fewer when K > 3072) and streams the weights
+ * once per group of rows.
+ *
+ * svdq_awq_prepare: W_t dev bf16 [N][K] (nn.Linear order); s dev float32 [K]
+ *   or NULL; bias dev bf16 [N] or NULL.  K % 64 == 0, N >= 1.  Synchronous
+ *   on `stream` (returns when the handle is ready).  The handle owns its
+ *   buffers until svdq_awq_free.
+ *   Errors: INVALID_ARG, SHAPE, ALIGNMENT, UNSUPPORTED_DEVICE, NO_MEMORY, CUDA.
+ * svdq_awq_linear: X dev bf16 [M][K], Y dev bf16 [M][N], M >= 0 (0: no-op).
+ *   Errors: INVALID_ARG (null, or the handle belongs to another device),
+ *   SHAPE, ALIGNMENT, UNSUPPORTED_DEVICE, CUDA.
+ * svdq_awq_view layouts (N_pad = N rounded up to 32; pad features hold
+ *   code 0, zero 0, scale 0):
+ *   code   uint8 [K/32][N_pad][16]: 16 bytes per (32-feature chunk c, n), the
+ *          codes of k = 32c .. 32c + 31, two per byte, even k in the low nibble
+ *   scale  binary16 [K/64][N_pad];  zero  uint8 [K/64][N_pad]
+ *   inv_s  float32 [K] = fl32(1/s);  bias  float32 [N_pad]
+ * ------------------------------------------------------------------------ */
+typedef struct svdq_awq_weights svdq_awq_weights;
+typedef struct {
+  int K, N, N_pad;
+  const void* code;
+  const void* scale;
+  const void* zero;
+  const float* inv_s;
+  const float* bias;
+} svdq_awq_info;
+svdq_status svdq_awq_prepare(int K, int N, const void* W_t, const float* s, const void* bias,
+                             cudaStream_t stream, svdq_awq_weights** out);
+svdq_status svdq_awq_free(svdq_awq_weights* w);
+svdq_status svdq_awq_view(const svdq_awq_weights* w, svdq_awq_info* info);
+svdq_status svdq_awq_linear(const svdq_awq_weights* w, int M, const void* X, void* Y, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * Diagnostics.
  * svdq_poll_device_error: synchronizes `stream`, then reads and clears the
  *   current device's error word.  Returns SVDQ_OK, SVDQ_ERR_TIMEOUT (a wait

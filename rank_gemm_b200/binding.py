@@ -49,6 +49,12 @@ class WeightsInfo(ctypes.Structure):
                 ("s_tX", ctypes.c_float), ("alpha", ctypes.c_float)]
 
 
+class AwqInfo(ctypes.Structure):
+    _fields_ = [("K", ctypes.c_int), ("N", ctypes.c_int), ("N_pad", ctypes.c_int), ("code", ctypes.c_void_p),
+                ("scale", ctypes.c_void_p), ("zero", ctypes.c_void_p), ("inv_s", ctypes.c_void_p),
+                ("bias", ctypes.c_void_p)]
+
+
 _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 _SIGS = {
     "svdq_status_string": (ctypes.c_char_p, [_i]),
@@ -71,6 +77,10 @@ _SIGS = {
     "svdq_lowrank_up": (_i, [_vp, _i, _vp, _i, _vp, _vp]),
     "svdq_linear_unfused": (_i, [_vp, _i, _vp, _i, _vp, _vp, _sz, _vp]),
     "svdq_linear_noalloc": (_i, [_vp, _i, _vp, _i, _vp, _vp]),
+    "svdq_awq_prepare": (_i, [_i, _i, _vp, _vp, _vp, _vp, ctypes.POINTER(_vp)]),
+    "svdq_awq_free": (_i, [_vp]),
+    "svdq_awq_view": (_i, [_vp, ctypes.POINTER(AwqInfo)]),
+    "svdq_awq_linear": (_i, [_vp, _i, _vp, _vp, _vp]),
     "svdq_poll_device_error": (_i, [_vp]),
     "svdq_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
     "svdq_debug_override_cc": (None, [_i, _i]),
@@ -205,6 +215,28 @@ def svdq_linear_noalloc(w, M, X, epi, Y, stream=None):
 
 
 SVDQ_NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def svdq_awq_prepare(K, N, W_t, s=None, bias=None, stream=None) -> int:
+    """Returns the opaque AWQ W4A16 handle (an int); release it with svdq_awq_free."""
+    h = _vp()
+    _check(lib.svdq_awq_prepare(K, N, _ptr(W_t), _ptr(s), _ptr(bias), _stream(stream), ctypes.byref(h)),
+           "svdq_awq_prepare")
+    return h.value
+
+
+def svdq_awq_free(w):
+    _check(lib.svdq_awq_free(w), "svdq_awq_free")
+
+
+def svdq_awq_view(w) -> AwqInfo:
+    info = AwqInfo()
+    _check(lib.svdq_awq_view(w, ctypes.byref(info)), "svdq_awq_view")
+    return info
+
+
+def svdq_awq_linear(w, M, X, Y, stream=None):
+    _check(lib.svdq_awq_linear(w, M, _ptr(X), _ptr(Y), _stream(stream)), "svdq_awq_linear")
 
 
 def svdq_poll_device_error(stream=None) -> int:

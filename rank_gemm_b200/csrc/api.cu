@@ -261,6 +261,28 @@ svdq_status run_k2(const svdq_weights* w, int M, const void* qX, const void* sX,
   return from_cuda(launch_gemm_int4(tmX8, w->tm_qR8, tmLR, w->tm_L2a_i4, p, d->num_sms, stream));
 }
 
+}  // namespace
+
+struct svdq_awq_weights {
+  int dev;
+  int K, N, N_pad;
+  uint8_t* code;
+  __half* scale;
+  uint8_t* zero;
+  float* inv_s;
+  float* bias_f;
+};
+
+namespace {
+
+void free_awq(svdq_awq_weights* w) {
+  cudaFree(w->code);
+  cudaFree(w->scale);
+  cudaFree(w->zero);
+  cudaFree(w->inv_s);
+  cudaFree(w->bias_f);
+}
+
 void free_buffers(svdq_weights* w) {
   cudaFree(w->qR);
   cudaFree(w->sR);
@@ -639,6 +661,109 @@ svdq_status svdq_linear_unfused(const svdq_weights* w, int M, const void* X, svd
   if ((s = svdq_lowrank_down(w, M, X, LR, stream)) != SVDQ_OK) return s;
   if ((s = svdq_w4a4_gemm(w, M, qX, sX, Y, stream)) != SVDQ_OK) return s;
   return svdq_lowrank_up(w, M, LR, epi, Y, stream);
+}
+
+svdq_status svdq_awq_prepare(int K, int N, const void* W_t, const float* s, const void* bias, cudaStream_t stream,
+                             svdq_awq_weights** out) {
+  if (out) *out = nullptr;
+  if (!out || !W_t) return SVDQ_ERR_INVALID_ARG;
+  if (K <= 0 || K % 64 || N <= 0) return SVDQ_ERR_SHAPE;
+  if (!aligned16(W_t) || !aligned16(s) || !aligned16(bias)) return SVDQ_ERR_ALIGNMENT;
+  DevState* d = nullptr;
+  svdq_status st = current_device(&d);
+  if (st != SVDQ_OK) return st;
+  svdq_awq_weights* w = new (std::nothrow) svdq_awq_weights();
+  if (!w) return SVDQ_ERR_NO_MEMORY;
+  cudaGetDevice(&w->dev);
+  w->K = K;
+  w->N = N;
+  w->N_pad = round_up(N, 32);
+  const size_t G = (size_t)K / 64;
+  const bool ok = cudaMalloc(&w->code, (size_t)w->N_pad * K / 2) == cudaSuccess &&
+                  cudaMalloc(&w->scale, G * w->N_pad * 2) == cudaSuccess &&
+                  cudaMalloc(&w->zero, G * w->N_pad) == cudaSuccess &&
+                  cudaMalloc(&w->inv_s, (size_t)K * 4) == cudaSuccess &&
+                  cudaMalloc(&w->bias_f, (size_t)w->N_pad * 4) == cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    free_awq(w);
+    delete w;
+    return SVDQ_ERR_NO_MEMORY;
+  }
+  AwqPrepParams p;
+  p.K = K;
+  p.N = N;
+  p.N_pad = w->N_pad;
+  p.Wt = static_cast<const __nv_bfloat16*>(W_t);
+  p.s = s;
+  p.bias = static_cast<const __nv_bfloat16*>(bias);
+  p.code = w->code;
+  p.scale = w->scale;
+  p.zero = w->zero;
+  p.inv_s = w->inv_s;
+  p.bias_f = w->bias_f;
+  cudaError_t e = launch_awq_quantize(p, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) {
+    free_awq(w);
+    delete w;
+    return from_cuda(e);
+  }
+  *out = w;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_awq_free(svdq_awq_weights* w) {
+  if (!w) return SVDQ_OK;
+  int prev = -1;
+  cudaGetDevice(&prev);
+  cudaSetDevice(w->dev);
+  cudaDeviceSynchronize();
+  free_awq(w);
+  if (prev >= 0) cudaSetDevice(prev);
+  delete w;
+  cudaGetLastError();
+  return SVDQ_OK;
+}
+
+svdq_status svdq_awq_view(const svdq_awq_weights* w, svdq_awq_info* info) {
+  if (!w || !info) return SVDQ_ERR_INVALID_ARG;
+  info->K = w->K;
+  info->N = w->N;
+  info->N_pad = w->N_pad;
+  info->code = w->code;
+  info->scale = w->scale;
+  info->zero = w->zero;
+  info->inv_s = w->inv_s;
+  info->bias = w->bias_f;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_awq_linear(const svdq_awq_weights* w, int M, const void* X, void* Y, cudaStream_t stream) {
+  if (!w || (M > 0 && (!X || !Y))) return SVDQ_ERR_INVALID_ARG;
+  if (M < 0) return SVDQ_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(Y)) return SVDQ_ERR_ALIGNMENT;
+  if (M == 0) return SVDQ_OK;
+  DevState* d = nullptr;
+  svdq_status st = current_device(&d);
+  if (st != SVDQ_OK) return st;
+  int dev = -1;
+  cudaGetDevice(&dev);
+  if (dev != w->dev) return SVDQ_ERR_INVALID_ARG;
+  AwqParams p;
+  p.M = M;
+  p.K = w->K;
+  p.N = w->N;
+  p.N_pad = w->N_pad;
+  p.mb = awq_rows_per_block(w->K, M);
+  p.X = static_cast<const __nv_bfloat16*>(X);
+  p.code = w->code;
+  p.scale = w->scale;
+  p.zero = w->zero;
+  p.inv_s = w->inv_s;
+  p.bias = w->bias_f;
+  p.Y = static_cast<__nv_bfloat16*>(Y);
+  return from_cuda(launch_awq_gemv(p, stream));
 }
 
 svdq_status svdq_poll_device_error(cudaStream_t stream) {

@@ -130,4 +130,37 @@ cudaError_t launch_prepare_quantize(const PrepParams& p, float s_tR, float alpha
 
 cudaError_t launch_selftest_timeout(DeviceErr err, cudaStream_t stream);
 
+// ---------------------------------------------------------------- AWQ W4A16 layer
+// Codes: uint8 [K/32][N_pad][16] (chunk c holds k in [32c, 32c+32) of feature
+// n, two codes per byte, even k in the low nibble); scale binary16 and zero
+// uint8 [K/64][N_pad]; N_pad = N rounded up to 32.
+constexpr int AWQ_WARPS = 8;      // warps of a CTA, splitting K
+constexpr int AWQ_MB_MAX = 4;     // activation rows per pass over the weights
+static_assert(AWQ_MB_MAX <= AWQ_WARPS, "one warp per row writes the outputs");
+struct AwqPrepParams {
+  int K, N, N_pad;
+  const __nv_bfloat16* Wt;        // [N][K]
+  const float* s;                 // [K] AWQ input-channel scales, or null (all 1)
+  const __nv_bfloat16* bias;      // [N] or null
+  uint8_t* code;
+  __half* scale;
+  uint8_t* zero;
+  float* inv_s;                   // [K] fl32(1/s)
+  float* bias_f;                  // [N_pad]
+};
+struct AwqParams {
+  int M, K, N, N_pad, mb;         // mb: activation rows staged per pass
+  const __nv_bfloat16* X;         // [M][K]
+  const uint8_t* code;
+  const __half* scale;
+  const uint8_t* zero;
+  const float* inv_s;             // [K] fl32(1/s)
+  const float* bias;              // [N_pad]
+  __nv_bfloat16* Y;               // [M][N]
+};
+cudaError_t launch_awq_quantize(const AwqPrepParams& p, cudaStream_t stream);
+cudaError_t launch_awq_gemv(AwqParams p, cudaStream_t stream);
+int awq_rows_per_block(int K, int M);
+size_t awq_smem_bytes(int K, int mb);
+
 }  // namespace svdq

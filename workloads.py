@@ -157,3 +157,46 @@ def dyadic_layer(M: int, K: int, N: int, rank: int, seed: int) -> dict:
     X = torch.randint(-8, 9, (M, K), generator=g).float() / 16.0
     L1 = torch.randint(-8, 9, (K, rank), generator=g).float() / 16.0
     return dict(X=X.numpy(), L1f=L1.numpy())
+
+
+# ---------------------------------------------------------------------------
+# AWQ W4A16 (the Diffusers blog's awq_w4a16 kernel family): the adaptive-norm
+# modulation projection of a FLUX-style block, Linear(3072 -> 6 * 3072), fed
+# with SiLU of the conditioning embedding, one row per image.
+# Recipe (one torch CPU generator, draws in this order):
+#   X = silu(randn(M, K)) rounded to bf16;  W = randn(K, N) * 0.02 -> bf16;
+#   bias = randn(N) * 0.01 -> bf16;  s = exp(uniform(-1, 1, K)) (float32),
+#   the AWQ per-input-channel scale, drawn only when asked for.
+# ---------------------------------------------------------------------------
+
+@dataclass
+class AwqLayer:
+    name: str
+    M: int
+    K: int
+    N: int
+    X: np.ndarray       # (M, K) float32, bf16 values
+    W: np.ndarray       # (K, N) float32, bf16 values
+    bias: np.ndarray    # (N,) float32, bf16 values
+    s: Optional[np.ndarray] = None   # (K,) float32 or None
+    seed: int = 0
+
+
+AWQ_ADALN = dict(name="awq_w4a16_adaln_M1_K3072_N18432", M=1, K=3072, N=18432, seed=5)
+
+
+def draw_awq_layer(name: str, M: int, K: int, N: int, seed: int, with_scale: bool = False) -> AwqLayer:
+    g = torch.Generator("cpu").manual_seed(seed)
+    X = torch.nn.functional.silu(torch.randn(M, K, generator=g))
+    W = torch.randn(K, N, generator=g) * 0.02
+    b = torch.randn(N, generator=g) * 0.01
+    s = torch.exp(torch.rand(K, generator=g) * 2.0 - 1.0).numpy().astype(np.float32) if with_scale else None
+    return AwqLayer(name=name, M=M, K=K, N=N, X=_bf16(X), W=_bf16(W), bias=_bf16(b), s=s, seed=seed)
+
+
+def awq_adaln(M: int = 1) -> AwqLayer:
+    d = dict(AWQ_ADALN)
+    d["M"] = M
+    if M != 1:
+        d["name"] = "awq_w4a16_adaln_M%d_K3072_N18432" % M
+    return draw_awq_layer(**d)
