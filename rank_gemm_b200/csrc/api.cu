@@ -19,6 +19,39 @@
 
 using namespace svdq;
 
+namespace svdq {
+
+// (kernel, device) -> the dynamic shared-memory limit already set
+cudaError_t ensure_dynamic_smem(const void* kernel, size_t bytes) {
+  struct Entry {
+    const void* fn;
+    int dev;
+    size_t bytes;
+  };
+  static std::mutex mu;
+  static Entry table[256];
+  static int used = 0;
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  int i = 0;
+  for (; i < used; ++i)
+    if (table[i].fn == kernel && table[i].dev == dev) break;
+  if (i < used && table[i].bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return e;
+  if (i == used) {
+    if (used == 256) return cudaSuccess;   // table full: correct, only slower (set on every call)
+    table[used++] = Entry{kernel, dev, bytes};
+  } else {
+    table[i].bytes = bytes;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace svdq
+
 // Device error word: kernels OR ERR_* bits into it (one copy per device).
 __device__ unsigned g_svdq_error_word;
 
@@ -131,6 +164,19 @@ bool tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t i
   cuuint32_t es[2] = {1, 1};
   return g_encode(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D uint8 tensor [d2][d1][d0] with byte strides s1 (between d1 rows) and
+// s2 (between d2 planes), no swizzle.
+bool tmap_3d_u8(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1, uint64_t s2,
+                uint32_t b0, uint32_t b1, uint32_t b2) {
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1, s2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t es[3] = {1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // NVFP4: packed codes; INT4: one E4M3 byte per code
@@ -271,6 +317,7 @@ struct svdq_awq_weights {
   uint8_t* zero;
   float* inv_s;
   float* bias_f;
+  CUtensorMap tm_code, tm_scale, tm_zero;   // the layer kernel's TMA views of the three
 };
 
 namespace {
@@ -709,6 +756,18 @@ svdq_status svdq_awq_prepare(int K, int N, const void* W_t, const float* s, cons
     delete w;
     return from_cuda(e);
   }
+  // stage boxes: 16 code chunks x 32 features x 16 bytes; 8 groups x 32 features of scales and zero points
+  const bool maps =
+      tmap_3d_u8(&w->tm_code, w->code, 16, w->N_pad, (uint64_t)K / 32, 16, (uint64_t)w->N_pad * 16, 16, 32, 16) &&
+      tmap_2d(&w->tm_scale, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, w->scale, w->N_pad, G, (uint64_t)w->N_pad * 2, 32, 8,
+              CU_TENSOR_MAP_SWIZZLE_NONE) &&
+      tmap_2d(&w->tm_zero, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->zero, w->N_pad, G, w->N_pad, 32, 8,
+              CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (!maps) {
+    free_awq(w);
+    delete w;
+    return SVDQ_ERR_CUDA;
+  }
   *out = w;
   return SVDQ_OK;
 }
@@ -763,7 +822,8 @@ svdq_status svdq_awq_linear(const svdq_awq_weights* w, int M, const void* X, voi
   p.inv_s = w->inv_s;
   p.bias = w->bias_f;
   p.Y = static_cast<__nv_bfloat16*>(Y);
-  return from_cuda(launch_awq_gemv(p, stream));
+  p.err = dev_err(d);
+  return from_cuda(launch_awq_gemv(w->tm_code, w->tm_scale, w->tm_zero, p, d->num_sms, stream));
 }
 
 svdq_status svdq_poll_device_error(cudaStream_t stream) {

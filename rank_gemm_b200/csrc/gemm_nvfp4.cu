@@ -282,8 +282,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 cudaError_t launch_gemm_nvfp4(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmLR,
                               const CUtensorMap& tmL2, K2Params p, int num_sms, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)SMEM_BYTES);
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(gemm_nvfp4_kernel), SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int tiles = p.num_m_blocks * p.num_n_blocks;
   const int grid = tiles < num_sms ? tiles : num_sms;

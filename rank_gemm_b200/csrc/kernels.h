@@ -11,6 +11,12 @@
 
 namespace svdq {
 
+// Raises `kernel`'s dynamic shared-memory limit on the current device to at
+// least `bytes`, calling the runtime only the first time a larger limit is
+// needed (the call costs microseconds of host time, more than a small
+// kernel's launch).
+cudaError_t ensure_dynamic_smem(const void* kernel, size_t bytes);
+
 // ---------------------------------------------------------------- kernel 1
 struct K1Params {
   int M, K, K_pad, r_tot, r_pad;
@@ -136,6 +142,7 @@ cudaError_t launch_selftest_timeout(DeviceErr err, cudaStream_t stream);
 // uint8 [K/64][N_pad]; N_pad = N rounded up to 32.
 constexpr int AWQ_WARPS = 8;      // warps of a CTA, splitting K
 constexpr int AWQ_MB_MAX = 4;     // activation rows per pass over the weights
+constexpr int AWQ_STAGES = 4;     // TMA ring depth (stages of 8 groups x 32 features)
 static_assert(AWQ_MB_MAX <= AWQ_WARPS, "one warp per row writes the outputs");
 struct AwqPrepParams {
   int K, N, N_pad;
@@ -157,9 +164,13 @@ struct AwqParams {
   const float* inv_s;             // [K] fl32(1/s)
   const float* bias;              // [N_pad]
   __nv_bfloat16* Y;               // [M][N]
+  DeviceErr err;
 };
 cudaError_t launch_awq_quantize(const AwqPrepParams& p, cudaStream_t stream);
-cudaError_t launch_awq_gemv(AwqParams p, cudaStream_t stream);
+// tmCode: codes as a 3-D uint8 tensor [K/32][N_pad][16], box {16, 32, 16};
+// tmScale / tmZero: [K/64][N_pad] binary16 / uint8, box {32, 8}.
+cudaError_t launch_awq_gemv(const CUtensorMap& tmCode, const CUtensorMap& tmScale, const CUtensorMap& tmZero,
+                           AwqParams p, int num_sms, cudaStream_t stream);
 int awq_rows_per_block(int K, int M);
 size_t awq_smem_bytes(int K, int mb);
 

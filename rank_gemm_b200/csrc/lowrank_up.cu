@@ -98,8 +98,7 @@ __global__ void __launch_bounds__(THREADS) lowrank_up_kernel(UpParams p) {
 
 cudaError_t launch_lowrank_up(UpParams p, cudaStream_t stream) {
   const size_t smem = (size_t)2 * TM * (p.r_tot + 8) * 2;
-  cudaError_t e = cudaFuncSetAttribute(lowrank_up_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(lowrank_up_kernel), (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((p.N + TN - 1) / TN, (p.M + TM - 1) / TM);
   lowrank_up_kernel<<<grid, THREADS, smem, stream>>>(p);

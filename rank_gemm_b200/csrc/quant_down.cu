@@ -377,8 +377,7 @@ cudaError_t launch_quant_down(const CUtensorMap& tmX, K1Params p, cudaStream_t s
   const int ns = (p.K_pad / BK + 1) / 2;   // the larger of the two CTAs' stage counts
   const size_t smem = quant_down_smem_bytes(p.r_tot, p.do_lr != 0, &p.stages, ns);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;   // never launch past the shared-memory limit
-  cudaError_t e = cudaFuncSetAttribute(quant_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(quant_down_kernel), smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   // row blocks up to the next multiple of 128, so that every row of the last
