@@ -137,6 +137,36 @@ svdq_status svdq_calibrate(int M, int K, int N, const void* X, const void* W_t, 
                            size_t ws_bytes, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * The low-rank split on the device (Stage 3 of the overview figure: the
+ * truncated SVD of W^ = diag(lambda) W), for callers without factors.
+ * Randomized range finder with subspace iteration (Halko, Martinsson, Tropp,
+ * "Finding structure with randomness", SIAM Review 2011, Algorithms 4.4 and
+ * 5.1), float64 throughout: a Rademacher sketch of l = min(rank + 8, K, N)
+ * columns drawn from Philox4x32-10 (Salmon et al., SC 2011; entry (n, j) is
+ * the top bit of word n l + j, block at counter (index lo, index hi, 0, 0),
+ * key (seed lo, seed hi)), three subspace iterations with CholeskyQR2
+ * orthonormalization, then the small SVD through the eigenproblem of the
+ * projected Gram matrix.  Returns the factors folded as svdq_prepare_weights
+ * takes them, each right singular vector signed so its largest-magnitude
+ * entry is positive.  It approximates the exact truncated SVD; for a matrix
+ * of rank <= l it is exact to float64 rounding.
+ *   W_t     dev bf16 [N][K];  lambda dev float32 [K]
+ *   seed    the sketch's Philox key
+ *   L1f     dev bf16 [K][rank]  = bf16(diag(lambda)^-1 U_r S_r)
+ *   L2      dev bf16 [rank][N]  = bf16(V_r^T)
+ *   sigma   host double [min(rank + 8, K, N)] or NULL: the estimated
+ *           singular values, descending
+ * Synchronous (returns when done); allocates and frees its own device
+ * scratch (8 K N bytes for W^ plus a few tall-skinny blocks).
+ * Errors: INVALID_ARG, SHAPE (rank < 1 or > min(K, N)), ALIGNMENT,
+ *         UNSUPPORTED_DEVICE, NO_MEMORY, CUDA.
+ * ------------------------------------------------------------------------ */
+#define SVDQ_SPLIT_SEED 0x5EEDull
+svdq_status svdq_lowrank_factors(int K, int N, int rank, const void* W_t, const float* lambda,
+                                 unsigned long long seed, void* L1f, void* L2, double* sigma,
+                                 cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * Offline weight preparation (Stage 3 of the overview figure: W^ splits into
  * a 16-bit rank-r branch and a 4-bit residual; abstract: LoRAs join the
  * low-rank branch without re-quantizing the residual).
@@ -156,16 +186,19 @@ svdq_status svdq_calibrate(int M, int K, int N, const void* X, const void* W_t, 
  *   fmt        SVDQ_NVFP4 or SVDQ_INT4
  *   W_t        dev bf16 [N][K]
  *   lambda     dev float32 [K]    smoothing factors (see svdq_calibrate)
- *   L1f        dev bf16 [K][rank] row-major
- *   L2         dev bf16 [rank][N] row-major
+ *   L1f        dev bf16 [K][rank] row-major, or NULL together with L2: the
+ *              factors then come from svdq_lowrank_factors (seed
+ *              SVDQ_SPLIT_SEED) on the device; rank <= min(K, N)
+ *   L2         dev bf16 [rank][N] row-major, or NULL (see L1f)
  *   bias       dev bf16 [N] or NULL (no bias)
  *   lora_A     dev bf16 [K][lora_rank] or NULL (then lora_rank must be 0)
  *   lora_B     dev bf16 [lora_rank][N] or NULL
  *   act_scale  NVFP4 static activation tensor scale s_tX (> 0, finite);
  *              ignored for INT4
  *   out        host: receives the new handle (NULL on error)
- * The call synchronizes `stream` before returning.  Errors: INVALID_ARG,
- * SHAPE, ALIGNMENT, UNSUPPORTED_DEVICE, NO_MEMORY, CUDA; nothing is leaked.
+ * The call synchronizes `stream` before returning.  Errors: INVALID_ARG
+ * (including exactly one of L1f, L2 NULL), SHAPE, ALIGNMENT,
+ * UNSUPPORTED_DEVICE, NO_MEMORY, CUDA; nothing is leaked.
  * ------------------------------------------------------------------------ */
 svdq_status svdq_prepare_weights(svdq_format fmt, int K, int N, int rank, const void* W_t,
                                  const float* lambda, const void* L1f, const void* L2,

@@ -63,6 +63,7 @@ _SIGS = {
     "svdq_prepare_weights": (_i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _f, _vp,
                                   ctypes.POINTER(_vp)]),
     "svdq_free_weights": (_i, [_vp]),
+    "svdq_lowrank_factors": (_i, [_i, _i, _i, _vp, _vp, ctypes.c_ulonglong, _vp, _vp, _vp, _vp]),
     "svdq_weights_view": (_i, [_vp, ctypes.POINTER(WeightsInfo)]),
     "svdq_act_buffer_sizes": (_i, [_vp, _i, ctypes.POINTER(_sz), ctypes.POINTER(_sz), ctypes.POINTER(_sz)]),
     "svdq_quantize_act_lowrank_down": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp]),
@@ -136,6 +137,19 @@ def svdq_prepare_weights(fmt, K, N, rank, W_t, lam, L1f, L2, bias=None, lora_A=N
                                     _ptr(lora_A), _ptr(lora_B), lora_rank, float(act_scale), _stream(stream),
                                     ctypes.byref(h)), "svdq_prepare_weights")
     return h.value
+
+
+SVDQ_SPLIT_SEED = 0x5EED
+
+
+def svdq_lowrank_factors(K, N, rank, W_t, lam, L1f, L2, seed=SVDQ_SPLIT_SEED, stream=None):
+    """The device's randomized split of diag(lam) W; fills L1f / L2 and returns
+    the estimated singular values (a list of min(rank + 8, K, N) floats)."""
+    n_sig = min(rank + 8, K, N)
+    sig = (ctypes.c_double * n_sig)()
+    _check(lib.svdq_lowrank_factors(K, N, rank, _ptr(W_t), _ptr(lam), seed, _ptr(L1f), _ptr(L2), sig,
+                                    _stream(stream)), "svdq_lowrank_factors")
+    return list(sig)
 
 
 def svdq_free_weights(w):

@@ -7,6 +7,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -392,7 +393,7 @@ svdq_status svdq_prepare_weights(svdq_format fmt, int K, int N, int rank, const 
                                  const void* lora_B, int lora_rank, float act_scale, cudaStream_t stream,
                                  svdq_weights** out) {
   if (out) *out = nullptr;
-  if (!out || !W_t || !lambda || !L1f || !L2) return SVDQ_ERR_INVALID_ARG;
+  if (!out || !W_t || !lambda || (!L1f) != (!L2)) return SVDQ_ERR_INVALID_ARG;
   if (fmt != SVDQ_NVFP4 && fmt != SVDQ_INT4) return SVDQ_ERR_INVALID_ARG;
   if (lora_rank < 0 || (lora_rank > 0) != (lora_A != nullptr) || (lora_rank > 0) != (lora_B != nullptr))
     return SVDQ_ERR_INVALID_ARG;
@@ -405,6 +406,25 @@ svdq_status svdq_prepare_weights(svdq_format fmt, int K, int N, int rank, const 
   DevState* d = nullptr;
   svdq_status s = current_device(&d);
   if (s != SVDQ_OK) return s;
+  if (!L1f) {
+    // no factors given: the library's randomized split of diag(lambda) W
+    if (rank > std::min(K, N)) return SVDQ_ERR_SHAPE;
+    void *f1 = nullptr, *f2 = nullptr;
+    if (cudaMalloc(&f1, (size_t)K * rank * 2) != cudaSuccess || cudaMalloc(&f2, (size_t)rank * N * 2) != cudaSuccess) {
+      cudaGetLastError();
+      cudaFree(f1);
+      cudaFree(f2);
+      return SVDQ_ERR_NO_MEMORY;
+    }
+    s = from_cuda(lowrank_factors(K, N, rank, static_cast<const __nv_bfloat16*>(W_t), lambda, SVDQ_SPLIT_SEED,
+                                  static_cast<__nv_bfloat16*>(f1), static_cast<__nv_bfloat16*>(f2), nullptr, stream));
+    if (s == SVDQ_OK)
+      s = svdq_prepare_weights(fmt, K, N, rank, W_t, lambda, f1, f2, bias, lora_A, lora_B, lora_rank, act_scale,
+                               stream, out);
+    cudaFree(f1);
+    cudaFree(f2);
+    return s;
+  }
 
   svdq_weights* w = new (std::nothrow) svdq_weights();
   if (!w) return SVDQ_ERR_NO_MEMORY;
@@ -512,6 +532,23 @@ svdq_status svdq_prepare_weights(svdq_format fmt, int K, int N, int rank, const 
   }
   *out = w;
   return SVDQ_OK;
+}
+
+svdq_status svdq_lowrank_factors(int K, int N, int rank, const void* W_t, const float* lambda,
+                                 unsigned long long seed, void* L1f, void* L2, double* sigma, cudaStream_t stream) {
+  if (!W_t || !lambda || !L1f || !L2) return SVDQ_ERR_INVALID_ARG;
+  if (K <= 0 || N <= 0 || rank < 1 || rank > std::min(K, N)) return SVDQ_ERR_SHAPE;
+  if (!aligned16(W_t) || !aligned16(lambda) || !aligned16(L1f) || !aligned16(L2)) return SVDQ_ERR_ALIGNMENT;
+  DevState* d = nullptr;
+  svdq_status s = current_device(&d);
+  if (s != SVDQ_OK) return s;
+  cudaError_t e = lowrank_factors(K, N, rank, static_cast<const __nv_bfloat16*>(W_t), lambda, seed,
+                                  static_cast<__nv_bfloat16*>(L1f), static_cast<__nv_bfloat16*>(L2), sigma, stream);
+  if (e == cudaErrorMemoryAllocation) {
+    cudaGetLastError();
+    return SVDQ_ERR_NO_MEMORY;
+  }
+  return from_cuda(e);
 }
 
 svdq_status svdq_free_weights(svdq_weights* w) {

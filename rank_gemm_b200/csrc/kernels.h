@@ -136,6 +136,12 @@ cudaError_t launch_prepare_quantize(const PrepParams& p, float s_tR, float alpha
 
 cudaError_t launch_selftest_timeout(DeviceErr err, cudaStream_t stream);
 
+// Randomized truncated SVD of W^ = diag(lambda) W (see rsvd.cu); synchronous.
+// L1f bf16 [K][r], L2 bf16 [r][N] on the device; sigma_out (host, may be
+// null) receives the min(r + 8, K, N) estimated singular values.
+cudaError_t lowrank_factors(int K, int N, int r, const __nv_bfloat16* Wt, const float* lam, uint64_t seed,
+                            __nv_bfloat16* L1f, __nv_bfloat16* L2, double* sigma_out, cudaStream_t s);
+
 // ---------------------------------------------------------------- AWQ W4A16 layer
 // Codes: uint8 [K/32][N_pad][16] (chunk c holds k in [32c, 32c+32) of feature
 // n, two codes per byte, even k in the low nibble); scale binary16 and zero
