@@ -253,21 +253,26 @@ def run_reference(args, world, rank):
 
 # ------------------------------------------------------------------ our arm
 def gpu_factors(B, Wt, X, rank, torch):
-    """Offline quantizer step on the GPU: smoothing factors and activation
-    scale with the library's calibration kernel, then the SVD of W^ with
-    torch.linalg.svd (cuSOLVER), folded like the library expects."""
+    """Offline quantizer step on the GPU, all in the library: smoothing
+    factors and activation scale from the calibration kernel, then the
+    low-rank split of W^ (svdq_lowrank_factors: randomized subspace
+    iteration in float64)."""
     M, K = X.shape
     N = Wt.shape[0]
     lam = torch.empty(K, dtype=torch.float32, device="cuda")
     act = torch.empty(1, dtype=torch.float32, device="cuda")
     ws = torch.empty(B.svdq_calibrate_workspace_bytes(K), dtype=torch.uint8, device="cuda")
     B.svdq_calibrate(M, K, N, X, Wt, 0.5, lam, act, ws)
-    What = (lam[:, None].double() * Wt.t().double()).float()
-    U, Sv, Vh = torch.linalg.svd(What, full_matrices=False)
-    L1f = ((U[:, :rank].double() * Sv[:rank].double()) / lam[:, None].double()).to(torch.bfloat16).contiguous()
-    L2 = Vh[:rank].to(torch.bfloat16).contiguous()
+    L1f = torch.empty(K, rank, dtype=torch.bfloat16, device="cuda")
+    L2 = torch.empty(rank, N, dtype=torch.bfloat16, device="cuda")
+    t0 = time.perf_counter()
+    B.svdq_lowrank_factors(K, N, rank, Wt, lam, L1f, L2)
+    SPLIT_SECONDS.append(time.perf_counter() - t0)
     torch.cuda.synchronize()
     return lam, float(act.item()), L1f, L2
+
+
+SPLIT_SECONDS = []
 
 
 def build_layer(name, B, torch, dev):
@@ -510,6 +515,8 @@ def run_ours(args, world, rank, local):
                "dynamic_scale": None if t_dyn is None else
                {"linear_us": round(t_linear * 1e3, 2), "linear_dynamic_us": round(t_dyn * 1e3, 2),
                 "overhead": round(t_dyn / t_linear - 1, 4)},
+               "prepare": {"lowrank_split_s": round(SPLIT_SECONDS[-1], 4) if SPLIT_SECONDS else None,
+                           "split": "svdq_lowrank_factors (randomized subspace iteration, float64)"},
                "gpu_launches": 2 * K_steps,
                "device_status": status,
                "clocks": clocks.summary()}
