@@ -292,6 +292,38 @@ svdq_status svdq_linear_dynamic(const svdq_weights* w, int M, const void* X, svd
                                 void* workspace, size_t ws_bytes, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
+ * One layer straight into the next (the cross-layer fusion of the Diffusers
+ * blog's "fused GELU/MLP" in "Introducing Nunchaku Lite": the first layer's
+ * epilogue produces the second layer's kernel-1 outputs, so its output
+ * never goes to memory in 16 bits and the second layer's kernel 1, which
+ * would read it back, does not run).
+ *
+ * svdq_linear_emit_next: layer w1 on X (kernel 1, then kernel 2 with the
+ *   epilogue `epi`) computes its bf16 output Y1 = bf16(epi(y)) tile by tile
+ *   and writes, instead of Y1, what svdq_quantize_act_lowrank_down(w2, M,
+ *   Y1, ...) would write: qX2 and sX2 (the NVFP4 codes and replicated scales
+ *   of Y1 diag(lambda2)^-1 with w2's static activation tensor scale),
+ *   identical to kernel 1's given the same Y1; and LR2 = bf16(Y1 L1f2) from
+ *   per-tile float32 partials added in a fixed order (the same on every run;
+ *   float32 summation order differs from kernel 1's, within the LR bound).
+ *   Requires both handles NVFP4, w2's K == w1's N and r_tot of w2 <= 32.
+ *   qX2, sX2, LR2  dev, sizes from svdq_act_buffer_sizes(w2, M)
+ *   workspace      dev, svdq_linear_emit_next_workspace_bytes(w1, w2, M)
+ * svdq_mlp: the pair: Y = layer w2 (epilogue epi2) of layer w1 (epi1) of X,
+ *   through svdq_linear_emit_next and kernel 2 of w2; Y dev bf16 [M][N2];
+ *   workspace svdq_mlp_workspace_bytes(w1, w2, M).
+ * Errors: as svdq_linear; SHAPE when the pair does not chain as above;
+ *         INVALID_ARG for an INT4 handle or handles on different devices.
+ * ------------------------------------------------------------------------ */
+size_t svdq_linear_emit_next_workspace_bytes(const svdq_weights* w1, const svdq_weights* w2, int M);
+svdq_status svdq_linear_emit_next(const svdq_weights* w1, const svdq_weights* w2, int M, const void* X,
+                                  svdq_epilogue epi, void* qX2, void* sX2, void* LR2, void* workspace,
+                                  size_t ws_bytes, cudaStream_t stream);
+size_t svdq_mlp_workspace_bytes(const svdq_weights* w1, const svdq_weights* w2, int M);
+svdq_status svdq_mlp(const svdq_weights* w1, const svdq_weights* w2, int M, const void* X, svdq_epilogue epi1,
+                     svdq_epilogue epi2, void* Y, void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
  * svdq_linear without a workspace argument (no counterpart in the paper: it
  * is an integration convenience, not part of the method).
  *

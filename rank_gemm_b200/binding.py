@@ -72,6 +72,10 @@ _SIGS = {
     "svdq_linear": (_i, [_vp, _i, _vp, _i, _vp, _vp, _sz, _vp]),
     "svdq_linear_dynamic_workspace_bytes": (_sz, [_vp, _i]),
     "svdq_linear_dynamic": (_i, [_vp, _i, _vp, _i, _vp, _vp, _sz, _vp]),
+    "svdq_linear_emit_next_workspace_bytes": (_sz, [_vp, _vp, _i]),
+    "svdq_linear_emit_next": (_i, [_vp, _vp, _i, _vp, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "svdq_mlp_workspace_bytes": (_sz, [_vp, _vp, _i]),
+    "svdq_mlp": (_i, [_vp, _vp, _i, _vp, _i, _i, _vp, _vp, _sz, _vp]),
     "svdq_quantize_act": (_i, [_vp, _i, _vp, _vp, _vp, _vp]),
     "svdq_lowrank_down": (_i, [_vp, _i, _vp, _vp, _vp]),
     "svdq_w4a4_gemm": (_i, [_vp, _i, _vp, _vp, _vp, _vp]),
@@ -197,6 +201,26 @@ def svdq_linear_dynamic(w, M, X, epi, Y, workspace, ws_bytes=None, stream=None):
     ws_bytes = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
     _check(lib.svdq_linear_dynamic(w, M, _ptr(X), epi, _ptr(Y), _ptr(workspace), ws_bytes, _stream(stream)),
            "svdq_linear_dynamic")
+
+
+def svdq_linear_emit_next_workspace_bytes(w1, w2, M) -> int:
+    return lib.svdq_linear_emit_next_workspace_bytes(w1, w2, M)
+
+
+def svdq_linear_emit_next(w1, w2, M, X, epi, qX2, sX2, LR2, workspace, ws_bytes=None, stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
+    _check(lib.svdq_linear_emit_next(w1, w2, M, _ptr(X), epi, _ptr(qX2), _ptr(sX2), _ptr(LR2), _ptr(workspace),
+                                     ws_bytes, _stream(stream)), "svdq_linear_emit_next")
+
+
+def svdq_mlp_workspace_bytes(w1, w2, M) -> int:
+    return lib.svdq_mlp_workspace_bytes(w1, w2, M)
+
+
+def svdq_mlp(w1, w2, M, X, epi1, epi2, Y, workspace, ws_bytes=None, stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
+    _check(lib.svdq_mlp(w1, w2, M, _ptr(X), epi1, epi2, _ptr(Y), _ptr(workspace), ws_bytes, _stream(stream)),
+           "svdq_mlp")
 
 
 def svdq_quantize_act(w, M, X, qX, sX, stream=None):

@@ -64,6 +64,7 @@ struct svdq_weights {
   uint8_t* sR;
   uint8_t* sR_rep;   // NVFP4: kernel 2's replicated copy of sR
   uint8_t* qR8;      // INT4: kernel 2's copy of qR, one E4M3 byte per code [N_pad][K_pad]
+  float* L1f32;      // NVFP4: [K_pad][r_tot] fp32 copy of [L1f | A], read when the layer before emits into this one
   __nv_bfloat16* L1t;
   __nv_bfloat16* L2a;
   float* bias_f;
@@ -248,7 +249,7 @@ svdq_status run_k1(const svdq_weights* w, int M, const void* X, void* qX, void* 
 
 svdq_status run_k2(const svdq_weights* w, int M, const void* qX, const void* sX, const void* LR,
                    svdq_epilogue epi, void* Y, bool lowrank, cudaStream_t stream,
-                   const DynScale* dyn = nullptr) {
+                   const DynScale* dyn = nullptr, const K2Params::Next* next = nullptr) {
   DevState* d = nullptr;
   svdq_status s = check_handle_device(w, &d);
   if (s != SVDQ_OK) return s;
@@ -283,7 +284,9 @@ svdq_status run_k2(const svdq_weights* w, int M, const void* qX, const void* sX,
     p.epi = (int)epi;
     p.Y = static_cast<__nv_bfloat16*>(Y);
     p.err = dev_err(d);
-    return from_cuda(launch_gemm_nvfp4(tmA, w->tm_qR, tmLR, w->tm_L2a, p, d->num_sms, stream));
+    std::memset(&p.next, 0, sizeof(p.next));
+    if (next) p.next = *next;
+    return from_cuda(launch_gemm_nvfp4(tmA, w->tm_qR, tmLR, w->tm_L2a, p, d->num_sms, stream, next != nullptr));
   }
   CUtensorMap tmX8;
   if (!tmap_2d(&tmX8, CU_TENSOR_MAP_DATA_TYPE_UINT8, qX, w->K_pad, M, w->K_pad, 128, K2_I4_ROWS))
@@ -336,6 +339,7 @@ void free_buffers(svdq_weights* w) {
   cudaFree(w->sR);
   cudaFree(w->sR_rep);
   cudaFree(w->qR8);
+  cudaFree(w->L1f32);
   cudaFree(w->L1t);
   cudaFree(w->L2a);
   cudaFree(w->bias_f);
@@ -445,6 +449,7 @@ svdq_status svdq_prepare_weights(svdq_format fmt, int K, int N, int rank, const 
   bool ok = cudaMalloc(&w->qR, qr_b) == cudaSuccess && cudaMalloc(&w->sR, sr_b) == cudaSuccess &&
             (fmt != SVDQ_NVFP4 || cudaMalloc(&w->sR_rep, 4 * sr_b) == cudaSuccess) &&
             (fmt != SVDQ_INT4 || cudaMalloc(&w->qR8, 2 * qr_b) == cudaSuccess) &&
+            (fmt != SVDQ_NVFP4 || cudaMalloc(&w->L1f32, (size_t)w->K_pad * r_tot * 4) == cudaSuccess) &&
             cudaMalloc(&w->L1t, (size_t)r_tot * w->K_pad * 2) == cudaSuccess &&
             cudaMalloc(&w->L2a, (size_t)w->N_pad * w->r_pad * 2) == cudaSuccess &&
             cudaMalloc(&w->bias_f, (size_t)w->N_pad * 4) == cudaSuccess &&
@@ -482,6 +487,7 @@ svdq_status svdq_prepare_weights(svdq_format fmt, int K, int N, int rank, const 
   p.sR = w->sR;
   p.sR_rep = w->sR_rep;
   p.qR8 = w->qR8;
+  p.L1f32 = w->L1f32;
   p.L1t = w->L1t;
   p.L2a = w->L2a;
   p.bias_f = w->bias_f;
@@ -680,6 +686,75 @@ svdq_status svdq_linear_dynamic(const svdq_weights* w, int M, const void* X, svd
   if (s != SVDQ_OK) return s;
   if ((s = run_k1(w, M, X, qX, sX, LR, 1, 1, stream, &dyn)) != SVDQ_OK) return s;
   return run_k2(w, M, qX, sX, LR, epi, Y, true, stream, &dyn);
+}
+
+// ---------------------------------------------------------------- one layer into the next
+// [layer 1's workspace | the next layer's LR partials]
+static size_t emit_part_bytes(const svdq_weights* w1, const svdq_weights* w2, int M) {
+  return align256((size_t)2 * (w1->N_pad / 256) * round_up(M, 128) * w2->r_tot * 4);
+}
+
+static svdq_status check_pair(const svdq_weights* w1, const svdq_weights* w2) {
+  if (!w1 || !w2) return SVDQ_ERR_INVALID_ARG;
+  if (w1->fmt != SVDQ_NVFP4 || w2->fmt != SVDQ_NVFP4) return SVDQ_ERR_INVALID_ARG;
+  if (w2->K != w1->N || w2->K_pad != w1->N_pad || w2->r_tot > 32) return SVDQ_ERR_SHAPE;
+  return w1->dev == w2->dev ? SVDQ_OK : SVDQ_ERR_INVALID_ARG;
+}
+
+size_t svdq_linear_emit_next_workspace_bytes(const svdq_weights* w1, const svdq_weights* w2, int M) {
+  if (check_pair(w1, w2) != SVDQ_OK || M < 0) return 0;
+  return svdq_linear_workspace_bytes(w1, M) + emit_part_bytes(w1, w2, M);
+}
+
+svdq_status svdq_linear_emit_next(const svdq_weights* w1, const svdq_weights* w2, int M, const void* X,
+                                  svdq_epilogue epi, void* qX2, void* sX2, void* LR2, void* workspace, size_t ws_bytes,
+                                  cudaStream_t stream) {
+  svdq_status s = check_pair(w1, w2);
+  if (s != SVDQ_OK) return s;
+  if (M > 0 && (!X || !qX2 || !sX2 || !LR2)) return SVDQ_ERR_INVALID_ARG;
+  if (epi != SVDQ_EPI_NONE && epi != SVDQ_EPI_GELU_TANH) return SVDQ_ERR_INVALID_ARG;
+  if (M < 0) return SVDQ_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(qX2) || !aligned16(sX2) || !aligned16(LR2)) return SVDQ_ERR_ALIGNMENT;
+  if (M == 0) return SVDQ_OK;
+  if (!workspace || ws_bytes < svdq_linear_emit_next_workspace_bytes(w1, w2, M)) return SVDQ_ERR_WORKSPACE;
+  void *qX, *sX, *LR;
+  if ((s = carve(w1, M, workspace, ws_bytes, &qX, &sX, &LR)) != SVDQ_OK) return s;
+  float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + svdq_linear_workspace_bytes(w1, M));
+  if ((s = run_k1(w1, M, X, qX, sX, LR, 1, 1, stream)) != SVDQ_OK) return s;
+  K2Params::Next nx;
+  nx.inv_lambda = w2->lambda_inv;
+  nx.L1f32 = w2->L1f32;
+  nx.s_t = w2->s_tX;
+  nx.six_st = 6.0f * w2->s_tX;   // one IEEE float32 multiply, as for kernel 1
+  nx.r_tot = w2->r_tot;
+  nx.qX = static_cast<uint8_t*>(qX2);
+  nx.sX = static_cast<uint8_t*>(sX2);
+  nx.part = part;
+  if ((s = run_k2(w1, M, qX, sX, LR, epi, nullptr, true, stream, nullptr, &nx)) != SVDQ_OK) return s;
+  return from_cuda(launch_next_lr_reduce(part, 2 * (w1->N_pad / 256), M, round_up(M, 128), w2->r_tot, w2->r_pad,
+                                         static_cast<__nv_bfloat16*>(LR2), stream));
+}
+
+size_t svdq_mlp_workspace_bytes(const svdq_weights* w1, const svdq_weights* w2, int M) {
+  if (check_pair(w1, w2) != SVDQ_OK || M < 0) return 0;
+  return svdq_linear_emit_next_workspace_bytes(w1, w2, M) + svdq_linear_workspace_bytes(w2, M);
+}
+
+svdq_status svdq_mlp(const svdq_weights* w1, const svdq_weights* w2, int M, const void* X, svdq_epilogue epi1,
+                     svdq_epilogue epi2, void* Y, void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  svdq_status s = check_pair(w1, w2);
+  if (s != SVDQ_OK) return s;
+  if (M > 0 && (!X || !Y)) return SVDQ_ERR_INVALID_ARG;
+  if (epi2 != SVDQ_EPI_NONE && epi2 != SVDQ_EPI_GELU_TANH) return SVDQ_ERR_INVALID_ARG;
+  if (M < 0) return SVDQ_ERR_SHAPE;
+  if (!aligned16(X) || !aligned16(Y)) return SVDQ_ERR_ALIGNMENT;
+  if (M == 0) return SVDQ_OK;
+  if (!workspace || ws_bytes < svdq_mlp_workspace_bytes(w1, w2, M)) return SVDQ_ERR_WORKSPACE;
+  const size_t e1 = svdq_linear_emit_next_workspace_bytes(w1, w2, M);
+  void *qX2, *sX2, *LR2;
+  if ((s = carve(w2, M, static_cast<uint8_t*>(workspace) + e1, ws_bytes - e1, &qX2, &sX2, &LR2)) != SVDQ_OK) return s;
+  if ((s = svdq_linear_emit_next(w1, w2, M, X, epi1, qX2, sX2, LR2, workspace, e1, stream)) != SVDQ_OK) return s;
+  return run_k2(w2, M, qX2, sX2, LR2, epi2, Y, true, stream);
 }
 
 svdq_status svdq_quantize_act(const svdq_weights* w, int M, const void* X, void* qX, void* sX,

@@ -443,6 +443,13 @@ __device__ __forceinline__ void fma2_rn(float a0, float a1, float b0, float b1, 
   asm("mov.b64 {%0, %1}, %2;" : "=f"(c0), "=f"(c1) : "l"(r));
 }
 
+// Packed float32 pairs in 64-bit registers (element 0 in the low half): a * b + c.
+__device__ __forceinline__ uint64_t fma2_u64(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));

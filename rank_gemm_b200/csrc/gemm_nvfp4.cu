@@ -57,7 +57,8 @@ struct Ctl {
 };
 
 constexpr int BIAS_BYTES = EPI_WARPS * 128 * 4;   // warp-private bias slices
-constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + BIAS_BYTES + 1024 + sizeof(Ctl);
+constexpr int TAB_BYTES = 128 * 4;                // emit mode: the next layer's 1/scale table
+constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + BIAS_BYTES + TAB_BYTES + 1024 + sizeof(Ctl);
 
 // Tile order: groups of 8 row blocks, column blocks within a group, so the
 // CTAs running at the same time share each activation tile among ~8 and each
@@ -85,6 +86,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 }  // namespace
 
+// EMIT: instead of Y, write the next layer's kernel-1 outputs from this
+// layer's bf16 output (see K2Params::Next).
+template <bool EMIT>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const __grid_constant__ CUtensorMap tmLR, const __grid_constant__ CUtensorMap tmL2,
@@ -92,7 +96,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* bias_s = reinterpret_cast<float*>(base + STAGES * STAGE_BYTES);
-  Ctl* ctl = reinterpret_cast<Ctl*>(base + STAGES * STAGE_BYTES + BIAS_BYTES);
+  float* inv_tab2 = reinterpret_cast<float*>(base + STAGES * STAGE_BYTES + BIAS_BYTES);
+  Ctl* ctl = reinterpret_cast<Ctl*>(base + STAGES * STAGE_BYTES + BIAS_BYTES + TAB_BYTES);
   volatile int* abort_flag = &ctl->abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -116,6 +121,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     tmem_alloc(smem_u32(&ctl->tmem_base), TMEM_COLS);
     tmem_relinquish();
   }
+  if (EMIT && threadIdx.x >= 64 && threadIdx.x < 192)
+    inv_tab2[threadIdx.x - 64] = nvfp4_inv_entry((uint32_t)(threadIdx.x - 64), p.next.s_t);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -245,29 +252,111 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (lane == 0) mbar_arrive(smem_u32(&ctl->tempty));
       acc_phase ^= 1;
       const int m = mb * BLOCK_M + row;
-      if (m < p.M) {
-        __nv_bfloat16* yrow = p.Y + (size_t)m * p.N;
-        // 16 columns (32 bytes, one full sector) per store
+      if (!EMIT) {
+        if (m < p.M) {
+          __nv_bfloat16* yrow = p.Y + (size_t)m * p.N;
+          // 16 columns (32 bytes, one full sector) per store
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const int col = c * 32 + q * 16;
+              const int n = n0 + col;
+              if (n < p.N) {
+                float y[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                  y[j] = fmaf(alpha, __uint_as_float(r[c][q * 16 + j]), bslice[col + j]);
+                  if (p.epi == 1) y[j] = gelu_tanh(y[j]);
+                }
+                uint32_t o[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) o[j] = pack_bf16x2(y[2 * j], y[2 * j + 1]);
+                st_global_v8(yrow + n, o);
+              }
+            }
+          }
+        }
+      } else {
+        // ------------------------------------------------ the next layer's kernel 1 on this tile
+        // x2 = bf16(y) is the next layer's activation: its 16-column groups
+        // here are its NVFP4 groups (codes and replicated scales exactly as
+        // kernel 1 writes them), and sum_n x2[m,n] L1f2[n,:] over this
+        // warp's 128 columns is a partial of its LR
+        const K2Params::Next& nx = p.next;
+        const size_t qrow = (size_t)p.N_pad / 2;
+        uint64_t lr[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) lr[i] = 0ull;
+        uint32_t sword = 0u;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
             const int col = c * 32 + q * 16;
             const int n = n0 + col;
-            if (n < p.N) {
-              float y[16];
+            float xb[16];
 #pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                y[j] = fmaf(alpha, __uint_as_float(r[c][q * 16 + j]), bslice[col + j]);
-                if (p.epi == 1) y[j] = gelu_tanh(y[j]);
+            for (int j = 0; j < 16; j += 2) {
+              float y0 = fmaf(alpha, __uint_as_float(r[c][q * 16 + j]), bslice[col + j]);
+              float y1 = fmaf(alpha, __uint_as_float(r[c][q * 16 + j + 1]), bslice[col + j + 1]);
+              if (p.epi == 1) {
+                y0 = gelu_tanh(y0);
+                y1 = gelu_tanh(y1);
               }
-              uint32_t o[8];
+              const uint32_t b2 = pack_bf16x2(y0, y1);
+              xb[j] = __uint_as_float(b2 << 16);
+              xb[j + 1] = __uint_as_float(b2 & 0xFFFF0000u);
+            }
+            // quantize x^2 = fl32(x2 / lambda2) (zero 1/lambda2 past the next layer's K)
+            float v[16];
 #pragma unroll
-              for (int j = 0; j < 8; ++j) o[j] = pack_bf16x2(y[2 * j], y[2 * j + 1]);
-              st_global_v8(yrow + n, o);
+            for (int j = 0; j < 16; j += 4) {
+              float4 il = make_float4(0.f, 0.f, 0.f, 0.f);
+              if (n + j < p.N) il = __ldg(reinterpret_cast<const float4*>(nx.inv_lambda + n + j));
+              v[j] = __fmul_rn(xb[j], il.x);
+              v[j + 1] = __fmul_rn(xb[j + 1], il.y);
+              v[j + 2] = __fmul_rn(xb[j + 2], il.z);
+              v[j + 3] = __fmul_rn(xb[j + 3], il.w);
+            }
+            uint2 codes;
+            uint32_t sc;
+            quant_nvfp4_16_tab(v, nx.six_st, inv_tab2, codes, sc);
+            sword |= sc << (8 * (2 * (c & 1) + q));
+            if (m < p.M) *reinterpret_cast<uint2*>(nx.qX + (size_t)m * qrow + n / 2) = codes;
+            if ((c & 1) && q) {   // the 64-column block's four scales: one word, four replicas
+              const uint32_t wv = m < p.M ? sword : 0u;
+#pragma unroll
+              for (int rep = 0; rep < 4; ++rep)
+                *reinterpret_cast<uint32_t*>(nx.sX + sfx_rep_offset(m, (n0 + c * 32 - 32) / 64, rep, p.N_pad)) = wv;
+              sword = 0u;
+            }
+            // LR partial: lr[i] += x2[n + j] L1f2[n + j][i], two ranks per packed FMA
+#pragma unroll 4
+            for (int j = 0; j < 16; ++j) {
+              const float4* lrow = reinterpret_cast<const float4*>(nx.L1f32 + (size_t)(n + j) * nx.r_tot);
+              const uint64_t xx = ((uint64_t)__float_as_uint(xb[j]) << 32) | __float_as_uint(xb[j]);
+#pragma unroll
+              for (int i4 = 0; i4 < 8; ++i4) {
+                if (4 * i4 < nx.r_tot) {
+                  const float4 l4 = __ldg(lrow + i4);
+                  lr[2 * i4] = fma2_u64(xx, ((uint64_t)__float_as_uint(l4.y) << 32) | __float_as_uint(l4.x), lr[2 * i4]);
+                  lr[2 * i4 + 1] =
+                      fma2_u64(xx, ((uint64_t)__float_as_uint(l4.w) << 32) | __float_as_uint(l4.z), lr[2 * i4 + 1]);
+                }
+              }
             }
           }
         }
+        // this warp's partial: the 128 columns ch of column block nb
+        float* prow = nx.part + ((size_t)(2 * nb + ch) * (p.num_m_blocks * BLOCK_M) + m) * nx.r_tot;
+#pragma unroll
+        for (int i4 = 0; i4 < 8; ++i4)
+          if (4 * i4 < nx.r_tot)
+            *reinterpret_cast<float4*>(prow + 4 * i4) =
+                make_float4(__uint_as_float((uint32_t)lr[2 * i4]), __uint_as_float((uint32_t)(lr[2 * i4] >> 32)),
+                            __uint_as_float((uint32_t)lr[2 * i4 + 1]),
+                            __uint_as_float((uint32_t)(lr[2 * i4 + 1] >> 32)));
       }
     }
   }
@@ -281,8 +370,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 cudaError_t launch_gemm_nvfp4(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmLR,
-                              const CUtensorMap& tmL2, K2Params p, int num_sms, cudaStream_t stream) {
-  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(gemm_nvfp4_kernel), SMEM_BYTES);
+                              const CUtensorMap& tmL2, K2Params p, int num_sms, cudaStream_t stream, bool emit_next) {
+  void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap, K2Params) =
+      emit_next ? gemm_nvfp4_kernel<true> : gemm_nvfp4_kernel<false>;
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int tiles = p.num_m_blocks * p.num_n_blocks;
   const int grid = tiles < num_sms ? tiles : num_sms;
@@ -296,7 +387,25 @@ cudaError_t launch_gemm_nvfp4(const CUtensorMap& tmA, const CUtensorMap& tmB, co
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemm_nvfp4_kernel, tmA, tmB, tmLR, tmL2, p);
+  return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmLR, tmL2, p);
+}
+
+__global__ void next_lr_reduce_kernel(const float* __restrict__ part, int parts, int M, int M_128, int r_tot, int r_pad,
+                                      __nv_bfloat16* LR) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= M * r_pad) return;
+  const int m = i / r_pad, c = i - m * r_pad;
+  float acc = 0.f;
+  if (c < r_tot)
+    for (int q = 0; q < parts; ++q) acc += part[((size_t)q * M_128 + m) * r_tot + c];   // fixed order
+  LR[i] = __float2bfloat16_rn(acc);
+}
+
+cudaError_t launch_next_lr_reduce(const float* part, int parts, int M, int M_128, int r_tot, int r_pad,
+                                  __nv_bfloat16* LR, cudaStream_t stream) {
+  const int n = M * r_pad;
+  next_lr_reduce_kernel<<<(n + 255) / 256, 256, 0, stream>>>(part, parts, M, M_128, r_tot, r_pad, LR);
+  return cudaGetLastError();
 }
 
 }  // namespace svdq

@@ -59,6 +59,17 @@ struct K2Params {
   int epi;                 // 0 none, 1 GELU (tanh form)
   __nv_bfloat16* Y;        // [M][N]
   DeviceErr err;
+  // Emit mode (the next layer's kernel-1 outputs instead of Y): this
+  // layer's bf16 output Y is the next layer's activation X2 (its K = N)
+  struct Next {
+    const float* inv_lambda;   // [N] the next layer's 1/lambda
+    const float* L1f32;        // [N_pad][r_tot] its first factor (with any LoRA A) in fp32
+    float s_t, six_st;         // its static NVFP4 activation tensor scale and fl32(6 s_t)
+    int r_tot;                 // <= 32
+    uint8_t* qX;               // [M][N_pad / 2]
+    uint8_t* sX;               // replicated layout over N_pad (sfx_rep_offset)
+    float* part;               // [2 num_n_blocks][M_128][r_tot] partial LR, one per 128-column half tile
+  } next;
 };
 // TMA box heights the host encodes for kernel 2's operands (rows of a tile):
 // NVFP4 stages 128 rows of qX / LR and 256 rows of qR / L2a per k-tile; INT4
@@ -67,7 +78,11 @@ constexpr int K2_NV_ROWS_A = 128, K2_NV_ROWS_B = 256;
 constexpr int K2_I4_ROWS = 128;
 cudaError_t launch_gemm_nvfp4(const CUtensorMap& tmA, const CUtensorMap& tmB,
                               const CUtensorMap& tmLR, const CUtensorMap& tmL2, K2Params p,
-                              int num_sms, cudaStream_t stream);
+                              int num_sms, cudaStream_t stream, bool emit_next = false);
+// LR of the next layer from the emit mode's partials: bf16 of their sum in
+// partial order, zeros for r_tot <= i < r_pad.
+cudaError_t launch_next_lr_reduce(const float* part, int parts, int M, int M_128, int r_tot, int r_pad,
+                                  __nv_bfloat16* LR, cudaStream_t stream);
 
 struct K2I8Params {
   int M, N, K_pad, r_tot, r_pad, N_pad;
@@ -125,6 +140,7 @@ struct PrepParams {
   uint8_t* sR_rep;             // NVFP4: kernel 2's replicated copy (sfw_rep_offset)
   uint8_t* qR8;                // INT4: kernel 2's copy of the codes as E4M3 bytes [N_pad][K_pad]
   __nv_bfloat16* L1t;          // [K_pad/64][r_tot][64], 128-byte swizzled
+  float* L1f32;                // NVFP4: [K_pad][r_tot] fp32 copy of [L1f | A] (zeros past K), or null
   __nv_bfloat16* L2a;          // [N_pad][r_pad]
   float* bias_f;               // [N_pad]
   float* lambda_inv;           // [K]

@@ -172,6 +172,7 @@ __global__ void factors_kernel(PrepParams p, float alpha) {
     const int kb = k >> 6, c = k & 63;
     const size_t off = (size_t)kb * p.r_tot * 64 + (size_t)r * 64 + ((((c >> 3) ^ (r & 7)) << 3) | (c & 7));
     p.L1t[off] = v;
+    if (p.L1f32) p.L1f32[(size_t)k * p.r_tot + r] = __bfloat162float(v);
   }
   // L2a [N_pad][r_pad] = ([L2 ; B] / alpha)^T, zero padded
   for (int i = tid; i < p.N_pad * p.r_pad; i += stride) {
