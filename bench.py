@@ -42,7 +42,7 @@ sys.path.insert(0, ROOT)
 WORKLOAD = dict(name="nvfp4_qkv_M4608_K3072_N9216_r32", fmt="nvfp4", M=4608, K=3072, N=9216, rank=32)
 # --workload: the QKV projection is the bench line; the others are the
 # remaining parity configurations, timed the same way for their profiles.
-WORKLOADS = ("qkv", "int4_qkv", "mlp_fc1", "mlp_fc2", "lora", "awq_adaln")
+WORKLOADS = ("qkv", "int4_qkv", "mlp_fc1", "mlp_fc2", "lora", "awq_adaln", "mlp_pair")
 INT8_PER_BF16 = 2.0         # nominal dense INT8 : BF16 tensor throughput (4.5 : 2.25)
 METRIC = "SVDQuant W4A4 linear effective TFLOPS & % of FP4 tensor peak; µs/layer"
 UNIT = "TFLOP/s"
@@ -531,6 +531,107 @@ def run_ours(args, world, rank, local):
         print(json.dumps(out), flush=True)
 
 
+# ------------------------------------------------------------------ fused MLP pair arm
+def run_mlp_pair(args, world, rank, local):
+    """The FLUX-like MLP pair (fc1 3072 -> 12288 + GELU, fc2 12288 -> 3072,
+    M = 4608) as one svdq_mlp call per step (fc1's epilogue writes fc2's
+    kernel-1 outputs), against the two layers run separately."""
+    import numpy as np
+    import torch
+    import workloads
+    from rank_gemm_b200 import build as _b
+    if rank == 0:
+        _b.build()
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", init_method="env://", world_size=world, rank=rank,
+                                timeout=__import__("datetime").timedelta(seconds=120))
+        dist.barrier()
+    from rank_gemm_b200 import binding as B
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    l1 = build_layer("mlp_fc1", B, torch, dev)
+    fc1, (W2, b2, _) = workloads.mlp_pair()
+    M, K, N1 = l1["M"], l1["K"], l1["N"]
+    # fc2 prepared on this library's fc1 output, as the mlp_fc2 workload does
+    Y1 = torch.empty(M, N1, dtype=torch.bfloat16, device=dev)
+    ws1 = torch.empty(B.svdq_linear_workspace_bytes(l1["h"], M), dtype=torch.uint8, device=dev)
+    B.svdq_linear(l1["h"], M, l1["X0"], B.SVDQ_EPI_GELU_TANH, Y1, ws1)
+    Wt2 = torch.from_numpy(np.ascontiguousarray(W2.T)).to(torch.bfloat16).to(dev)
+    lam2, act2, L1f2, L22 = gpu_factors(B, Wt2, Y1, 32, torch)
+    h2 = B.svdq_prepare_weights("nvfp4", N1, W2.shape[1], 32, Wt2, lam2, L1f2, L22,
+                                torch.from_numpy(b2).to(torch.bfloat16).to(dev), act_scale=act2)
+    N2 = W2.shape[1]
+    sets = 3
+    Xs = [l1["X0"]] + [l1["X0"].clone() for _ in range(sets - 1)]
+    Ys = [torch.empty(M, N2, dtype=torch.bfloat16, device=dev) for _ in range(sets)]
+    wss = [torch.empty(B.svdq_mlp_workspace_bytes(l1["h"], h2, M), dtype=torch.uint8, device=dev)
+           for _ in range(sets)]
+    stream = torch.cuda.current_stream(dev)
+    step = lambda i: B.svdq_mlp(l1["h"], h2, M, Xs[i % sets], B.SVDQ_EPI_GELU_TANH, B.SVDQ_EPI_NONE, Ys[i % sets],
+                                wss[i % sets], None, stream)
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    max_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+    status = B.svdq_poll_device_error(stream)
+    # the same pair as two separate layers (fc1's bf16 output through HBM)
+    Y1s = [torch.empty(M, N1, dtype=torch.bfloat16, device=dev) for _ in range(sets)]
+    wl1 = [torch.empty(B.svdq_linear_workspace_bytes(l1["h"], M), dtype=torch.uint8, device=dev) for _ in range(sets)]
+    wl2 = [torch.empty(B.svdq_linear_workspace_bytes(h2, M), dtype=torch.uint8, device=dev) for _ in range(sets)]
+
+    def sep(i):
+        B.svdq_linear(l1["h"], M, Xs[i % sets], B.SVDQ_EPI_GELU_TANH, Y1s[i % sets], wl1[i % sets], None, stream)
+        B.svdq_linear(h2, M, Y1s[i % sets], B.SVDQ_EPI_NONE, Ys[i % sets], wl2[i % sets], None, stream)
+    n_sep = min(args.steps, 300)
+    for i in range(3):
+        sep(i)
+    torch.cuda.synchronize()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for i in range(n_sep):
+        sep(i)
+    s1.record(stream)
+    torch.cuda.synchronize()
+    sep_us = max_over_ranks(s0.elapsed_time(s1), world, dev) / n_sep * 1e3
+    us = max_ms / args.steps * 1e3
+    flops = 2.0 * M * K * N1 + 2.0 * M * N1 * N2
+    value = weak_scaling_value(flops, args.steps, world, max_ms)
+    peaks = measured_peaks()
+    out = None
+    if rank == 0:
+        out = {"metric": "SVDQuant W4A4 MLP pair (fc1 + GELU -> fc2) effective TFLOPS; µs/pair", "value": round(value, 3),
+               "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+               "ms_per_step": round(max_ms / args.steps, 5), "us_per_pair": round(us, 2),
+               "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4",
+               "data": "synthetic (seeded, FLUX-shaped MLP), random-init weights",
+               "config": {"workload": "nvfp4_mlp_pair_M%d_3072_12288_3072_r32_gelu" % M, "M": M, "K": K, "N1": N1,
+                          "N2": N2, "rank": 32, "parallelism": "replicas x%d (each rank its own batch)" % world,
+                          "l2": "3 rotating X/Y/workspace sets > 126 MB L2"},
+               "fp4_peak_frac": round(value / world / (peaks["bf16"] * FP4_PER_BF16), 4),
+               "separate_layers_us": round(sep_us, 2), "fused_saving": round(1 - us / sep_us, 4),
+               "gpu_launches": 5 * args.steps, "device_status": status, "clocks": clocks.summary()}
+    B.svdq_free_weights(l1["h"])
+    B.svdq_free_weights(h2)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
 # ------------------------------------------------------------------ AWQ W4A16 arm
 AWQ_METRIC = "AWQ W4A16 linear effective TFLOPS & % of HBM bandwidth; µs/layer"
 
@@ -685,6 +786,8 @@ def main():
         run_reference(args, world, rank)
     elif args.workload == "awq_adaln":
         run_awq(args, world, rank, local)
+    elif args.workload == "mlp_pair":
+        run_mlp_pair(args, world, rank, local)
     else:
         run_ours(args, world, rank, local)
 

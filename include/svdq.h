@@ -23,7 +23,10 @@
  *   - Requirements: K % 64 == 0, N % 16 == 0, M >= 0 (M == 0 is a no-op),
  *     rank + lora_rank a multiple of 16 in [16, 256].
  *   - "dev" pointers are device memory of the current CUDA device; "host"
- *     pointers are host memory.  Every device pointer must be 16-byte aligned.
+ *     pointers are host memory.  Every device pointer must be 16-byte aligned;
+ *     the output Y of the W4A4 layer calls (svdq_linear, svdq_linear_dynamic,
+ *     svdq_linear_unfused, svdq_mlp, svdq_w4a4_gemm_lowrank_up, svdq_w4a4_gemm)
+ *     32-byte aligned, because their GEMM writes Y in 32-byte row segments.
  *   - The caller owns X, Y, qX, sX, LR and any workspace; their sizes come from
  *     the query calls.  The library owns the buffers behind an svdq_weights
  *     handle and frees them in svdq_free_weights.
@@ -76,7 +79,7 @@ typedef enum {
   SVDQ_OK = 0,
   SVDQ_ERR_INVALID_ARG = 1,        /* null pointer, unknown enum, bad scalar */
   SVDQ_ERR_SHAPE = 2,              /* dimension outside the requirements above */
-  SVDQ_ERR_ALIGNMENT = 3,          /* a device pointer is not 16-byte aligned */
+  SVDQ_ERR_ALIGNMENT = 3,          /* a device pointer below its alignment (16 bytes; 32 for a layer's Y) */
   SVDQ_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not compute capability 10.0 */
   SVDQ_ERR_WORKSPACE = 5,          /* workspace missing or smaller than required */
   SVDQ_ERR_CUDA = 6,               /* a CUDA runtime or driver call failed */
@@ -307,7 +310,9 @@ svdq_status svdq_linear_dynamic(const svdq_weights* w, int M, const void* X, svd
  *   per-tile float32 partials added in a fixed order (the same on every run;
  *   float32 summation order differs from kernel 1's, within the LR bound).
  *   Requires both handles NVFP4, w2's K == w1's N and r_tot of w2 <= 32.
- *   qX2, sX2, LR2  dev, sizes from svdq_act_buffer_sizes(w2, M)
+ *   qX2, sX2, LR2  dev, sizes from svdq_act_buffer_sizes(w2, M); qX2 32-byte
+ *                  aligned (each row's codes of a 64-column block go out as
+ *                  one 32-byte store)
  *   workspace      dev, svdq_linear_emit_next_workspace_bytes(w1, w2, M)
  * svdq_mlp: the pair: Y = layer w2 (epilogue epi2) of layer w1 (epi1) of X,
  *   through svdq_linear_emit_next and kernel 2 of w2; Y dev bf16 [M][N2];

@@ -64,7 +64,7 @@ struct svdq_weights {
   uint8_t* sR;
   uint8_t* sR_rep;   // NVFP4: kernel 2's replicated copy of sR
   uint8_t* qR8;      // INT4: kernel 2's copy of qR, one E4M3 byte per code [N_pad][K_pad]
-  float* L1f32;      // NVFP4: [K_pad][r_tot] fp32 copy of [L1f | A], read when the layer before emits into this one
+  uint32_t* L1frag;  // NVFP4, r_tot <= 32: [L1f | A] as mma B fragments, read when the layer before emits into this one
   __nv_bfloat16* L1t;
   __nv_bfloat16* L2a;
   float* bias_f;
@@ -105,6 +105,8 @@ unsigned long long wait_limit_ns() {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// kernel 2 writes Y in 32-byte row segments (one st.global.v8 each)
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 svdq_status from_cuda(cudaError_t e) {
@@ -339,7 +341,7 @@ void free_buffers(svdq_weights* w) {
   cudaFree(w->sR);
   cudaFree(w->sR_rep);
   cudaFree(w->qR8);
-  cudaFree(w->L1f32);
+  cudaFree(w->L1frag);
   cudaFree(w->L1t);
   cudaFree(w->L2a);
   cudaFree(w->bias_f);
@@ -449,7 +451,7 @@ svdq_status svdq_prepare_weights(svdq_format fmt, int K, int N, int rank, const 
   bool ok = cudaMalloc(&w->qR, qr_b) == cudaSuccess && cudaMalloc(&w->sR, sr_b) == cudaSuccess &&
             (fmt != SVDQ_NVFP4 || cudaMalloc(&w->sR_rep, 4 * sr_b) == cudaSuccess) &&
             (fmt != SVDQ_INT4 || cudaMalloc(&w->qR8, 2 * qr_b) == cudaSuccess) &&
-            (fmt != SVDQ_NVFP4 || cudaMalloc(&w->L1f32, (size_t)w->K_pad * r_tot * 4) == cudaSuccess) &&
+            (fmt != SVDQ_NVFP4 || r_tot > 32 || cudaMalloc(&w->L1frag, (size_t)w->K_pad * 64) == cudaSuccess) &&
             cudaMalloc(&w->L1t, (size_t)r_tot * w->K_pad * 2) == cudaSuccess &&
             cudaMalloc(&w->L2a, (size_t)w->N_pad * w->r_pad * 2) == cudaSuccess &&
             cudaMalloc(&w->bias_f, (size_t)w->N_pad * 4) == cudaSuccess &&
@@ -487,7 +489,7 @@ svdq_status svdq_prepare_weights(svdq_format fmt, int K, int N, int rank, const 
   p.sR = w->sR;
   p.sR_rep = w->sR_rep;
   p.qR8 = w->qR8;
-  p.L1f32 = w->L1f32;
+  p.L1frag = w->L1frag;
   p.L1t = w->L1t;
   p.L2a = w->L2a;
   p.bias_f = w->bias_f;
@@ -616,7 +618,7 @@ svdq_status svdq_w4a4_gemm_lowrank_up(const svdq_weights* w, int M, const void* 
   if (!w || (M > 0 && (!qX || !sX || !LR || !Y))) return SVDQ_ERR_INVALID_ARG;
   if (epi != SVDQ_EPI_NONE && epi != SVDQ_EPI_GELU_TANH) return SVDQ_ERR_INVALID_ARG;
   if (M < 0) return SVDQ_ERR_SHAPE;
-  if (!aligned16(qX) || !aligned16(sX) || !aligned16(LR) || !aligned16(Y)) return SVDQ_ERR_ALIGNMENT;
+  if (!aligned16(qX) || !aligned16(sX) || !aligned16(LR) || !aligned32(Y)) return SVDQ_ERR_ALIGNMENT;
   if (M == 0) return SVDQ_OK;
   return run_k2(w, M, qX, sX, LR, epi, Y, true, stream);
 }
@@ -642,7 +644,7 @@ svdq_status svdq_linear(const svdq_weights* w, int M, const void* X, svdq_epilog
   if (!w || (M > 0 && (!X || !Y))) return SVDQ_ERR_INVALID_ARG;
   if (epi != SVDQ_EPI_NONE && epi != SVDQ_EPI_GELU_TANH) return SVDQ_ERR_INVALID_ARG;
   if (M < 0) return SVDQ_ERR_SHAPE;
-  if (!aligned16(X) || !aligned16(Y)) return SVDQ_ERR_ALIGNMENT;
+  if (!aligned16(X) || !aligned32(Y)) return SVDQ_ERR_ALIGNMENT;
   if (M == 0) return SVDQ_OK;
   void *qX, *sX, *LR;
   svdq_status s = carve(w, M, workspace, ws_bytes, &qX, &sX, &LR);
@@ -663,7 +665,7 @@ svdq_status svdq_linear_dynamic(const svdq_weights* w, int M, const void* X, svd
   if (!w || (M > 0 && (!X || !Y))) return SVDQ_ERR_INVALID_ARG;
   if (epi != SVDQ_EPI_NONE && epi != SVDQ_EPI_GELU_TANH) return SVDQ_ERR_INVALID_ARG;
   if (M < 0) return SVDQ_ERR_SHAPE;
-  if (!aligned16(X) || !aligned16(Y)) return SVDQ_ERR_ALIGNMENT;
+  if (!aligned16(X) || !aligned32(Y)) return SVDQ_ERR_ALIGNMENT;
   if (M == 0) return SVDQ_OK;
   if (!workspace || ws_bytes < svdq_linear_dynamic_workspace_bytes(w, M)) return SVDQ_ERR_WORKSPACE;
   void *qX, *sX, *LR;
@@ -691,7 +693,7 @@ svdq_status svdq_linear_dynamic(const svdq_weights* w, int M, const void* X, svd
 // ---------------------------------------------------------------- one layer into the next
 // [layer 1's workspace | the next layer's LR partials]
 static size_t emit_part_bytes(const svdq_weights* w1, const svdq_weights* w2, int M) {
-  return align256((size_t)2 * (w1->N_pad / 256) * round_up(M, 128) * w2->r_tot * 4);
+  return align256((size_t)2 * (w1->N_pad / 256) * round_up(M, 128) * LR_PART_STRIDE * 4);
 }
 
 static svdq_status check_pair(const svdq_weights* w1, const svdq_weights* w2) {
@@ -714,7 +716,7 @@ svdq_status svdq_linear_emit_next(const svdq_weights* w1, const svdq_weights* w2
   if (M > 0 && (!X || !qX2 || !sX2 || !LR2)) return SVDQ_ERR_INVALID_ARG;
   if (epi != SVDQ_EPI_NONE && epi != SVDQ_EPI_GELU_TANH) return SVDQ_ERR_INVALID_ARG;
   if (M < 0) return SVDQ_ERR_SHAPE;
-  if (!aligned16(X) || !aligned16(qX2) || !aligned16(sX2) || !aligned16(LR2)) return SVDQ_ERR_ALIGNMENT;
+  if (!aligned16(X) || !aligned32(qX2) || !aligned16(sX2) || !aligned16(LR2)) return SVDQ_ERR_ALIGNMENT;
   if (M == 0) return SVDQ_OK;
   if (!workspace || ws_bytes < svdq_linear_emit_next_workspace_bytes(w1, w2, M)) return SVDQ_ERR_WORKSPACE;
   void *qX, *sX, *LR;
@@ -723,7 +725,7 @@ svdq_status svdq_linear_emit_next(const svdq_weights* w1, const svdq_weights* w2
   if ((s = run_k1(w1, M, X, qX, sX, LR, 1, 1, stream)) != SVDQ_OK) return s;
   K2Params::Next nx;
   nx.inv_lambda = w2->lambda_inv;
-  nx.L1f32 = w2->L1f32;
+  nx.L1frag = w2->L1frag;
   nx.s_t = w2->s_tX;
   nx.six_st = 6.0f * w2->s_tX;   // one IEEE float32 multiply, as for kernel 1
   nx.r_tot = w2->r_tot;
@@ -747,7 +749,7 @@ svdq_status svdq_mlp(const svdq_weights* w1, const svdq_weights* w2, int M, cons
   if (M > 0 && (!X || !Y)) return SVDQ_ERR_INVALID_ARG;
   if (epi2 != SVDQ_EPI_NONE && epi2 != SVDQ_EPI_GELU_TANH) return SVDQ_ERR_INVALID_ARG;
   if (M < 0) return SVDQ_ERR_SHAPE;
-  if (!aligned16(X) || !aligned16(Y)) return SVDQ_ERR_ALIGNMENT;
+  if (!aligned16(X) || !aligned32(Y)) return SVDQ_ERR_ALIGNMENT;
   if (M == 0) return SVDQ_OK;
   if (!workspace || ws_bytes < svdq_mlp_workspace_bytes(w1, w2, M)) return SVDQ_ERR_WORKSPACE;
   const size_t e1 = svdq_linear_emit_next_workspace_bytes(w1, w2, M);
@@ -778,7 +780,7 @@ svdq_status svdq_w4a4_gemm(const svdq_weights* w, int M, const void* qX, const v
                            cudaStream_t stream) {
   if (!w || (M > 0 && (!qX || !sX || !Y))) return SVDQ_ERR_INVALID_ARG;
   if (M < 0) return SVDQ_ERR_SHAPE;
-  if (!aligned16(qX) || !aligned16(sX) || !aligned16(Y)) return SVDQ_ERR_ALIGNMENT;
+  if (!aligned16(qX) || !aligned16(sX) || !aligned32(Y)) return SVDQ_ERR_ALIGNMENT;
   if (M == 0) return SVDQ_OK;
   return run_k2(w, M, qX, sX, nullptr, SVDQ_EPI_NONE, Y, false, stream);
 }
@@ -811,7 +813,7 @@ svdq_status svdq_linear_unfused(const svdq_weights* w, int M, const void* X, svd
   if (!w || (M > 0 && (!X || !Y))) return SVDQ_ERR_INVALID_ARG;
   if (epi != SVDQ_EPI_NONE && epi != SVDQ_EPI_GELU_TANH) return SVDQ_ERR_INVALID_ARG;
   if (M < 0) return SVDQ_ERR_SHAPE;
-  if (!aligned16(X) || !aligned16(Y)) return SVDQ_ERR_ALIGNMENT;
+  if (!aligned16(X) || !aligned32(Y)) return SVDQ_ERR_ALIGNMENT;
   if (M == 0) return SVDQ_OK;
   void *qX, *sX, *LR;
   svdq_status s = carve(w, M, workspace, ws_bytes, &qX, &sX, &LR);

@@ -45,6 +45,7 @@ constexpr int THREADS = 320;              // producer, MMA, 8 epilogue warps
 constexpr int EPI_WARPS = 8;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0, SFA_COL = 256, SFB_COL = 272;
+constexpr uint32_t STASH_COL = 320;   // emit mode: bf16 pairs of the row slices, 64 columns per half
 constexpr uint32_t IDESC_F4 = idesc_nvf4(BLOCK_M, BLOCK_N);
 constexpr uint32_t IDESC_BF = idesc_bf16_f32(BLOCK_M, BLOCK_N);
 
@@ -58,7 +59,9 @@ struct Ctl {
 
 constexpr int BIAS_BYTES = EPI_WARPS * 128 * 4;   // warp-private bias slices
 constexpr int TAB_BYTES = 128 * 4;                // emit mode: the next layer's 1/scale table
-constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + BIAS_BYTES + TAB_BYTES + 1024 + sizeof(Ctl);
+constexpr int INVL_BYTES = EPI_WARPS * 128 * 4;   // emit mode: warp-private slices of the next layer's 1/lambda
+constexpr size_t SMEM_BYTES =
+    (size_t)STAGES * STAGE_BYTES + BIAS_BYTES + TAB_BYTES + INVL_BYTES + 1024 + sizeof(Ctl);
 
 // Tile order: groups of 8 row blocks, column blocks within a group, so the
 // CTAs running at the same time share each activation tile among ~8 and each
@@ -97,7 +100,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* bias_s = reinterpret_cast<float*>(base + STAGES * STAGE_BYTES);
   float* inv_tab2 = reinterpret_cast<float*>(base + STAGES * STAGE_BYTES + BIAS_BYTES);
-  Ctl* ctl = reinterpret_cast<Ctl*>(base + STAGES * STAGE_BYTES + BIAS_BYTES + TAB_BYTES);
+  float* invl_s = reinterpret_cast<float*>(base + STAGES * STAGE_BYTES + BIAS_BYTES + TAB_BYTES);
+  Ctl* ctl = reinterpret_cast<Ctl*>(base + STAGES * STAGE_BYTES + BIAS_BYTES + TAB_BYTES + INVL_BYTES);
   volatile int* abort_flag = &ctl->abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -217,12 +221,16 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else {
     // -------------------------------------------------------------- epilogue
     // Warp e = warp - 2 drains TMEM lanes 32 (warp % 4) .. +31 (its sub-partition),
-    // columns [128 (e / 4), +128): all four 32-column loads are issued before one
-    // wait, the accumulator is released at once, and the bias / GELU / bf16 /
-    // store work then overlaps the MMAs of the next tile.
+    // the 64-column blocks 2 k + e / 4, k = 0, 1, as four 32-column chunks
+    // c (block c / 2, half c % 2; the two warps of a sub-partition interleave
+    // by 64 columns, so in emit mode each owns whole scale blocks): all four
+    // loads are issued before one wait, the accumulator is released at once,
+    // and the bias / GELU / bf16 / store work then overlaps the MMAs of the
+    // next tile.
     const int e = warp - 2, sub = warp & 3, ch = e >> 2;
     const int row = sub * 32 + lane;
     float* bslice = bias_s + e * 128;
+    float* ilslice = invl_s + e * 128;
     // per-call activation tensor scale: alpha = s_tX s_tR = 2^j from the amax
     // partials (kernel 1 scaled LR to match)
     const float alpha =
@@ -232,20 +240,25 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       int mb, nb;
       tile_coords(tile, p.num_m_blocks, p.num_n_blocks, mb, nb);
-      const int n0 = nb * BLOCK_N + ch * 128;
+      const int n0 = nb * BLOCK_N + ch * 64;   // chunk c covers n0 + 128 (c / 2) + 32 (c % 2) .. +31
       // this warp's 128 bias values, staged before the accumulator is ready
-      const float4 bv = __ldg(reinterpret_cast<const float4*>(p.bias + n0) + lane);
+      const int nl = n0 + 128 * (lane >> 4) + 32 * ((lane >> 3) & 1) + 4 * (lane & 7);   // value 4 lane of the slice
+      const float4 bv = __ldg(reinterpret_cast<const float4*>(p.bias + nl));
+      // emit mode: the next layer's 1/lambda for the same columns (zeros past its K)
+      float4 ilv = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (EMIT && nl < p.N) ilv = __ldg(reinterpret_cast<const float4*>(p.next.inv_lambda + nl));
       __syncwarp();
       reinterpret_cast<float4*>(bslice)[lane] = bv;
+      if (EMIT) reinterpret_cast<float4*>(ilslice)[lane] = ilv;
       __syncwarp();
       if (!mbar_wait(smem_u32(&ctl->tfull), acc_phase, abort_flag, p.err)) break;
       tc_fence_after();
       uint32_t r[4][32];
-      const uint32_t taddr = tmem + ((uint32_t)(sub * 32) << 16) + ACC_COL + ch * 128;
+      const uint32_t taddr = tmem + ((uint32_t)(sub * 32) << 16) + ACC_COL + ch * 64;
       tmem_ld32(taddr, r[0]);
       tmem_ld32(taddr + 32, r[1]);
-      tmem_ld32(taddr + 64, r[2]);
-      tmem_ld32(taddr + 96, r[3]);
+      tmem_ld32(taddr + 128, r[2]);
+      tmem_ld32(taddr + 160, r[3]);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
@@ -260,8 +273,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int c = 0; c < 4; ++c) {
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
-              const int col = c * 32 + q * 16;
-              const int n = n0 + col;
+              const int col = c * 32 + q * 16;   // in bslice
+              const int n = n0 + 128 * (c >> 1) + 32 * (c & 1) + q * 16;
               if (n < p.N) {
                 float y[16];
 #pragma unroll
@@ -285,26 +298,99 @@ __global__ void __launch_bounds__(THREADS, 1)
         // warp's 128 columns is a partial of its LR
         const K2Params::Next& nx = p.next;
         const size_t qrow = (size_t)p.N_pad / 2;
-        uint64_t lr[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) lr[i] = 0ull;
-        uint32_t sword = 0u;
+        // phase A: the row slice to bf16 pairs, parked in free TMEM columns of
+        // this warp's lanes (the fp32 accumulator registers are free after it)
+        const uint32_t stash = tmem + ((uint32_t)(sub * 32) << 16) + STASH_COL + ch * 64;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const int col = c * 32 + q * 16;
-            const int n = n0 + col;
+          for (int j = 0; j < 32; j += 2) {
+            float y0 = fmaf(alpha, __uint_as_float(r[c][j]), bslice[c * 32 + j]);
+            float y1 = fmaf(alpha, __uint_as_float(r[c][j + 1]), bslice[c * 32 + j + 1]);
+            if (p.epi == 1) {
+              y0 = gelu_tanh(y0);
+              y1 = gelu_tanh(y1);
+            }
+            pk[j / 2] = pack_bf16x2(y0, y1);
+          }
+          tmem_st16(stash + c * 16, pk);
+        }
+        tmem_wait_st();
+        // phase B1: the LR partial on the tensor cores (mma.m16n8k16 over this
+        // warp's 32 rows x its 128 columns x 32 ranks).  The A fragments come
+        // straight from the stash with tcgen05.ld.16x256b (all sixteen loads
+        // before one wait), whose k order inside a 16-column group the B
+        // fragments' layout matches; B streams from L2 two groups ahead.
+        const int fi = lane >> 2, fq = lane & 3;
+        float acc[2][4][4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int e2 = 0; e2 < 4; ++e2) acc[h][nt][e2] = 0.f;
+        {
+          uint32_t fr[8][2][4];
+#pragma unroll
+          for (int g = 0; g < 8; ++g) {
+            tmem_ld_16x256b(stash + g * 8, fr[g][0]);                 // rows 0-15 of this warp
+            tmem_ld_16x256b(stash + g * 8 + (16u << 16), fr[g][1]);   // rows 16-31
+          }
+          auto bfrag = [&](int g) {
+            const int nn = n0 + 128 * (g >> 2) + 16 * (g & 3);
+            return reinterpret_cast<const uint4*>(nx.L1frag + ((size_t)(nn >> 4) * 32 + lane) * 8);
+          };
+          uint4 bq[2][2];
+          bq[0][0] = __ldg(bfrag(0));
+          bq[0][1] = __ldg(bfrag(0) + 1);
+          bq[1][0] = __ldg(bfrag(1));
+          bq[1][1] = __ldg(bfrag(1) + 1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int g = 0; g < 8; ++g) {
+            const uint4 b01 = bq[g & 1][0], b23 = bq[g & 1][1];
+            if (g + 2 < 8) {
+              bq[g & 1][0] = __ldg(bfrag(g + 2));
+              bq[g & 1][1] = __ldg(bfrag(g + 2) + 1);
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint32_t* f = fr[g][h];
+              mma_bf16_16816(acc[h][0], f[0], f[2], f[1], f[3], b01.x, b01.y);
+              mma_bf16_16816(acc[h][1], f[0], f[2], f[1], f[3], b01.z, b01.w);
+              mma_bf16_16816(acc[h][2], f[0], f[2], f[1], f[3], b23.x, b23.y);
+              mma_bf16_16816(acc[h][3], f[0], f[2], f[1], f[3], b23.z, b23.w);
+            }
+          }
+        }
+        // this warp's partial over its 128 columns of column block nb: rows
+        // 16 h + fi (+ 8), ranks 8 nt + 2 fq, +1 (zeros past r_tot)
+        float* pbase = nx.part + ((size_t)(2 * nb + ch) * (p.num_m_blocks * BLOCK_M) + mb * BLOCK_M + sub * 32) *
+                                     LR_PART_STRIDE;
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int nt = 0; nt < 4; ++nt)
+            if (8 * nt < nx.r_tot) {
+              float* pr = pbase + (size_t)(16 * h + fi) * LR_PART_STRIDE + 8 * nt + 2 * fq;
+              *reinterpret_cast<float2*>(pr) = make_float2(acc[h][nt][0], acc[h][nt][1]);
+              *reinterpret_cast<float2*>(pr + 8 * LR_PART_STRIDE) = make_float2(acc[h][nt][2], acc[h][nt][3]);
+            }
+        // phase B2: codes and scales, the whole stash in two loads and one wait
+        {
+          uint32_t pa[32], pb[32];
+          tmem_ld32(stash, pa);
+          tmem_ld32(stash + 32, pb);
+          tmem_wait_ld();
+          uint32_t sword = 0u, cw[8];
+#pragma unroll
+          for (int g = 0; g < 8; ++g) {
+            const int n = n0 + 128 * (g >> 2) + 16 * (g & 3);
             float xb[16];
 #pragma unroll
             for (int j = 0; j < 16; j += 2) {
-              float y0 = fmaf(alpha, __uint_as_float(r[c][q * 16 + j]), bslice[col + j]);
-              float y1 = fmaf(alpha, __uint_as_float(r[c][q * 16 + j + 1]), bslice[col + j + 1]);
-              if (p.epi == 1) {
-                y0 = gelu_tanh(y0);
-                y1 = gelu_tanh(y1);
-              }
-              const uint32_t b2 = pack_bf16x2(y0, y1);
+              const uint32_t b2 = g < 4 ? pa[g * 8 + j / 2] : pb[(g - 4) * 8 + j / 2];
               xb[j] = __uint_as_float(b2 << 16);
               xb[j + 1] = __uint_as_float(b2 & 0xFFFF0000u);
             }
@@ -312,8 +398,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             float v[16];
 #pragma unroll
             for (int j = 0; j < 16; j += 4) {
-              float4 il = make_float4(0.f, 0.f, 0.f, 0.f);
-              if (n + j < p.N) il = __ldg(reinterpret_cast<const float4*>(nx.inv_lambda + n + j));
+              const float4 il = *reinterpret_cast<const float4*>(ilslice + g * 16 + j);
               v[j] = __fmul_rn(xb[j], il.x);
               v[j + 1] = __fmul_rn(xb[j + 1], il.y);
               v[j + 2] = __fmul_rn(xb[j + 2], il.z);
@@ -322,41 +407,20 @@ __global__ void __launch_bounds__(THREADS, 1)
             uint2 codes;
             uint32_t sc;
             quant_nvfp4_16_tab(v, nx.six_st, inv_tab2, codes, sc);
-            sword |= sc << (8 * (2 * (c & 1) + q));
-            if (m < p.M) *reinterpret_cast<uint2*>(nx.qX + (size_t)m * qrow + n / 2) = codes;
-            if ((c & 1) && q) {   // the 64-column block's four scales: one word, four replicas
+            sword |= sc << (8 * (g & 3));
+            cw[2 * (g & 3)] = codes.x;
+            cw[2 * (g & 3) + 1] = codes.y;
+            if ((g & 3) == 3) {   // one 64-column block: 32 bytes of codes, one scale word in four replicas
+              const int kb = (n - 48) / 64;
+              if (m < p.M) st_global_v8(nx.qX + (size_t)m * qrow + kb * 32, cw);
               const uint32_t wv = m < p.M ? sword : 0u;
 #pragma unroll
               for (int rep = 0; rep < 4; ++rep)
-                *reinterpret_cast<uint32_t*>(nx.sX + sfx_rep_offset(m, (n0 + c * 32 - 32) / 64, rep, p.N_pad)) = wv;
+                *reinterpret_cast<uint32_t*>(nx.sX + sfx_rep_offset(m, kb, rep, p.N_pad)) = wv;
               sword = 0u;
-            }
-            // LR partial: lr[i] += x2[n + j] L1f2[n + j][i], two ranks per packed FMA
-#pragma unroll 4
-            for (int j = 0; j < 16; ++j) {
-              const float4* lrow = reinterpret_cast<const float4*>(nx.L1f32 + (size_t)(n + j) * nx.r_tot);
-              const uint64_t xx = ((uint64_t)__float_as_uint(xb[j]) << 32) | __float_as_uint(xb[j]);
-#pragma unroll
-              for (int i4 = 0; i4 < 8; ++i4) {
-                if (4 * i4 < nx.r_tot) {
-                  const float4 l4 = __ldg(lrow + i4);
-                  lr[2 * i4] = fma2_u64(xx, ((uint64_t)__float_as_uint(l4.y) << 32) | __float_as_uint(l4.x), lr[2 * i4]);
-                  lr[2 * i4 + 1] =
-                      fma2_u64(xx, ((uint64_t)__float_as_uint(l4.w) << 32) | __float_as_uint(l4.z), lr[2 * i4 + 1]);
-                }
-              }
             }
           }
         }
-        // this warp's partial: the 128 columns ch of column block nb
-        float* prow = nx.part + ((size_t)(2 * nb + ch) * (p.num_m_blocks * BLOCK_M) + m) * nx.r_tot;
-#pragma unroll
-        for (int i4 = 0; i4 < 8; ++i4)
-          if (4 * i4 < nx.r_tot)
-            *reinterpret_cast<float4*>(prow + 4 * i4) =
-                make_float4(__uint_as_float((uint32_t)lr[2 * i4]), __uint_as_float((uint32_t)(lr[2 * i4] >> 32)),
-                            __uint_as_float((uint32_t)lr[2 * i4 + 1]),
-                            __uint_as_float((uint32_t)(lr[2 * i4 + 1] >> 32)));
       }
     }
   }
@@ -397,7 +461,7 @@ __global__ void next_lr_reduce_kernel(const float* __restrict__ part, int parts,
   const int m = i / r_pad, c = i - m * r_pad;
   float acc = 0.f;
   if (c < r_tot)
-    for (int q = 0; q < parts; ++q) acc += part[((size_t)q * M_128 + m) * r_tot + c];   // fixed order
+    for (int q = 0; q < parts; ++q) acc += part[((size_t)q * M_128 + m) * LR_PART_STRIDE + c];   // fixed order
   LR[i] = __float2bfloat16_rn(acc);
 }
 

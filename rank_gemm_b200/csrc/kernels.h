@@ -63,14 +63,26 @@ struct K2Params {
   // layer's bf16 output Y is the next layer's activation X2 (its K = N)
   struct Next {
     const float* inv_lambda;   // [N] the next layer's 1/lambda
-    const float* L1f32;        // [N_pad][r_tot] its first factor (with any LoRA A) in fp32
+    const uint32_t* L1frag;    // its first factor (with any LoRA A) as m16n8k16 B fragments (l1frag_offset)
     float s_t, six_st;         // its static NVFP4 activation tensor scale and fl32(6 s_t)
     int r_tot;                 // <= 32
     uint8_t* qX;               // [M][N_pad / 2]
     uint8_t* sX;               // replicated layout over N_pad (sfx_rep_offset)
-    float* part;               // [2 num_n_blocks][M_128][r_tot] partial LR, one per 128-column half tile
+    float* part;               // [2 num_n_blocks][M_128][LR_PART_STRIDE] partial LR, one per warp column set
   } next;
 };
+constexpr int LR_PART_STRIDE = 32;   // floats per row of an emit-mode LR partial
+// Emit mode's copy of a first factor L1 ([K][r_tot] bf16, r_tot <= 32, zeros
+// past K and r_tot) in the B-fragment order of mma.m16n8k16 over 16-row k
+// groups: the bf16 offset of element (k, r).  Lane t of a warp holds, for
+// rank 8 nt + t / 4, the four consecutive k = 16 G + 4 (t % 4) .. +3 as two
+// registers (b0, b1) at word 2 nt, 2 nt + 1 of its 8 words per group; the k
+// order this gives inside a group matches the A fragments read from TMEM with
+// tcgen05.ld.16x256b (slot pair s < 4 <- pair 2 s, slot pair s + 4 <- pair 2 s + 1).
+__host__ __device__ __forceinline__ size_t l1frag_offset(int k, int r) {
+  const int G = k >> 4, kk = k & 15, t = 4 * (r & 7) + (kk >> 2);
+  return (((size_t)G * 32 + t) * 8 + 2 * (r >> 3)) * 2 + (kk & 3);
+}
 // TMA box heights the host encodes for kernel 2's operands (rows of a tile):
 // NVFP4 stages 128 rows of qX / LR and 256 rows of qR / L2a per k-tile; INT4
 // stages 128 of each.
@@ -140,7 +152,7 @@ struct PrepParams {
   uint8_t* sR_rep;             // NVFP4: kernel 2's replicated copy (sfw_rep_offset)
   uint8_t* qR8;                // INT4: kernel 2's copy of the codes as E4M3 bytes [N_pad][K_pad]
   __nv_bfloat16* L1t;          // [K_pad/64][r_tot][64], 128-byte swizzled
-  float* L1f32;                // NVFP4: [K_pad][r_tot] fp32 copy of [L1f | A] (zeros past K), or null
+  uint32_t* L1frag;            // NVFP4 with r_tot <= 32: [L1f | A] in l1frag_offset order ([K_pad / 16][32][8] words), or null
   __nv_bfloat16* L2a;          // [N_pad][r_pad]
   float* bias_f;               // [N_pad]
   float* lambda_inv;           // [K]

@@ -215,6 +215,36 @@ def test_capability_check_rejects_other_devices(B):
         g.close()
 
 
+def test_output_alignment_is_checked_before_launch(B):
+    """The 4-bit GEMM writes Y in 32-byte row segments: a Y that is 16- but not
+    32-byte aligned is refused on the host (status 3) before any launch, and
+    a 32-byte aligned one inside the same buffer works."""
+    for fmt in ("nvfp4", "int4"):
+        L = workloads.draw_layer("align", fmt, 32, 256, 256, 16, seed=20, n_out=2)
+        g = GpuLayer(L.fmt, L.X, L.W, L.bias, L.rank)
+        try:
+            Xd = dev_bf16(L.X)
+            buf = torch.empty(L.M * L.N + 32, dtype=torch.bfloat16, device="cuda")
+            assert buf.data_ptr() % 32 == 0
+            Y16 = buf[8: 8 + L.M * L.N]            # 16 bytes past a 32-byte boundary
+            ws = torch.empty(B.svdq_linear_workspace_bytes(g.h, L.M), dtype=torch.uint8, device="cuda")
+            calls = [lambda Y: B.svdq_linear(g.h, L.M, Xd, 0, Y, ws),
+                     lambda Y: B.svdq_linear_unfused(g.h, L.M, Xd, 0, Y, ws)]
+            for call in calls:
+                with pytest.raises(B.SvdqError) as e:
+                    call(Y16)
+                assert e.value.status == 3
+            torch.cuda.synchronize()
+            assert B.svdq_poll_device_error() == 0
+            Y32 = buf[16: 16 + L.M * L.N]
+            B.svdq_linear(g.h, L.M, Xd, 0, Y32, ws)
+            ref = torch.empty(L.M, L.N, dtype=torch.bfloat16, device="cuda")
+            B.svdq_linear(g.h, L.M, Xd, 0, ref, ws)
+            assert torch.equal(Y32.view(L.M, L.N), ref)
+        finally:
+            g.close()
+
+
 # ------------------------------------------------------------------ INT4 (int8 tensor-core path)
 def test_int4_small_parity(B):
     L = workloads.draw_layer("int4", "int4", 200, 512, 384, 32, seed=21, n_out=4)
