@@ -606,8 +606,31 @@ def run_mlp_pair(args, world, rank, local):
     s1.record(stream)
     torch.cuda.synchronize()
     sep_us = max_over_ranks(s0.elapsed_time(s1), world, dev) / n_sep * 1e3
+    # the pair's two calls timed apart: fc1 in emit mode (kernel 1, kernel 2
+    # writing fc2's kernel-1 outputs, the LR reduction), then fc2's kernel 2
+    qs, ss, ls = B.svdq_act_buffer_sizes(h2, M)
+    nb = [[torch.empty(v, dtype=torch.uint8, device=dev) for v in (qs, ss, ls)] for _ in range(sets)]
+    wse = [torch.empty(B.svdq_linear_emit_next_workspace_bytes(l1["h"], h2, M), dtype=torch.uint8, device=dev)
+           for _ in range(sets)]
+
+    def part_us(fn):
+        for i in range(3):
+            fn(i)
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for i in range(n_sep):
+            fn(i)
+        a1.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(a0.elapsed_time(a1), world, dev) / n_sep * 1e3
+    emit_us = part_us(lambda i: B.svdq_linear_emit_next(l1["h"], h2, M, Xs[i % sets], B.SVDQ_EPI_GELU_TANH,
+                                                        *nb[i % sets], wse[i % sets], None, stream))
+    fc2_us = part_us(lambda i: B.svdq_w4a4_gemm_lowrank_up(h2, M, *nb[i % sets], B.SVDQ_EPI_NONE, Ys[i % sets],
+                                                           stream))
     us = max_ms / args.steps * 1e3
     flops = 2.0 * M * K * N1 + 2.0 * M * N1 * N2
+    fc1_flops = 2.0 * M * K * N1
     value = weak_scaling_value(flops, args.steps, world, max_ms)
     peaks = measured_peaks()
     out = None
@@ -622,7 +645,13 @@ def run_mlp_pair(args, world, rank, local):
                           "l2": "3 rotating X/Y/workspace sets > 126 MB L2"},
                "fp4_peak_frac": round(value / world / (peaks["bf16"] * FP4_PER_BF16), 4),
                "separate_layers_us": round(sep_us, 2), "fused_saving": round(1 - us / sep_us, 4),
-               "gpu_launches": 5 * args.steps, "device_status": status, "clocks": clocks.summary()}
+               "split_us": {"fc1_emit": round(emit_us, 2), "fc2_kernel2": round(fc2_us, 2)},
+               "roofline": {"bound": "tensor", "kernel": "fc1 in emit mode (kernel 1 + emit kernel 2 + LR reduce)",
+                            "achieved": round(fc1_flops / (emit_us * 1e-6) / 1e12, 2),
+                            "peak": round(peaks["bf16"] * FP4_PER_BF16, 1), "unit": "TFLOP/s",
+                            "frac": round(fc1_flops / (emit_us * 1e-6) / 1e12 / (peaks["bf16"] * FP4_PER_BF16), 4),
+                            "traffic": None},
+               "gpu_launches": 4 * args.steps, "device_status": status, "clocks": clocks.summary()}
     B.svdq_free_weights(l1["h"])
     B.svdq_free_weights(h2)
     if world > 1:
