@@ -24,9 +24,10 @@
  *     rank + lora_rank a multiple of 16 in [16, 256].
  *   - "dev" pointers are device memory of the current CUDA device; "host"
  *     pointers are host memory.  Every device pointer must be 16-byte aligned;
- *     the output Y of the W4A4 layer calls (svdq_linear, svdq_linear_dynamic,
- *     svdq_linear_unfused, svdq_mlp, svdq_w4a4_gemm_lowrank_up, svdq_w4a4_gemm)
- *     32-byte aligned, because their GEMM writes Y in 32-byte row segments.
+ *     the output Y of the W4A4 layer calls (svdq_linear, svdq_linear_noalloc,
+ *     svdq_linear_dynamic, svdq_linear_unfused, svdq_mlp,
+ *     svdq_w4a4_gemm_lowrank_up, svdq_w4a4_gemm) 32-byte aligned, because
+ *     their GEMM writes Y in 32-byte row segments.
  *   - The caller owns X, Y, qX, sX, LR and any workspace; their sizes come from
  *     the query calls.  The library owns the buffers behind an svdq_weights
  *     handle and frees them in svdq_free_weights.
