@@ -22,10 +22,16 @@
 //               tile, then tcgen05.mma.kind::f16 adds LR (L2/alpha) into the
 //               same tile; tcgen05.commit releases ring slots and hands the
 //               finished tile to the epilogue.
-//   warps 2-9   epilogue: two warps per TMEM sub-partition, 128 columns each;
+//   warps 2-9   epilogue: two warps per TMEM sub-partition, 128 columns each
+//               (two 64-column blocks, interleaved with the other warp's);
 //               the whole 128 x 256 tile is loaded to registers and the TMEM
 //               accumulator released before y = alpha acc + b, optional GELU,
-//               bf16 and the 16-byte stores, which overlap the next tile's MMAs.
+//               bf16 and the 32-byte stores, which overlap the next tile's MMAs.
+//               In emit mode (cross-layer fusion) the epilogue instead writes
+//               the next layer's kernel-1 outputs: its NVFP4 codes and
+//               replicated scales, and float32 partials of its low-rank down
+//               projection computed with mma.sync from bf16 pairs parked in
+//               free TMEM columns.
 // All waits are bounded (see mbar_wait); TMEM is freed on every exit path.
 #include "common.cuh"
 #include "kernels.h"
