@@ -82,6 +82,34 @@ def test_argument_errors_before_device(B):
     assert L.svdq_selftest_wait_timeout(0, None) == 1
 
 
+
+def test_argument_errors_of_the_wider_calls(B):
+    """The per-call-scale, cross-layer, W4A16 and device-split entries also
+    reject bad arguments with a status before touching the device."""
+    L = B.lib
+    # per-call tensor scale: null handle
+    assert L.svdq_linear_dynamic(None, 4, 16, 0, 32, 16, 1 << 20, None) == 1
+    # cross-layer fusion: null handles; sizes of an invalid pair are 0
+    assert L.svdq_linear_emit_next(None, None, 4, 16, 0, 32, 16, 16, 16, 1 << 20, None) == 1
+    assert L.svdq_mlp(None, None, 4, 16, 0, 0, 32, 16, 1 << 20, None) == 1
+    assert L.svdq_linear_emit_next_workspace_bytes(None, None, 64) == 0
+    assert L.svdq_mlp_workspace_bytes(None, None, 64) == 0
+    # AWQ W4A16: null output / weight, K % 64, alignment; null handle
+    h = ctypes.c_void_p()
+    assert L.svdq_awq_prepare(64, 16, 16, None, None, None, None) == 1
+    assert L.svdq_awq_prepare(64, 16, None, None, None, None, ctypes.byref(h)) == 1
+    assert L.svdq_awq_prepare(96, 16, 16, None, None, None, ctypes.byref(h)) == 2
+    assert L.svdq_awq_prepare(64, 0, 16, None, None, None, ctypes.byref(h)) == 2
+    assert L.svdq_awq_prepare(64, 16, 24, None, None, None, ctypes.byref(h)) == 3
+    assert h.value is None
+    assert L.svdq_awq_linear(None, 1, 16, 16, None) == 1
+    # device split: null pointers, rank outside [1, min(K, N)], alignment
+    assert L.svdq_lowrank_factors(64, 32, 8, None, 16, 5, 16, 16, None, None) == 1
+    assert L.svdq_lowrank_factors(64, 32, 0, 16, 16, 5, 16, 16, None, None) == 2
+    assert L.svdq_lowrank_factors(64, 32, 33, 16, 16, 5, 16, 16, None, None) == 2
+    assert L.svdq_lowrank_factors(64, 32, 8, 16, 24, 5, 16, 16, None, None) == 3
+
+
 def test_no_gpu_means_unsupported_device(B):
     import torch
     if torch.cuda.is_available():
