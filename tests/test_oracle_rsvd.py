@@ -66,3 +66,21 @@ def test_signs_and_near_optimality_on_the_synthetic_layer():
     assert err <= opt * 1.02
     # the outlier-driven leading values are found to high accuracy
     assert np.allclose(s[:4], sv[:4], rtol=1e-8)
+
+
+def test_folded_factors_rebuild_the_smoothed_weight():
+    """With W of exact rank r and power-of-two lambda (exact scaling), the
+    folded factors rebuild diag(lambda) W through diag(lambda) L1f L2 up to
+    their bf16 rounding: the fold divides U_r Sigma_r by lambda, once."""
+    from oracle import formats as F
+    rng = np.random.default_rng(3)
+    K, N, k = 128, 96, 8
+    W = _orth(rng, K, k) @ np.diag(np.linspace(3.0, 0.5, k)) @ _orth(rng, N, k).T
+    lam = (2.0 ** rng.integers(-3, 4, size=K)).astype(np.float32)
+    L1f, L2, sigma = R.randomized_factors(W, lam, k)
+    assert np.array_equal(F.bf16_round(L1f), L1f) and np.array_equal(F.bf16_round(L2), L2)
+    target = lam.astype(np.float64)[:, None] * W
+    rebuilt = lam.astype(np.float64)[:, None] * (L1f @ L2)
+    assert np.linalg.norm(rebuilt - target) <= 2.0 ** -7 * np.linalg.norm(target)
+    # and the singular values are those of diag(lambda) W
+    assert np.allclose(sigma[:k], np.linalg.svd(target, compute_uv=False)[:k], rtol=1e-10)
