@@ -6,7 +6,9 @@ import numpy as np
 from oracle import awq as A
 from oracle import formats as F
 from oracle import rsvd as R
+from oracle import svdquant as S
 import test_oracle_awq as TA
+import test_oracle_quant as TQ
 import test_oracle_rsvd as TR
 
 
@@ -111,3 +113,26 @@ def test_mutation_lambda_multiplied_into_the_first_factor(monkeypatch):
         return F.bf16_round(U * sigma[None, :rank] * lam64[:, None]), F.bf16_round(Vt), sigma
     monkeypatch.setattr(R, "randomized_factors", bad)
     assert _fails(TR.test_folded_factors_rebuild_the_smoothed_weight)
+
+
+# ---------------------------------------------------------------- per-call activation tensor scale
+def test_mutation_dynamic_scale_exponent_not_smallest(monkeypatch):
+    def bad(pw, X):                                    # frexp's exponent taken as is: one power too high at a tie
+        Xh = S.smooth_activation(X, pw.inv_lam)
+        a = float(np.max(np.abs(Xh))) if np.size(Xh) else 0.0
+        x = (a if a > 0 else 2688.0) * float(np.float32(pw.s_tR)) / 2688.0
+        j = int(np.frexp(x)[1])
+        return np.float32(np.float32(np.ldexp(1.0, j)) / np.float32(pw.s_tR)), j
+    monkeypatch.setattr(S, "dynamic_act_scale", bad)
+    assert _fails(TQ.test_dynamic_scale_is_tight_at_an_exact_power_of_two)
+
+
+def test_mutation_dynamic_scale_exponent_rounded_down(monkeypatch):
+    def bad(pw, X):                                    # largest j with 2^j <= x: the scale no longer covers the batch
+        Xh = S.smooth_activation(X, pw.inv_lam)
+        a = float(np.max(np.abs(Xh))) if np.size(Xh) else 0.0
+        x = (a if a > 0 else 2688.0) * float(np.float32(pw.s_tR)) / 2688.0
+        j = int(np.floor(np.log2(x)))
+        return np.float32(np.float32(np.ldexp(1.0, j)) / np.float32(pw.s_tR)), j
+    monkeypatch.setattr(S, "dynamic_act_scale", bad)
+    assert _fails(TQ.test_dynamic_scale_pairs_to_a_power_of_two_and_covers_the_batch)

@@ -142,6 +142,21 @@ def test_dynamic_scale_pairs_to_a_power_of_two_and_covers_the_batch():
         assert F.e4m3_decode(sX).max() <= 448.0
 
 
+def test_dynamic_scale_is_tight_at_an_exact_power_of_two():
+    # "smallest j with 2^j >= s_tR a / 2688": when that ratio is exactly 2^t,
+    # j = t and the scale is tight (s 2688 = a), not one power above
+    from dataclasses import replace
+    L, pw = _prepared_small()
+    for t_r, k in ((-10, 3), (-7, -2), (-12, 0)):
+        pw2 = replace(pw, s_tR=np.float32(2.0 ** t_r), inv_lam=np.ones_like(pw.inv_lam))
+        X = np.zeros((4, L.K), np.float32)
+        X[1, 5] = np.float32(-2688.0 * 2.0 ** k)      # exact in bf16: 2688 = 21 * 2^7
+        X[2, 7] = np.float32(1.5)
+        s, j = S.dynamic_act_scale(pw2, X)
+        assert j == k + t_r
+        assert float(s) * 2688.0 == 2688.0 * 2.0 ** k
+
+
 def test_dynamic_scale_is_equivariant_under_powers_of_two():
     # scaling X by 2^p scales the dynamic tensor scale by 2^p exactly and leaves every code and block scale
     L, pw = _prepared_small()
