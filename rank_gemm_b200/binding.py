@@ -99,10 +99,18 @@ EXPORTED = tuple(_SIGS)
 
 
 def _ptr(t) -> Optional[int]:
+    """Device address of a tensor argument (every tensor the ABI takes is
+    device memory read as a packed array): a host tensor or a strided view
+    is refused here, before the call, instead of being read as raw memory."""
     if t is None:
         return None
     if isinstance(t, int):
         return t
+    if isinstance(t, torch.Tensor):
+        if not t.is_cuda:
+            raise ValueError("svdq: a tensor argument is in host memory; the library takes device memory")
+        if not t.is_contiguous():
+            raise ValueError("svdq: a tensor argument is not contiguous; the library reads packed arrays")
     return t.data_ptr()
 
 

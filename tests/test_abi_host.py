@@ -119,3 +119,16 @@ def test_no_gpu_means_unsupported_device(B):
                                       ctypes.byref(h)) == 4
     assert B.lib.svdq_poll_device_error(None) == 4
     assert B.lib.svdq_calibrate(4, 64, 16, 16, 16, ctypes.c_float(0.5), 16, 16, 16, 1 << 20, None) == 4
+
+
+def test_binding_refuses_host_and_strided_tensors(B):
+    """Tensor arguments are device memory read as packed arrays: the binding
+    refuses a host tensor before the call (a host address given to a kernel
+    as device memory would fault), and passes None and integers through."""
+    import torch
+    assert B._ptr(None) is None and B._ptr(16) == 16
+    with pytest.raises(ValueError, match="host memory"):
+        B._ptr(torch.zeros(4))
+    with pytest.raises(ValueError, match="host memory"):
+        B.svdq_linear(None, 4, torch.zeros(4, 64, dtype=torch.bfloat16), 0,
+                      torch.zeros(4, 16, dtype=torch.bfloat16), torch.zeros(1024, dtype=torch.uint8))
