@@ -196,3 +196,31 @@ def test_low_rank_branch_reduces_quantization_error():
     e_smooth = err(lam, 0)
     e_plain = err(np.ones(L.K, np.float32), 0)
     assert e_svdq < e_smooth < e_plain, (e_svdq, e_smooth, e_plain)
+
+
+# ------------------------------------------------------------ the fused GELU (tanh form)
+def check_gelu_tanh():
+    """gelu_tanh against PyTorch's own float64 tanh-approximation GELU (an
+    implementation independent of this oracle) on a dense grid and far
+    tails, plus facts that hold for the tanh form only: it is odd-symmetric
+    about y/2 (g(y) - g(-y) = y), g(0) = 0, it differs from the erf-form GELU
+    by at most 5e-4 but by more than 1e-4 near |y| = 2 (so it is not the erf
+    form), and at y = 1 it equals 0.5 (1 + tanh(1.044715 sqrt(2/pi))) written
+    with tanh from Python's math module."""
+    import math
+    import torch
+    y = np.concatenate([np.arange(-12.0, 12.0, 1.0 / 64), [-1e3, -40.0, 40.0, 1e3], [0.0]])
+    g = S.gelu_tanh(y)
+    ref = torch.nn.functional.gelu(torch.from_numpy(y), approximate="tanh").numpy()
+    assert np.all(np.abs(g - ref) <= 1e-14 * np.maximum(1.0, np.abs(ref))), np.max(np.abs(g - ref))
+    assert S.gelu_tanh(np.array([0.0]))[0] == 0.0
+    assert np.all(np.abs(S.gelu_tanh(y) - S.gelu_tanh(-y) - y) <= 1e-13 * np.maximum(1.0, np.abs(y)))
+    erf_form = np.array([0.5 * v * (1.0 + math.erf(v / math.sqrt(2.0))) for v in y])
+    gap = np.abs(g - erf_form)
+    assert gap.max() <= 5e-4 and gap[np.abs(np.abs(y) - 2.0) < 0.5].max() > 1e-4
+    one = 0.5 * (1.0 + math.tanh(math.sqrt(2.0 / math.pi) * 1.044715))
+    assert abs(S.gelu_tanh(np.array([1.0]))[0] - one) <= 1e-15
+
+
+def test_gelu_tanh_matches_the_tanh_form():
+    check_gelu_tanh()

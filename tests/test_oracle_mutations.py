@@ -8,6 +8,7 @@ from oracle import formats as F
 from oracle import svdquant as S
 import test_oracle_formats as TF
 import test_oracle_layer as TL
+import test_oracle_quant as TQ
 
 
 def _fails(fn, *a, **k):
@@ -78,3 +79,50 @@ def test_mutation_lowrank_not_rounded(monkeypatch):
     orig = S.lowrank_down
     monkeypatch.setattr(S, "lowrank_down", lambda X, L1f, round_bf16=True: orig(X, L1f, False))
     assert _fails(TL.check_brute_force, "nvfp4", 8, 16, 16, 4, 41)
+
+
+def test_mutation_act_tensor_scale_divides_by_448(monkeypatch):
+    def bad(X, inv_lam):
+        a = np.float32(np.max(np.abs(S.smooth_activation(X, inv_lam)))) if np.size(X) else np.float32(0)
+        return np.float32(1.0) if a == 0 else np.float32(a / np.float32(448.0))
+    monkeypatch.setattr(S, "act_tensor_scale", bad)
+    assert _fails(TQ.check_act_tensor_scale_definition)
+
+
+def test_mutation_act_tensor_scale_amax_over_raw_x(monkeypatch):
+    def bad(X, inv_lam):
+        a = np.float32(np.max(np.abs(np.asarray(X, np.float32)))) if np.size(X) else np.float32(0)
+        return np.float32(1.0) if a == 0 else np.float32(a / S.NVFP4_TENSOR_DIVISOR)
+    monkeypatch.setattr(S, "act_tensor_scale", bad)
+    assert _fails(TQ.check_act_tensor_scale_definition)
+
+
+def test_mutation_act_tensor_scale_without_abs(monkeypatch):
+    def bad(X, inv_lam):
+        a = np.float32(np.max(S.smooth_activation(X, inv_lam))) if np.size(X) else np.float32(0)
+        return np.float32(1.0) if a == 0 else np.float32(a / S.NVFP4_TENSOR_DIVISOR)
+    monkeypatch.setattr(S, "act_tensor_scale", bad)
+    assert _fails(TQ.check_act_tensor_scale_definition)
+
+
+def test_mutation_gelu_erf_form(monkeypatch):
+    import math
+    monkeypatch.setattr(S, "gelu_tanh", lambda y: np.array(
+        [0.5 * v * (1.0 + math.erf(v / math.sqrt(2.0))) for v in np.asarray(y, np.float64).ravel()]).reshape(np.shape(y)))
+    assert _fails(TL.check_gelu_tanh)
+
+
+def test_mutation_gelu_wrong_cubic_coefficient(monkeypatch):
+    def bad(y):
+        y = np.asarray(y, np.float64)
+        return 0.5 * y * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (y + 0.0447 * y ** 3)))
+    monkeypatch.setattr(S, "gelu_tanh", bad)
+    assert _fails(TL.check_gelu_tanh)
+
+
+def test_mutation_gelu_missing_half(monkeypatch):
+    def bad(y):
+        y = np.asarray(y, np.float64)
+        return y * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (y + 0.044715 * y ** 3)))
+    monkeypatch.setattr(S, "gelu_tanh", bad)
+    assert _fails(TL.check_gelu_tanh)

@@ -182,3 +182,35 @@ def test_dynamic_forward_tracks_the_batch_where_the_static_scale_saturates():
     e_dynamic = rel(S.forward(pw, X, dynamic=True)["Y"], X)
     assert e_dynamic < 1.05 * e_calib + 1e-4
     assert e_static > 3 * e_dynamic
+
+
+# ------------------------------------------------------------ static NVFP4 activation tensor scale
+def check_act_tensor_scale_definition():
+    """act_tensor_scale = amax(|X^|) / 2688 (2688 = 6 x 448, the largest
+    E2M1 magnitude times the largest E4M3 block scale), with X^ = X / lambda.
+    Hand-built so that every step is exact: lambda is a power of two per
+    channel, the largest |X^| is 336 = 2688 / 8 (so the scale is 0.125), it
+    is a negative entry, and it sits in a channel whose raw |X| is NOT the
+    largest (channel 3 holds |X| = 400, which lambda = 4 brings down to 100).
+    Dividing by 448, taking the amax over X instead of X^, or dropping the
+    absolute value all give another number."""
+    lam = np.array([1.0, 2.0, 0.5, 4.0], np.float32)
+    X = np.array([[10.0, -30.0, -168.0, 400.0],
+                  [-50.0, 60.0, 20.0, -8.0]], np.float32)
+    inv = S.inverse_lambda(lam)
+    assert np.array_equal(inv, np.array([1.0, 0.5, 2.0, 0.25], np.float32))
+    s = S.act_tensor_scale(X, inv)
+    assert s.dtype == np.float32 and s == np.float32(0.125), s
+    # a second exact point: amax(|X^|) = 2688 * 2^-10 -> 2^-10
+    X2 = np.array([[2.625, -1.0, 0.5, 0.0]], np.float32)            # X^ = 2.625, -0.5, 1, 0
+    assert S.act_tensor_scale(X2, inv) == np.float32(2.0 ** -10)
+    # an all-zero calibration batch gives the reading's fallback of 1
+    assert S.act_tensor_scale(np.zeros((3, 4), np.float32), inv) == np.float32(1.0)
+    # with the calibrated scale, the block holding the batch's amax gets the
+    # largest E4M3 block scale, 448, and its amax element code 6 (E2M1 0x7)
+    codes, sc = S.quantize_nvfp4(np.pad(S.smooth_activation(X, inv), ((0, 0), (0, 12))), s)
+    assert F.e4m3_decode(sc[0])[0] == 448.0 and codes[0, 2] == 0xF    # -6: sign bit + code 7
+
+
+def test_act_tensor_scale_definition():
+    check_act_tensor_scale_definition()
