@@ -132,17 +132,55 @@ def read_device(ptr: int, nbytes: int) -> np.ndarray:
 
 
 # ------------------------------------------------------------------ tolerance
+def bf16_ulp(v):
+    """Spacing of bf16 values at |v| (8 significant bits)."""
+    return np.exp2(np.floor(np.log2(np.maximum(np.abs(v), 1e-30))) - 7)
+
+
 def y_check(Y_gpu: np.ndarray, Y_o: np.ndarray, rel: float = 1e-2, slack=0.0):
-    """max|dY| <= rel * rms(Y_o) + slack; an element above that must still be
-    within one bf16 ulp of Y_o plus slack (both sides round to bf16 at a tie
-    boundary).  `slack` (scalar or per element) is what the bf16 LR
-    intermediate may move Y by (see lr_slack)."""
+    """The layer's output bar, max|dY| <= rel * rms(Y_o), and what to report
+    about the elements over it: n_over counts them; n_bad counts those that
+    are also more than one bf16 ulp of Y_o (plus `slack`, scalar or per
+    element: what the bf16 LR intermediate may move Y by, see lr_slack)
+    away; `over` lists (row, col, Y_o, Y_gpu, |dY| / rms, |dY| / ulp) of up
+    to 8 of the worst."""
     rms = float(np.sqrt(np.mean(Y_o ** 2)))
     diff = np.abs(Y_gpu - Y_o)
-    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(Y_o), 1e-30))) - 7)
-    bad = (diff > rel * rms + slack) & (diff > ulp * (1 + 1e-9) + slack)
-    return dict(max_abs=float(diff.max()), rms=rms, max_rel_rms=float(diff.max() / rms),
-                n_over=int(np.sum(diff > rel * rms)), n_bad=int(bad.sum()))
+    ulp = bf16_ulp(Y_o)
+    over = diff > rel * rms
+    bad = over & (diff > ulp * (1 + 1e-9) + slack)
+    idx = np.argwhere(over)
+    worst = idx[np.argsort(-diff[over])][:8] if idx.size else idx
+    return dict(max_abs=float(diff.max()) if diff.size else 0.0, rms=rms,
+                max_rel_rms=float(diff.max() / rms) if diff.size and rms > 0 else 0.0,
+                n_over=int(over.sum()), n_bad=int(bad.sum()),
+                over=[(int(i), int(j), float(Y_o[i, j]), float(Y_gpu[i, j]), round(float(diff[i, j] / rms), 5),
+                       round(float(diff[i, j] / ulp[i, j]), 3)) for i, j in worst])
+
+
+# Workloads where the bar of the first paragraph cannot hold, named one by one.
+# Their outputs reach |Y| >= 2.56 rms(Y), where one bf16 ulp (2^-7 |Y|
+# rounded down to a power of two) is larger than 1e-2 rms(Y): an element whose
+# float32 (GPU) and float64 (oracle) sums fall on two sides of a bf16 rounding
+# boundary is then one ulp apart and over the bar although both results are
+# correctly rounded.  For these the bar is: every element over 1e-2 rms is at
+# most one bf16 ulp (plus the LR slack) from the oracle.
+ULP_EXCEPTIONS = {
+    "qkv_nvfp4_full", "qkv_int4_full", "mlp_fc1_full", "mlp_fc2_full", "lora_sweep_full",
+}
+
+
+def assert_y(Y_gpu, Y_o, rel=1e-2, slack=0.0, exception=None):
+    """max|dY| <= rel * rms(Y_o) on every element (n_over == 0), unless
+    `exception` names a workload of ULP_EXCEPTIONS: there, every element over
+    that bar must be within one bf16 ulp of Y_o plus `slack`."""
+    r = y_check(Y_gpu, Y_o, rel, slack)
+    if exception is None:
+        assert r["n_over"] == 0, r
+    else:
+        assert exception in ULP_EXCEPTIONS, exception
+        assert r["n_bad"] == 0, r
+    return r
 
 
 def lr_bound(X, L1f):
@@ -176,12 +214,6 @@ def lr_check(lr_gpu, X, L1f):
     err = np.abs(np.asarray(lr_gpu, np.float64) - lr_o)
     return dict(ok=bool(np.all(err <= bound)), n_beyond_ulp=int(np.sum(err > ulp * (1 + 1e-9))),
                 max_err_over_bound=float(np.max(err / bound)))
-
-
-def assert_y(Y_gpu, Y_o, rel=1e-2, slack=0.0):
-    r = y_check(Y_gpu, Y_o, rel, slack)
-    assert r["n_bad"] == 0, r
-    return r
 
 
 # ------------------------------------------------------------------ the layer on the GPU

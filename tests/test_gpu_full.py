@@ -3,8 +3,11 @@ benchmark times (the same entry points, grids and tile shapes).
 
 Codes, block scales and tensor scales are compared in full; LR in full (one
 bf16 ulp plus the float32 dot-product error bound); Y on 193 rows spread over
-M (the oracle computes those rows one by one in float64) within 1e-2 rms plus
-what the LR bound lets the up projection move.  Workloads:
+M (the oracle computes those rows one by one in float64).  Every workload here
+is named in svdq_harness.ULP_EXCEPTIONS: its outputs reach magnitudes where
+one bf16 ulp exceeds 1e-2 rms(Y), so an element over that bar must be one
+bf16 ulp from the oracle's (both sides round correctly, from float32 and
+float64 sums on either side of a rounding boundary).  Workloads:
   QKV      NVFP4, M=4608, K=3072, N=9216, rank 32
   MLP      NVFP4, fc1 3072 -> 12288 with GELU, fc2 12288 -> 3072 fed with the
            oracle's fc1 output (codes bit-exact); plus the all-GPU chain
@@ -36,8 +39,9 @@ def sample_rows(M, n=192):
     return np.unique(np.concatenate([np.linspace(0, M - 1, n).astype(np.int64), [M - 1]]))
 
 
-def check_layer(g, X, gelu=False, check_codes=True, rows=None):
-    """Codes of both sides, LR, and Y on sampled rows.  Returns (Y_gpu, stats)."""
+def check_layer(g, X, name, gelu=False, check_codes=True, rows=None):
+    """Codes of both sides, LR, and Y on sampled rows (Y against the bar of the
+    named exception, see svdq_harness.ULP_EXCEPTIONS).  Returns (Y_gpu, stats)."""
     pw, M = g.pw, X.shape[0]
     Xd = dev_bf16(X)
     if check_codes:
@@ -58,14 +62,14 @@ def check_layer(g, X, gelu=False, check_codes=True, rows=None):
     rows = sample_rows(M) if rows is None else rows
     Y_gpu = bf16_np(Yd[torch.from_numpy(rows).cuda()])
     Y_o = S.forward(pw, X[rows], gelu=gelu)["Y"]
-    return Yd, assert_y(Y_gpu, Y_o)
+    return Yd, assert_y(Y_gpu, Y_o, exception=name)
 
 
 def test_qkv_nvfp4_full(B):
     L = workloads.qkv()
     g = GpuLayer(L.fmt, L.X, L.W, L.bias, L.rank)
     try:
-        _, r = check_layer(g, L.X)
+        _, r = check_layer(g, L.X, "qkv_nvfp4_full")
         print("QKV nvfp4:", r)
     finally:
         g.close()
@@ -75,7 +79,7 @@ def test_qkv_int4_full(B):
     L = workloads.int4_qkv()
     g = GpuLayer(L.fmt, L.X, L.W, L.bias, L.rank)
     try:
-        _, r = check_layer(g, L.X)
+        _, r = check_layer(g, L.X, "qkv_int4_full")
         print("QKV int4:", r)
     finally:
         g.close()
@@ -85,13 +89,13 @@ def test_mlp_pair_full(B):
     fc1, (W2, b2, _) = workloads.mlp_pair()
     g1 = GpuLayer(fc1.fmt, fc1.X, fc1.W, fc1.bias, fc1.rank)
     try:
-        Y1d, r1 = check_layer(g1, fc1.X, gelu=True)
+        Y1d, r1 = check_layer(g1, fc1.X, "mlp_fc1_full", gelu=True)
         print("MLP fc1:", r1)
         # fc2's input for bit-exact codes: the oracle's own fc1 output
         Y1_o = S.forward(g1.pw, fc1.X, gelu=True)["Y"].astype(np.float32)
         g2 = GpuLayer("nvfp4", Y1_o, W2, b2, 32)
         try:
-            _, r2 = check_layer(g2, Y1_o)
+            _, r2 = check_layer(g2, Y1_o, "mlp_fc2_full")
             print("MLP fc2 (oracle input):", r2)
             # The all-GPU chain against the all-oracle chain.  fc1's outputs
             # differ by up to one bf16 ulp, which flips some of fc2's input codes
@@ -126,7 +130,7 @@ def test_lora_sweep_full(B):
             for M in workloads.LORA_SWEEP_M:
                 X = base.X[:M]
                 # codes and LR in full once per rank (at the largest M), Y at every M
-                _, res = check_layer(g, X, check_codes=(M == max(workloads.LORA_SWEEP_M)))
+                _, res = check_layer(g, X, "lora_sweep_full", check_codes=(M == max(workloads.LORA_SWEEP_M)))
                 print("LoRA r=%d M=%d:" % (r, M), res)
         finally:
             g.close()
