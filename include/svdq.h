@@ -343,13 +343,22 @@ svdq_status svdq_mlp(const svdq_weights* w1, const svdq_weights* w2, int M, cons
  * loads the library until the process exits).  It calls no cudaMalloc,
  * cudaFree or allocating library routine; the caller still passes X and Y.
  *   - Sizes: svdq_linear_workspace_bytes(w, M) must not exceed
- *     SVDQ_NOALLOC_SCRATCH_BYTES (32 MiB: at rank 32 about 1.9 KB per row
- *     for K = 3072, so M up to about 18,000, and about 4,700 rows for
- *     K = 12288); a larger request returns SVDQ_ERR_WORKSPACE before
- *     anything is launched.
+ *     SVDQ_NOALLOC_SCRATCH_BYTES (32 MiB).  Per row that is about
+ *     3 K_pad / 4 + 2 r_pad bytes for NVFP4 (codes K_pad / 2, scales in four
+ *     replicas K_pad / 4, LR 2 r_pad; r_pad = rank + LoRA rank rounded up to
+ *     64) and K_pad + K_pad / 16 + 2 r_pad bytes for INT4, with the scales
+ *     over M rounded up to 128 rows.  Largest M at r_pad = 64: NVFP4 13,784
+ *     rows at K = 3072 and 3,584 at K = 12288; INT4 9,886 at K = 3072 and
+ *     2,544 at K = 12288.  A larger request returns SVDQ_ERR_WORKSPACE
+ *     before anything is launched (after the argument and device checks,
+ *     in the order of svdq_linear).
  *   - The first call on each device looks up the scratch array's device
- *     address for that device (a runtime query, no allocation), so that
- *     first call should come before any stream capture.
+ *     address for that device (a runtime query, no allocation) and keeps it
+ *     for the life of the process, so that first call should come before
+ *     any stream capture.  A device reset (cudaDeviceReset, or anything that
+ *     destroys the primary context) invalidates this and every other piece
+ *     of per-device state the library keeps: do not call the library on a
+ *     device after resetting it.
  *   - All calls on a device share the one array and it keeps the previous
  *     call's contents; nothing in it needs clearing, because kernel 1
  *     rewrites every byte kernel 2 reads.  Calls whose kernels overlap on

@@ -202,6 +202,18 @@ svdq_status check_handle_device(const svdq_weights* w, DevState** d) {
   return dev == w->dev ? SVDQ_OK : SVDQ_ERR_INVALID_ARG;
 }
 
+}  // namespace
+
+// For entry points compiled in other files: the current device's check
+// (compute capability 10.0, or the debug override) and that the handle lives
+// on it.
+svdq_status svdq::handle_device_status(const svdq_weights* w) {
+  DevState* d = nullptr;
+  return check_handle_device(w, &d);
+}
+
+namespace {
+
 // Per-call NVFP4 activation tensor scale: where the amax slots are and where
 // kernel 1 reports the scale it chose.
 struct DynScale {

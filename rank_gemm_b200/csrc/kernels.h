@@ -8,6 +8,7 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "svdq.h"
 
 namespace svdq {
 
@@ -16,6 +17,10 @@ namespace svdq {
 // needed (the call costs microseconds of host time, more than a small
 // kernel's launch).
 cudaError_t ensure_dynamic_smem(const void* kernel, size_t bytes);
+
+// SVDQ_OK when the current device is supported (compute capability 10.0)
+// and holds the handle `w`; the status any entry point would return otherwise.
+svdq_status handle_device_status(const svdq_weights* w);
 
 // ---------------------------------------------------------------- kernel 1
 struct K1Params {

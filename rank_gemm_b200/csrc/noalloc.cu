@@ -7,6 +7,7 @@
 
 #include <mutex>
 
+#include "kernels.h"
 #include "svdq.h"
 
 namespace {
@@ -25,19 +26,19 @@ void* g_scratch_addr[MAX_DEVICES];   // device address of g_linear_scratch, per 
 
 extern "C" svdq_status svdq_linear_noalloc(const svdq_weights* w, int M, const void* X, svdq_epilogue epi,
                                            void* Y, cudaStream_t stream) {
+  // the checks of svdq_linear, in its order, before the size test
   if (!w || (M > 0 && (!X || !Y))) return SVDQ_ERR_INVALID_ARG;
+  if (epi != SVDQ_EPI_NONE && epi != SVDQ_EPI_GELU_TANH) return SVDQ_ERR_INVALID_ARG;
   if (M < 0) return SVDQ_ERR_SHAPE;
+  svdq_status s = svdq::handle_device_status(w);   // compute capability 10.0 and the handle's device
+  if (s != SVDQ_OK) return s;
   if (svdq_linear_workspace_bytes(w, M) > SVDQ_NOALLOC_SCRATCH_BYTES) return SVDQ_ERR_WORKSPACE;
 
-  int dev = -1, major = 0, minor = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES ||
-      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) {
     cudaGetLastError();
     return SVDQ_ERR_UNSUPPORTED_DEVICE;
   }
-  if (major != 10 || minor != 0) return SVDQ_ERR_UNSUPPORTED_DEVICE;
-
   void* scratch = nullptr;
   {
     // Set-up, once per device, with that device current: look up where the
