@@ -42,7 +42,7 @@ sys.path.insert(0, ROOT)
 WORKLOAD = dict(name="nvfp4_qkv_M4608_K3072_N9216_r32", fmt="nvfp4", M=4608, K=3072, N=9216, rank=32)
 # --workload: the QKV projection is the bench line; the others are the
 # remaining parity configurations, timed the same way for their profiles.
-WORKLOADS = ("qkv", "int4_qkv", "mlp_fc1", "mlp_fc2", "lora", "awq_adaln", "mlp_pair")
+WORKLOADS = ("qkv", "int4_qkv", "mlp_fc1", "mlp_fc2", "lora", "awq_adaln", "mlp_pair", "small", "lora_sweep")
 INT8_PER_BF16 = 2.0         # nominal dense INT8 : BF16 tensor throughput (4.5 : 2.25)
 METRIC = "SVDQuant W4A4 linear effective TFLOPS & % of FP4 tensor peak; µs/layer"
 UNIT = "TFLOP/s"
@@ -661,6 +661,144 @@ def run_mlp_pair(args, world, rank, local):
         print(json.dumps(out), flush=True)
 
 
+# ------------------------------------------------------------------ small shapes: config 0 and the LoRA sweep
+def layer_bytes(M, K, N, r_tot, fmt):
+    """Algorithmic HBM bytes of one whole layer call: X, 1/lambda, the
+    factors, the residual codes and scales (once), bias and Y.  The
+    intermediates qX, sX and LR pass between the two kernels through L2."""
+    g, sb = (16, 1) if fmt == "nvfp4" else (64, 2)
+    r_pad = -(-r_tot // 64) * 64
+    return (M * K * 2 + K * 4 + r_tot * K * 2 + N * K // 2 + N * (K // g) * sb + N * r_pad * 2 + N * 4
+            + M * N * 2)
+
+
+def run_points(args, world, rank, local, which):
+    """Per-point timing for shapes whose working set is smaller than L2: the
+    small NVFP4 layer (M=128, K=N=1024, rank 32) or the LoRA sweep (K = N =
+    3072, M in {256, 1024, 4096, 16384}, rank in {16, 32, 64, 128}, each with
+    a rank-16 LoRA).  Every timed call is preceded by an untimed write of a
+    buffer twice the L2 size, so weights and activations come from HBM as
+    they do when a model runs the layer once per block; a call is timed with
+    CUDA events on its stream.  Per point: the layer (kernel 1 + kernel 2),
+    kernel 2 alone (after an untimed kernel 1), the plain W4A4 path
+    (quantize + GEMM without the low-rank branch) and their ratio."""
+    import numpy as np
+    import torch
+    import workloads
+    from rank_gemm_b200 import build as _b
+    if rank == 0:
+        _b.build()
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", init_method="env://", world_size=world, rank=rank,
+                                timeout=__import__("datetime").timedelta(seconds=120))
+        dist.barrier()
+    from rank_gemm_b200 import binding as B
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    peaks = measured_peaks()
+    tc_peak = peaks["bf16"] * FP4_PER_BF16
+
+    def dev_bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16).to(dev)
+
+    def timed(fn, pre=None, n=100):
+        """Median over n calls of fn's device time, L2 flushed before each."""
+        for _ in range(3):
+            flush.zero_()
+            if pre:
+                pre()
+            fn()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        torch.cuda.synchronize()
+        for a, b in evs:
+            flush.zero_()
+            if pre:
+                pre()
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in evs) * 1e3
+
+    if which == "small":
+        L = workloads.small()
+        X_all = dev_bf16(L.X)
+        Wt = dev_bf16(L.W.T)
+        lam, act, L1f, L2 = gpu_factors(B, Wt, X_all, L.rank, torch)
+        specs = [(L.rank, 0, B.svdq_prepare_weights("nvfp4", L.K, L.N, L.rank, Wt, lam, L1f, L2, dev_bf16(L.bias),
+                                                    act_scale=act), [L.M])]
+        K, N, name = L.K, L.N, L.name
+    else:
+        base = workloads.lora_sweep_base()
+        X_all = dev_bf16(base.X)
+        Wt = dev_bf16(base.W.T)
+        rmax = max(workloads.LORA_SWEEP_R)
+        lam, act, L1f, L2 = gpu_factors(B, Wt, X_all, rmax, torch)   # one split; smaller ranks take its prefix
+        la, lb = dev_bf16(base.lora_A), dev_bf16(base.lora_B)
+        lora = base.lora_A.shape[1]
+        specs = []
+        for r in workloads.LORA_SWEEP_R:
+            h = B.svdq_prepare_weights("nvfp4", base.K, base.N, r, Wt, lam, L1f[:, :r].contiguous(),
+                                       L2[:r].contiguous(), dev_bf16(base.bias), la, lb, lora, act)
+            specs.append((r, lora, h, list(workloads.LORA_SWEEP_M)))
+        K, N, name = base.K, base.N, "nvfp4_lora_sweep_K3072_N3072_lora%d" % lora
+    n = max(10, min(args.steps, 200))
+    points = []
+    tot_flops = tot_us = 0.0
+    with ClockSampler(local) as clocks:
+        for r, lora, h, Ms in specs:
+            for M in Ms:
+                X = X_all[:M]
+                Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+                qb, sb, lb = B.svdq_act_buffer_sizes(h, M)
+                qX, sX, LR = (torch.empty(v, dtype=torch.uint8, device=dev) for v in (qb, sb, lb))
+                k1 = lambda: B.svdq_quantize_act_lowrank_down(h, M, X, qX, sX, LR, stream)
+                k2 = lambda: B.svdq_w4a4_gemm_lowrank_up(h, M, qX, sX, LR, B.SVDQ_EPI_NONE, Y, stream)
+                t_layer = timed(lambda: (k1(), k2()), n=n)
+                t_k2 = timed(k2, pre=k1, n=n)
+                t_plain = timed(lambda: (B.svdq_quantize_act(h, M, X, qX, sX, stream),
+                                         B.svdq_w4a4_gemm(h, M, qX, sX, Y, stream)), n=n)
+                flops = 2.0 * M * N * K
+                nbytes = layer_bytes(M, K, N, r + lora, "nvfp4")
+                t_roof = max(flops / (tc_peak * 1e12), nbytes / (peaks["hbm"] * 1e9)) * 1e6
+                points.append({"M": M, "rank": r, "lora_rank": lora, "us_per_layer": round(t_layer, 2),
+                               "tflops": round(flops / (t_layer * 1e-6) / 1e12, 2),
+                               "bound": "tensor" if flops / (tc_peak * 1e12) > nbytes / (peaks["hbm"] * 1e9)
+                               else "hbm",
+                               "roofline_us": round(t_roof, 2), "roofline_frac": round(t_roof / t_layer, 4),
+                               "kernel2_us": round(t_k2, 2), "plain_w4a4_us": round(t_plain, 2),
+                               "fused_over_plain": round(t_layer / t_plain - 1, 4)})
+                tot_flops += flops
+                tot_us += t_layer
+    status = B.svdq_poll_device_error(stream)
+    for _, _, h, _ in specs:
+        B.svdq_free_weights(h)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        one = points[0] if which == "small" else None
+        out = {"metric": METRIC, "value": round(tot_flops * world / (tot_us * 1e-6) / 1e12, 3), "unit": UNIT,
+               "n_gpus": world, "steps": n, "warmup": 3, "higher_is_better": True, "scaling": "weak",
+               "vs_baseline": None, "dtype": "nvfp4",
+               "data": "synthetic (seeded, outlier channels x20 / x5), random-init weights",
+               "config": {"workload": name, "K": K, "N": N, "format": "nvfp4", "group": 16,
+                          "parallelism": "replicas x%d (each rank its own batch)" % world,
+                          "l2": "a %d MB buffer written before every timed call (2 x L2)" % (2 * l2 // 2 ** 20),
+                          "timing": "median of %d calls per point, CUDA events around each" % n},
+               "points": points, "device_status": status, "clocks": clocks.summary(),
+               "gpu_launches": 2 * n * len(points)}
+        if one:
+            out["us_per_layer"] = one["us_per_layer"]
+            out["roofline"] = {"bound": one["bound"], "achieved": one["tflops"], "unit": "TFLOP/s",
+                               "frac": one["roofline_frac"], "roofline_us": one["roofline_us"]}
+        print(json.dumps(out), flush=True)
+
+
 # ------------------------------------------------------------------ AWQ W4A16 arm
 AWQ_METRIC = "AWQ W4A16 linear effective TFLOPS & % of HBM bandwidth; µs/layer"
 
@@ -817,6 +955,8 @@ def main():
         run_awq(args, world, rank, local)
     elif args.workload == "mlp_pair":
         run_mlp_pair(args, world, rank, local)
+    elif args.workload in ("small", "lora_sweep"):
+        run_points(args, world, rank, local, args.workload)
     else:
         run_ours(args, world, rank, local)
 
