@@ -28,6 +28,10 @@ Readings where the pages are silent (each one is a choice of this build):
     half to even, divisions are IEEE float32.
   * Dequantized weight: w^ = (code - zero) d, exact in float32.
   * Y = X' W^ + b in float64, rounded once to bf16.
+  * The tensor-core form (large batches, forward_16bit): the product runs
+    on 16-bit operands, as W4A16 GEMMs do; X'16 = bf16(X') (X itself when
+    s = 1) and w^16 = bf16((code - zero) d) (one rounding of the exact
+    product); Y = bf16(X'16 W^16 + b), float64 in between.
 """
 from __future__ import annotations
 
@@ -110,6 +114,18 @@ def dequantize(aw: AwqWeights) -> np.ndarray:
 def scaled_activation(aw: AwqWeights, X) -> np.ndarray:
     """X' = fl32(x * fl32(1/s_k))."""
     return (np.asarray(X, np.float32) * aw.inv_s[None, :]).astype(np.float32)
+
+
+def dequantize_16bit(aw: AwqWeights) -> np.ndarray:
+    """W^16 (K, N) float64 holding bf16 values: (code - zero) d rounded once."""
+    return F.bf16_round(dequantize(aw))
+
+
+def forward_16bit(aw: AwqWeights, X) -> dict:
+    """The tensor-core form: Y = bf16(bf16(X') W^16 + b), float64 in between."""
+    Xp16 = F.bf16_round(scaled_activation(aw, X).astype(np.float64))
+    y = Xp16 @ dequantize_16bit(aw) + aw.bias[None, :]
+    return dict(Xp16=Xp16, W16=dequantize_16bit(aw), Y=F.bf16_round(y))
 
 
 def forward(aw: AwqWeights, X) -> dict:

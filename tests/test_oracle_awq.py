@@ -115,3 +115,86 @@ def test_forward_against_exact_rationals():
                 wq = (int(aw.code[k, n]) - int(aw.zero[0, n])) * Fraction(float(aw.scale[0, n]))
                 acc += Fraction(float(X[m, k])) * wq
             assert Y[m, n] == F.bf16_round(float(acc)), (m, n)
+
+
+# ------------------------------------------------------------ the 16-bit-operand (tensor-core) form
+def _bf16_of_exact(q: Fraction) -> float:
+    """The bf16 value nearest to an exact rational (ties to the even
+    significand): the two multiples of the binade's step around it."""
+    import math
+    if q == 0:
+        return 0.0
+    a = abs(q)
+    e = math.floor(math.log2(float(a)))
+    while Fraction(2) ** e > a:          # the exact binade: 2^e <= |q| < 2^(e+1)
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    step = Fraction(2) ** (max(e, -126) - 7)
+    lo = (a / step).__floor__()
+    d_lo, d_hi = a - lo * step, (lo + 1) * step - a
+    c = lo if (d_lo < d_hi or (d_lo == d_hi and lo % 2 == 0)) else lo + 1
+    return math.copysign(float(c * step), float(q))
+
+
+def check_forward_16bit_against_exact_rationals(s_kind="none"):
+    """forward_16bit by the definition written out: every dequantized weight
+    and every scaled activation rounded once to bf16 from its exact value,
+    the sum in exact rationals, the output rounded once."""
+    W = _rand((2 * A.GROUP, 3), 21, 0.05)
+    X = _rand((2, 2 * A.GROUP), 22, 1.0)
+    b = _rand((3,), 23, 0.01)
+    s = None if s_kind == "none" else np.exp(np.random.default_rng(24).uniform(-1, 1, 2 * A.GROUP)).astype(np.float32)
+    aw = A.prepare(W, b, s=s)
+    Y = A.forward_16bit(aw, X)["Y"]
+    inv_s = [np.float32(1.0) / np.float32(v) for v in (s if s is not None else np.ones(2 * A.GROUP, np.float32))]
+    for m in range(2):
+        for n in range(3):
+            acc = Fraction(float(b[n]))
+            for k in range(2 * A.GROUP):
+                g = k // A.GROUP
+                w16 = _bf16_of_exact((int(aw.code[k, n]) - int(aw.zero[g, n])) * Fraction(float(aw.scale[g, n])))
+                x16 = _bf16_of_exact(Fraction(float(np.float32(np.float32(X[m, k]) * inv_s[k]))))
+                acc += Fraction(x16) * Fraction(w16)
+            assert Y[m, n] == _bf16_of_exact(acc), (m, n)
+
+
+def test_forward_16bit_against_exact_rationals():
+    check_forward_16bit_against_exact_rationals("none")
+
+
+def test_forward_16bit_with_awq_scale_against_exact_rationals():
+    check_forward_16bit_against_exact_rationals("random")
+
+
+def test_forward_16bit_is_forward_when_the_weights_fit_16_bits():
+    """With scales that are powers of two, (code - zero) d has at most 4
+    significant bits, and with s = 1 X' is X: the two forms then compute the
+    same exact sum and give identical outputs."""
+    d0 = 2.0 ** -7
+    rng = np.random.default_rng(25)
+    # every group spans exactly 15 steps (lo = -7 d0, hi = 8 d0), values on the grid
+    W = (rng.integers(-7, 9, (3 * A.GROUP, 5)) * d0).astype(np.float32)
+    W[0::A.GROUP] = -7 * d0
+    W[1::A.GROUP] = 8 * d0
+    X = _rand((6, 3 * A.GROUP), 26, 1.0)
+    b = _rand((5,), 27, 0.01)
+    aw = A.prepare(W, b)
+    assert np.all(aw.scale == np.float32(d0))
+    assert np.array_equal(A.dequantize_16bit(aw), A.dequantize(aw))
+    assert np.array_equal(A.forward_16bit(aw, X)["Y"], A.forward(aw, X)["Y"])
+
+
+def test_forward_16bit_stays_within_the_weight_rounding_of_forward():
+    """|Y16 - Y| <= sum_k |x'_k| |w^16 - w^| + the activations' bf16 rounding
+    + one bf16 ulp of each output: the 16-bit form only adds the roundings it
+    names."""
+    W = _rand((4 * A.GROUP, 40), 28)
+    X = _rand((8, 4 * A.GROUP), 29, 1.0)
+    aw = A.prepare(W, np.zeros(40))
+    o, o16 = A.forward(aw, X), A.forward_16bit(aw, X)
+    dw = np.abs(o16["W16"] - A.dequantize(aw))
+    bound = np.abs(o["Xp"]) @ dw + np.abs(o16["Xp16"] - o["Xp"]) @ np.abs(o16["W16"])
+    ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(o["Y"]), 1e-30))) - 7)
+    assert np.all(np.abs(o16["Y"] - o["Y"]) <= bound + 2 * ulp + 1e-12)
+    assert np.any(dw > 0)        # the case does exercise the rounding

@@ -136,3 +136,26 @@ def test_mutation_dynamic_scale_exponent_rounded_down(monkeypatch):
         return np.float32(np.float32(np.ldexp(1.0, j)) / np.float32(pw.s_tR)), j
     monkeypatch.setattr(S, "dynamic_act_scale", bad)
     assert _fails(TQ.test_dynamic_scale_pairs_to_a_power_of_two_and_covers_the_batch)
+
+
+def test_mutation_awq_16bit_weights_not_rounded(monkeypatch):
+    monkeypatch.setattr(A, "dequantize_16bit", lambda aw: A.dequantize(aw))
+    assert _fails(TA.check_forward_16bit_against_exact_rationals, "none")
+
+
+def test_mutation_awq_16bit_scale_rounded_before_the_product(monkeypatch):
+    def bad(aw):
+        z = np.repeat(aw.zero.astype(np.float64), A.GROUP, axis=0)
+        d = np.repeat(F.bf16_round(aw.scale.astype(np.float64)), A.GROUP, axis=0)
+        return F.bf16_round((aw.code.astype(np.float64) - z) * d)
+    monkeypatch.setattr(A, "dequantize_16bit", bad)
+    assert _fails(TA.check_forward_16bit_against_exact_rationals, "none")
+
+
+def test_mutation_awq_16bit_activation_scale_dropped(monkeypatch):
+    def bad(aw, X):
+        Xp16 = F.bf16_round(np.asarray(X, np.float64))
+        y = Xp16 @ A.dequantize_16bit(aw) + aw.bias[None, :]
+        return dict(Xp16=Xp16, W16=A.dequantize_16bit(aw), Y=F.bf16_round(y))
+    monkeypatch.setattr(A, "forward_16bit", bad)
+    assert _fails(TA.check_forward_16bit_against_exact_rationals, "random")
