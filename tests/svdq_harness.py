@@ -166,7 +166,8 @@ def y_check(Y_gpu: np.ndarray, Y_o: np.ndarray, rel: float = 1e-2, slack=0.0):
 # correctly rounded.  For these the bar is: every element over 1e-2 rms is at
 # most one bf16 ulp (plus the LR slack) from the oracle.
 ULP_EXCEPTIONS = {
-    "qkv_nvfp4_full", "qkv_int4_full", "mlp_fc1_full", "mlp_fc2_full", "lora_sweep_full",
+    "qkv_nvfp4_full", "qkv_int4_full", "mlp_fc1_full", "mlp_fc2_full", "lora_sweep_full", "awq_qkv_full",
+    "dynamic_qkv_full",
 }
 
 
