@@ -42,7 +42,7 @@ sys.path.insert(0, ROOT)
 WORKLOAD = dict(name="nvfp4_qkv_M4608_K3072_N9216_r32", fmt="nvfp4", M=4608, K=3072, N=9216, rank=32)
 # --workload: the QKV projection is the bench line; the others are the
 # remaining parity configurations, timed the same way for their profiles.
-WORKLOADS = ("qkv", "int4_qkv", "mlp_fc1", "mlp_fc2", "lora", "awq_adaln", "mlp_pair", "small", "lora_sweep")
+WORKLOADS = ("qkv", "int4_qkv", "mlp_fc1", "mlp_fc2", "lora", "awq_adaln", "mlp_pair", "small", "lora_sweep", "awq_qkv")
 INT8_PER_BF16 = 2.0         # nominal dense INT8 : BF16 tensor throughput (4.5 : 2.25)
 METRIC = "SVDQuant W4A4 linear effective TFLOPS & % of FP4 tensor peak; µs/layer"
 UNIT = "TFLOP/s"
@@ -461,24 +461,21 @@ def run_ours(args, world, rank, local):
                                                   stream), n_ov) if nv else None
     del wss
 
-    # end to end through the public call with host buffers
+    # end to end through the public call with host buffers: svdq_linear_host
+    # moves X in and Y out (page-locked host memory) in row slabs overlapped
+    # with the kernels; the events on the caller's stream cover every copy
     e2e_steps = min(K_steps, 50)
     Xh = torch.empty(M, K, dtype=torch.bfloat16, pin_memory=True)
     Xh.copy_(X0.cpu())
     Yh = torch.empty(M, N, dtype=torch.bfloat16, pin_memory=True)
-    ws = torch.empty(B.svdq_linear_workspace_bytes(h, M), dtype=torch.uint8, device=dev)
-    Xd, Yd = Xs[0], Ys[0]
+    ws = torch.empty(B.svdq_linear_host_workspace_bytes(h, M), dtype=torch.uint8, device=dev)
     for _ in range(3):
-        Xd.copy_(Xh, non_blocking=True)
-        B.svdq_linear(h, M, Xd, epi, Yd, ws, None, stream)
-        Yh.copy_(Yd, non_blocking=True)
+        B.svdq_linear_host(h, M, Xh, epi, Yh, ws, None, stream)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        Xd.copy_(Xh, non_blocking=True)
-        B.svdq_linear(h, M, Xd, epi, Yd, ws, None, stream)
-        Yh.copy_(Yd, non_blocking=True)
+        B.svdq_linear_host(h, M, Xh, epi, Yh, ws, None, stream)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / e2e_steps
@@ -507,7 +504,8 @@ def run_ours(args, world, rank, local):
                                "unit": "GB/s", "frac": round(bytes_k1 / (k1_ms * 1e-3) / 1e9 / peaks["hbm"], 4),
                                "traffic": traffic_k1, "algorithmic_bytes": bytes_k1, "us": round(k1_ms * 1e3, 2)},
                "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": M * K * 2,
-                       "d2h_bytes_per_step": M * N * 2, "ms_per_step": round(e2e_ms, 4)},
+                       "d2h_bytes_per_step": M * N * 2, "ms_per_step": round(e2e_ms, 4),
+                       "call": "svdq_linear_host (page-locked X and Y, copies overlapped with the kernels)"},
                "lowrank_overhead": {"plain_w4a4_us": round(t_plain * 1e3, 2), "fused_us": round(t_fused * 1e3, 2),
                                     "unfused_us": round(t_unfused * 1e3, 2),
                                     "fused_over_plain": round(t_fused / t_plain - 1, 4),
@@ -677,8 +675,9 @@ def run_points(args, world, rank, local, which):
     small NVFP4 layer (M=128, K=N=1024, rank 32) or the LoRA sweep (K = N =
     3072, M in {256, 1024, 4096, 16384}, rank in {16, 32, 64, 128}, each with
     a rank-16 LoRA).  Every timed call is preceded by an untimed write of a
-    buffer twice the L2 size, so weights and activations come from HBM as
-    they do when a model runs the layer once per block; a call is timed with
+    buffer twice the L2 size and a read of another one, so weights and
+    activations come from HBM as they do when a model runs the layer once per
+    block, and the L2 holds no dirty lines to write back; a call is timed with
     CUDA events on its stream.  Per point: the layer (kernel 1 + kernel 2),
     kernel 2 alone (after an untimed kernel 1), the plain W4A4 path
     (quantize + GEMM without the low-rank branch) and their ratio."""
@@ -699,6 +698,16 @@ def run_points(args, world, rank, local, which):
     stream = torch.cuda.current_stream(dev)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    evict = torch.ones(2 * l2 // 4, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def flush_l2():
+        # write twice the L2 size, then read another buffer of that size, so
+        # the timed call starts with a cold L2 that holds no dirty lines (a
+        # write alone would leave the L2 full of dirty lines whose write-back
+        # the timed call would pay for)
+        flush.zero_()
+        torch.sum(evict, dim=0, out=sink)
     peaks = measured_peaks()
     tc_peak = peaks["bf16"] * FP4_PER_BF16
 
@@ -708,14 +717,14 @@ def run_points(args, world, rank, local, which):
     def timed(fn, pre=None, n=100):
         """Median over n calls of fn's device time, L2 flushed before each."""
         for _ in range(3):
-            flush.zero_()
+            flush_l2()
             if pre:
                 pre()
             fn()
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
         torch.cuda.synchronize()
         for a, b in evs:
-            flush.zero_()
+            flush_l2()
             if pre:
                 pre()
             a.record(stream)
@@ -788,7 +797,8 @@ def run_points(args, world, rank, local, which):
                "data": "synthetic (seeded, outlier channels x20 / x5), random-init weights",
                "config": {"workload": name, "K": K, "N": N, "format": "nvfp4", "group": 16,
                           "parallelism": "replicas x%d (each rank its own batch)" % world,
-                          "l2": "a %d MB buffer written before every timed call (2 x L2)" % (2 * l2 // 2 ** 20),
+                          "l2": "before every timed call a %d MB buffer is written and another read (2 x L2 each): "
+                                "cold L2, no dirty lines" % (2 * l2 // 2 ** 20),
                           "timing": "median of %d calls per point, CUDA events around each" % n},
                "points": points, "device_status": status, "clocks": clocks.summary(),
                "gpu_launches": 2 * n * len(points)}
@@ -937,6 +947,100 @@ def run_awq(args, world, rank, local):
         print(json.dumps(out), flush=True)
 
 
+def run_awq_qkv(args, world, rank, local):
+    """The W4A16 side of the "SVDQuant" abstract's comparison on the QKV shape
+    (M=4608, K=3072, N=9216): the same activation, weight and bias as the
+    NVFP4 QKV line, quantized as an AWQ W4A16 layer (int4, group 64) and run
+    by svdq_awq_gemm (16-bit operands on the tensor core); the NVFP4 W4A4
+    layer (svdq_linear) is timed the same way in the same process, and the
+    line reports their ratio."""
+    import numpy as np
+    import torch
+    import workloads
+    from rank_gemm_b200 import build as _b
+    if rank == 0:
+        _b.build()
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", init_method="env://", world_size=world, rank=rank,
+                                timeout=__import__("datetime").timedelta(seconds=120))
+        dist.barrier()
+    from rank_gemm_b200 import binding as B
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    L = workloads.awq_qkv()
+    M, K, N = L.M, L.K, L.N
+    Wt = torch.from_numpy(np.ascontiguousarray(L.W.T)).to(torch.bfloat16).to(dev)
+    bias = torch.from_numpy(L.bias).to(torch.bfloat16).to(dev)
+    ha = B.svdq_awq_prepare(K, N, Wt, None, bias)
+    lay = build_layer("qkv", B, torch, dev)
+    sets = 3
+    X0 = lay["X0"]
+    Xs = [X0] + [X0.clone() for _ in range(sets - 1)]
+    Ys = [torch.empty(M, N, dtype=torch.bfloat16, device=dev) for _ in range(sets)]
+    wss = [torch.empty(B.svdq_linear_workspace_bytes(lay["h"], M), dtype=torch.uint8, device=dev)
+           for _ in range(sets)]
+    awq = lambda i: B.svdq_awq_gemm(ha, M, Xs[i % sets], Ys[i % sets], stream)
+    w4a4 = lambda i: B.svdq_linear(lay["h"], M, Xs[i % sets], B.SVDQ_EPI_NONE, Ys[i % sets], wss[i % sets], None,
+                                   stream)
+    for i in range(args.warmup):
+        awq(i)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t0.record(stream)
+        for i in range(args.steps):
+            awq(i)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    max_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+    status = B.svdq_poll_device_error(stream)
+    n_cmp = min(args.steps, 300)
+    for i in range(3):
+        w4a4(i)
+    torch.cuda.synchronize()
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(stream)
+    for i in range(n_cmp):
+        w4a4(i)
+    c1.record(stream)
+    torch.cuda.synchronize()
+    w4a4_us = max_over_ranks(c0.elapsed_time(c1), world, dev) / n_cmp * 1e3
+    us = max_ms / args.steps * 1e3
+    flops = 2.0 * M * N * K
+    value = weak_scaling_value(flops, args.steps, world, max_ms)
+    peaks = measured_peaks()
+    out = None
+    if rank == 0:
+        out = {"metric": "AWQ W4A16 linear effective TFLOPS & % of BF16 tensor peak; µs/layer",
+               "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+               "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 5), "us_per_layer": round(us, 2),
+               "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 x int4 -> f32",
+               "data": "synthetic (the QKV workload's seeded X, W and bias), random-init weights",
+               "config": {"workload": L.name, "M": M, "K": K, "N": N, "group": 64, "awq_scale": "none",
+                          "parallelism": "replicas x%d (each rank its own batch)" % world,
+                          "l2": "3 rotating X/Y sets (%.0f MB) > 126 MB L2" % (sets * (M * K * 2 + M * N * 2) / 1e6)},
+               "roofline": {"kernel": "awq_gemm", "bound": "tensor", "achieved": round(flops / (us * 1e-6) / 1e12, 2),
+                            "peak": peaks["bf16"], "unit": "TFLOP/s",
+                            "frac": round(flops / (us * 1e-6) / 1e12 / peaks["bf16"], 4), "traffic": None,
+                            "peak_source": "%s bf16 (the product runs on bf16 operands)" % peaks["source"]},
+               "w4a4_nvfp4_us": round(w4a4_us, 2), "w4a4_over_w4a16_speedup": round(us / w4a4_us, 3),
+               "gpu_launches": args.steps, "device_status": status, "clocks": clocks.summary()}
+    B.svdq_awq_free(ha)
+    B.svdq_free_weights(lay["h"])
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -955,6 +1059,8 @@ def main():
         run_awq(args, world, rank, local)
     elif args.workload == "mlp_pair":
         run_mlp_pair(args, world, rank, local)
+    elif args.workload == "awq_qkv":
+        run_awq_qkv(args, world, rank, local)
     elif args.workload in ("small", "lora_sweep"):
         run_points(args, world, rank, local, args.workload)
     else:

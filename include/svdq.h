@@ -308,9 +308,11 @@ svdq_status svdq_linear_dynamic(const svdq_weights* w, int M, const void* X, svd
  *   Y1, ...) would write: qX2 and sX2 (the NVFP4 codes and replicated scales
  *   of Y1 diag(lambda2)^-1 with w2's static activation tensor scale),
  *   identical to kernel 1's given the same Y1; and LR2 = bf16(Y1 L1f2) from
- *   per-tile float32 partials added in a fixed order (the same on every run;
- *   float32 summation order differs from kernel 1's, within the LR bound).
- *   Requires both handles NVFP4, w2's K == w1's N and r_tot of w2 <= 32.
+ *   float32 partials, one per 256-column tile of Y1 (computed on the tensor
+ *   core from the tile's bf16 values held in tensor memory), added in a
+ *   fixed order (the same on every run; float32 summation order differs from
+ *   kernel 1's, within the LR bound).
+ *   Requires both handles NVFP4, w2's K == w1's N and r_tot of w2 <= 64.
  *   qX2, sX2, LR2  dev, sizes from svdq_act_buffer_sizes(w2, M); qX2 32-byte
  *                  aligned (each row's codes of a 64-column block go out as
  *                  one 32-byte store)
@@ -328,6 +330,34 @@ svdq_status svdq_linear_emit_next(const svdq_weights* w1, const svdq_weights* w2
 size_t svdq_mlp_workspace_bytes(const svdq_weights* w1, const svdq_weights* w2, int M);
 svdq_status svdq_mlp(const svdq_weights* w1, const svdq_weights* w2, int M, const void* X, svdq_epilogue epi1,
                      svdq_epilogue epi2, void* Y, void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * The whole layer from host memory to host memory, with the copies
+ * overlapped with the kernels (no counterpart in the paper: an integration
+ * convenience for callers whose activations live on the host).  M is cut
+ * into slabs of about M / 8 rows (a multiple of 128, at least 128); while the
+ * layer runs on slab i on `stream`, the library's own copy-in stream moves
+ * slab i + 1's X to the device and its copy-out stream moves slab i - 1's Y
+ * to the host (the two directions use separate copy engines).  Each slab is
+ * one cudaMemcpyAsync per direction.  Row m of Y depends on row m of X only,
+ * so the result is bit-identical to svdq_linear on the whole batch.
+ *   X_host  host bf16 [M][K], Y_host host bf16 [M][N]; page-locked memory
+ *           (cudaHostAlloc / cudaHostRegister) is needed for the copies to
+ *           run asynchronously and overlap
+ *   workspace  dev, 256-byte aligned, at least
+ *           svdq_linear_host_workspace_bytes(w, M) bytes (two X slabs, two
+ *           Y slabs and one slab's svdq_linear workspace)
+ * Ordering: the call's work starts after the work already on `stream`; work
+ * issued on `stream` afterwards starts after the last Y slab is on the host.
+ * The two copy streams and their events are created at a device's first call
+ * (no device memory is allocated) and are shared by every call on that device:
+ * calls from several host threads are serialised by a lock while they are
+ * issued.
+ * Errors: as svdq_linear.
+ * ------------------------------------------------------------------------ */
+size_t svdq_linear_host_workspace_bytes(const svdq_weights* w, int M);
+svdq_status svdq_linear_host(const svdq_weights* w, int M, const void* X_host, svdq_epilogue epi, void* Y_host,
+                             void* workspace, size_t ws_bytes, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
  * svdq_linear without a workspace argument (no counterpart in the paper: it
@@ -427,7 +457,10 @@ svdq_status svdq_linear_unfused(const svdq_weights* w, int M, const void* X, svd
  * svdq_awq_view layouts (N_pad = N rounded up to 32; pad features hold
  *   code 0, zero 0, scale 0):
  *   code   uint8 [K/32][N_pad][16]: 16 bytes per (32-feature chunk c, n), the
- *          codes of k = 32c .. 32c + 31, two per byte, even k in the low nibble
+ *          codes of k = 32c .. 32c + 31, 4 bits each; the 32-bit word w
+ *          (little-endian) holds k = 32c + 8w + i at bits 4p .. 4p + 3 with
+ *          p = i / 2 + 4 (i % 2) (even k in the low half-word, odd k in the
+ *          high half-word, each in increasing order)
  *   scale  binary16 [K/64][N_pad];  zero  uint8 [K/64][N_pad]
  *   inv_s  float32 [K] = fl32(1/s);  bias  float32 [N_pad]
  * ------------------------------------------------------------------------ */
@@ -445,6 +478,25 @@ svdq_status svdq_awq_prepare(int K, int N, const void* W_t, const float* s, cons
 svdq_status svdq_awq_free(svdq_awq_weights* w);
 svdq_status svdq_awq_view(const svdq_awq_weights* w, svdq_awq_info* info);
 svdq_status svdq_awq_linear(const svdq_awq_weights* w, int M, const void* X, void* Y, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * The same W4A16 layer on the tensor core, for batches where it is a dense
+ * contraction (the W4A16 side of the "SVDQuant" abstract's speed comparison,
+ * 3.0x / 3.1x for W4A4 over W4A16 on the pages' GPUs).  The product runs on
+ * 16-bit operands as W4A16 GEMMs do: each dequantized weight is rounded once
+ * to bf16, w^16 = bf16((code - zero) d), and the activation is
+ * X'16 = bf16(fl32(x fl32(1/s))) (X itself when the handle has no AWQ
+ * scale); Y = bf16(X'16 W^16 + b) with float32 accumulation.  Because of the
+ * weight rounding this differs from svdq_awq_linear (float32 weights) by up
+ * to sum_k |x'_k| |w^16 - w^| per output; use svdq_awq_linear for the
+ * precision-sensitive few-row modulation projections and this call for
+ * batches of hundreds of rows and more.
+ *   X dev bf16 [M][K] (16-byte aligned), Y dev bf16 [M][N] (32-byte aligned),
+ *   N % 16 == 0, M >= 0 (0: no-op).  Asynchronous on `stream`.
+ *   Errors: INVALID_ARG (null, or the handle belongs to another device),
+ *   SHAPE, ALIGNMENT, UNSUPPORTED_DEVICE, CUDA.
+ * ------------------------------------------------------------------------ */
+svdq_status svdq_awq_gemm(const svdq_awq_weights* w, int M, const void* X, void* Y, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
  * Diagnostics.

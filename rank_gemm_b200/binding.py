@@ -86,6 +86,9 @@ _SIGS = {
     "svdq_awq_free": (_i, [_vp]),
     "svdq_awq_view": (_i, [_vp, ctypes.POINTER(AwqInfo)]),
     "svdq_awq_linear": (_i, [_vp, _i, _vp, _vp, _vp]),
+    "svdq_awq_gemm": (_i, [_vp, _i, _vp, _vp, _vp]),
+    "svdq_linear_host_workspace_bytes": (ctypes.c_size_t, [_vp, _i]),
+    "svdq_linear_host": (_i, [_vp, _i, _vp, _i, _vp, _vp, ctypes.c_size_t, _vp]),
     "svdq_poll_device_error": (_i, [_vp]),
     "svdq_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
     "svdq_debug_override_cc": (None, [_i, _i]),
@@ -201,6 +204,28 @@ def svdq_linear(w, M, X, epi, Y, workspace, ws_bytes=None, stream=None):
            "svdq_linear")
 
 
+def _host_ptr(t) -> Optional[int]:
+    """Address of a host tensor argument (svdq_linear_host's X and Y)."""
+    if t is None:
+        return None
+    if isinstance(t, torch.Tensor):
+        if t.is_cuda:
+            raise ValueError("svdq: this argument is host memory; a device tensor was given")
+        if not t.is_contiguous():
+            raise ValueError("svdq: a tensor argument is not contiguous; the library reads packed arrays")
+    return t.data_ptr()
+
+
+def svdq_linear_host_workspace_bytes(w, M) -> int:
+    return lib.svdq_linear_host_workspace_bytes(w, M)
+
+
+def svdq_linear_host(w, M, X_host, epi, Y_host, workspace, ws_bytes=None, stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size() if ws_bytes is None else ws_bytes
+    _check(lib.svdq_linear_host(w, M, _host_ptr(X_host), epi, _host_ptr(Y_host), _ptr(workspace), ws_bytes,
+                                _stream(stream)), "svdq_linear_host")
+
+
 def svdq_linear_dynamic_workspace_bytes(w, M) -> int:
     return lib.svdq_linear_dynamic_workspace_bytes(w, M)
 
@@ -283,6 +308,10 @@ def svdq_awq_view(w) -> AwqInfo:
 
 def svdq_awq_linear(w, M, X, Y, stream=None):
     _check(lib.svdq_awq_linear(w, M, _ptr(X), _ptr(Y), _stream(stream)), "svdq_awq_linear")
+
+
+def svdq_awq_gemm(w, M, X, Y, stream=None):
+    _check(lib.svdq_awq_gemm(w, M, _ptr(X), _ptr(Y), _stream(stream)), "svdq_awq_gemm")
 
 
 def svdq_poll_device_error(stream=None) -> int:

@@ -64,7 +64,6 @@ struct svdq_weights {
   uint8_t* sR;
   uint8_t* sR_rep;   // NVFP4: kernel 2's replicated copy of sR
   uint8_t* qR8;      // INT4: kernel 2's copy of qR, one E4M3 byte per code [N_pad][K_pad]
-  uint32_t* L1frag;  // NVFP4, r_tot <= 32: [L1f | A] as mma B fragments, read when the layer before emits into this one
   __nv_bfloat16* L1t;
   __nv_bfloat16* L2a;
   float* bias_f;
@@ -234,6 +233,7 @@ K1Params k1_params(const svdq_weights* w, const DevState* d, int M, void* qX, vo
   p.do_quant = do_quant;
   p.do_lr = do_lr;
   p.stages = 0;
+  p.ksplit = 2;
   p.inv_lambda = w->lambda_inv_k1;
   p.L1t = w->L1t;
   p.s_t = w->s_tX;
@@ -258,7 +258,7 @@ svdq_status run_k1(const svdq_weights* w, int M, const void* X, void* qX, void* 
   CUtensorMap tmX;
   if (!tmap_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, w->K, M, (uint64_t)w->K * 2, 64, K1_BOX_ROWS))
     return SVDQ_ERR_CUDA;
-  return from_cuda(launch_quant_down(tmX, k1_params(w, d, M, qX, sX, LR, do_quant, do_lr, dyn), stream));
+  return from_cuda(launch_quant_down(tmX, k1_params(w, d, M, qX, sX, LR, do_quant, do_lr, dyn), d->num_sms, stream));
 }
 
 svdq_status run_k2(const svdq_weights* w, int M, const void* qX, const void* sX, const void* LR,
@@ -335,7 +335,9 @@ struct svdq_awq_weights {
   uint8_t* zero;
   float* inv_s;
   float* bias_f;
-  CUtensorMap tm_code, tm_scale, tm_zero;   // the layer kernel's TMA views of the three
+  CUtensorMap tm_code, tm_scale, tm_zero;   // the GEMV's TMA views of the three
+  CUtensorMap tm_code_g, tm_scale_g, tm_zero_g;   // the tensor-core GEMM's (256-feature boxes)
+  bool has_s;                                // an AWQ scale was given (the GEMM rescales X)
 };
 
 namespace {
@@ -353,7 +355,6 @@ void free_buffers(svdq_weights* w) {
   cudaFree(w->sR);
   cudaFree(w->sR_rep);
   cudaFree(w->qR8);
-  cudaFree(w->L1frag);
   cudaFree(w->L1t);
   cudaFree(w->L2a);
   cudaFree(w->bias_f);
@@ -463,7 +464,6 @@ svdq_status svdq_prepare_weights(svdq_format fmt, int K, int N, int rank, const 
   bool ok = cudaMalloc(&w->qR, qr_b) == cudaSuccess && cudaMalloc(&w->sR, sr_b) == cudaSuccess &&
             (fmt != SVDQ_NVFP4 || cudaMalloc(&w->sR_rep, 4 * sr_b) == cudaSuccess) &&
             (fmt != SVDQ_INT4 || cudaMalloc(&w->qR8, 2 * qr_b) == cudaSuccess) &&
-            (fmt != SVDQ_NVFP4 || r_tot > 32 || cudaMalloc(&w->L1frag, (size_t)w->K_pad * 64) == cudaSuccess) &&
             cudaMalloc(&w->L1t, (size_t)r_tot * w->K_pad * 2) == cudaSuccess &&
             cudaMalloc(&w->L2a, (size_t)w->N_pad * w->r_pad * 2) == cudaSuccess &&
             cudaMalloc(&w->bias_f, (size_t)w->N_pad * 4) == cudaSuccess &&
@@ -501,7 +501,6 @@ svdq_status svdq_prepare_weights(svdq_format fmt, int K, int N, int rank, const 
   p.sR = w->sR;
   p.sR_rep = w->sR_rep;
   p.qR8 = w->qR8;
-  p.L1frag = w->L1frag;
   p.L1t = w->L1t;
   p.L2a = w->L2a;
   p.bias_f = w->bias_f;
@@ -705,13 +704,13 @@ svdq_status svdq_linear_dynamic(const svdq_weights* w, int M, const void* X, svd
 // ---------------------------------------------------------------- one layer into the next
 // [layer 1's workspace | the next layer's LR partials]
 static size_t emit_part_bytes(const svdq_weights* w1, const svdq_weights* w2, int M) {
-  return align256((size_t)2 * (w1->N_pad / 256) * round_up(M, 128) * LR_PART_STRIDE * 4);
+  return align256((size_t)(w1->N_pad / 256) * round_up(M, 128) * LR_PART_STRIDE * 4);
 }
 
 static svdq_status check_pair(const svdq_weights* w1, const svdq_weights* w2) {
   if (!w1 || !w2) return SVDQ_ERR_INVALID_ARG;
   if (w1->fmt != SVDQ_NVFP4 || w2->fmt != SVDQ_NVFP4) return SVDQ_ERR_INVALID_ARG;
-  if (w2->K != w1->N || w2->K_pad != w1->N_pad || w2->r_tot > 32) return SVDQ_ERR_SHAPE;
+  if (w2->K != w1->N || w2->K_pad != w1->N_pad || w2->r_tot > 64) return SVDQ_ERR_SHAPE;
   return w1->dev == w2->dev ? SVDQ_OK : SVDQ_ERR_INVALID_ARG;
 }
 
@@ -737,7 +736,7 @@ svdq_status svdq_linear_emit_next(const svdq_weights* w1, const svdq_weights* w2
   if ((s = run_k1(w1, M, X, qX, sX, LR, 1, 1, stream)) != SVDQ_OK) return s;
   K2Params::Next nx;
   nx.inv_lambda = w2->lambda_inv;
-  nx.L1frag = w2->L1frag;
+  nx.L1t = w2->L1t;
   nx.s_t = w2->s_tX;
   nx.six_st = 6.0f * w2->s_tX;   // one IEEE float32 multiply, as for kernel 1
   nx.r_tot = w2->r_tot;
@@ -745,7 +744,7 @@ svdq_status svdq_linear_emit_next(const svdq_weights* w1, const svdq_weights* w2
   nx.sX = static_cast<uint8_t*>(sX2);
   nx.part = part;
   if ((s = run_k2(w1, M, qX, sX, LR, epi, nullptr, true, stream, nullptr, &nx)) != SVDQ_OK) return s;
-  return from_cuda(launch_next_lr_reduce(part, 2 * (w1->N_pad / 256), M, round_up(M, 128), w2->r_tot, w2->r_pad,
+  return from_cuda(launch_next_lr_reduce(part, w1->N_pad / 256, M, round_up(M, 128), w2->r_tot, w2->r_pad,
                                          static_cast<__nv_bfloat16*>(LR2), stream));
 }
 
@@ -883,8 +882,14 @@ svdq_status svdq_awq_prepare(int K, int N, const void* W_t, const float* s, cons
     return from_cuda(e);
   }
   // stage boxes: 16 code chunks x 32 features x 16 bytes; 8 groups x 32 features of scales and zero points
+  w->has_s = s != nullptr;
   const bool maps =
       tmap_3d_u8(&w->tm_code, w->code, 16, w->N_pad, (uint64_t)K / 32, 16, (uint64_t)w->N_pad * 16, 16, 32, 16) &&
+      tmap_3d_u8(&w->tm_code_g, w->code, 16, w->N_pad, (uint64_t)K / 32, 16, (uint64_t)w->N_pad * 16, 16, 256, 2) &&
+      tmap_2d(&w->tm_scale_g, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, w->scale, w->N_pad, G, (uint64_t)w->N_pad * 2, 256, 1,
+              CU_TENSOR_MAP_SWIZZLE_NONE) &&
+      tmap_2d(&w->tm_zero_g, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->zero, w->N_pad, G, w->N_pad, 256, 1,
+              CU_TENSOR_MAP_SWIZZLE_NONE) &&
       tmap_2d(&w->tm_scale, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, w->scale, w->N_pad, G, (uint64_t)w->N_pad * 2, 32, 8,
               CU_TENSOR_MAP_SWIZZLE_NONE) &&
       tmap_2d(&w->tm_zero, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->zero, w->N_pad, G, w->N_pad, 32, 8,
@@ -950,6 +955,34 @@ svdq_status svdq_awq_linear(const svdq_awq_weights* w, int M, const void* X, voi
   p.Y = static_cast<__nv_bfloat16*>(Y);
   p.err = dev_err(d);
   return from_cuda(launch_awq_gemv(w->tm_code, w->tm_scale, w->tm_zero, p, d->num_sms, stream));
+}
+
+svdq_status svdq_awq_gemm(const svdq_awq_weights* w, int M, const void* X, void* Y, cudaStream_t stream) {
+  if (!w || (M > 0 && (!X || !Y))) return SVDQ_ERR_INVALID_ARG;
+  if (M < 0 || w->N % 16) return SVDQ_ERR_SHAPE;
+  if (!aligned16(X) || !aligned32(Y)) return SVDQ_ERR_ALIGNMENT;
+  DevState* d = nullptr;
+  svdq_status st = current_device(&d);
+  if (st != SVDQ_OK) return st;
+  int dev = -1;
+  cudaGetDevice(&dev);
+  if (dev != w->dev) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  CUtensorMap tmX;
+  if (!tmap_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, w->K, M, (uint64_t)w->K * 2, 64, 128))
+    return SVDQ_ERR_CUDA;
+  AwqGemmParams p;
+  p.M = M;
+  p.K = w->K;
+  p.N = w->N;
+  p.N_pad = w->N_pad;
+  p.num_m_blocks = (M + 127) / 128;
+  p.num_n_blocks = (w->N + 255) / 256;
+  p.inv_s = w->inv_s;
+  p.bias = w->bias_f;
+  p.Y = static_cast<__nv_bfloat16*>(Y);
+  p.err = dev_err(d);
+  return from_cuda(launch_awq_gemm(tmX, w->tm_code_g, w->tm_scale_g, w->tm_zero_g, p, w->has_s, d->num_sms, stream));
 }
 
 svdq_status svdq_poll_device_error(cudaStream_t stream) {

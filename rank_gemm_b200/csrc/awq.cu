@@ -19,7 +19,8 @@
 // (512 contiguous bytes per warp and chunk); the 8 warps of a CTA split K;
 // x' sits in shared memory and every lane reads the same word (broadcast).
 // A code becomes a float with one logic operation: its nibble, kept at bit
-// 4j of a 16-bit half-word, is OR-ed into the mantissa of 2^23, giving
+// 4j of a 16-bit half-word (the codes of 8 consecutive k sit in a 32-bit word
+// in the order of awq_nibble_pos), is OR-ed into the mantissa of 2^23, giving
 // 2^23 + 16^j q exactly; subtracting 2^23 + 16^j zero leaves 16^j (q - zero),
 // and x' is staged pre-multiplied by 16^-j (exact), so one packed fp32 FMA
 // takes two codes.
@@ -98,7 +99,7 @@ __global__ void awq_quantize_kernel(AwqPrepParams p) {
 #pragma unroll
   for (int j = 0; j < GROUP; ++j) {
     const float q = fminf(fmaxf(rintf(__fdiv_rn(v[j], d)) + zf, 0.f), 15.f);
-    words[j >> 3] |= (uint32_t)q << (4 * (j & 7));
+    words[j >> 3] |= (uint32_t)q << (4 * awq_nibble_pos(j & 7));
   }
   for (int h = 0; h < 2; ++h)
     *reinterpret_cast<uint4*>(code + ((size_t)(2 * g + h) * p.N_pad + n) * 16) =
@@ -203,12 +204,14 @@ __global__ void __launch_bounds__(THREADS + 32, 3)
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
               const float x = __uint_as_float((j & 1) ? (xw[j >> 1] & 0xFFFF0000u) : (xw[j >> 1] << 16));
-              // fl32(x / s) times 16^-(j mod 4) (the column's position in its half-word): exact
-              o[j] = __fmul_rn(x, il[j]) * __uint_as_float((uint32_t)(127 - 4 * (j & 3)) << 23);
+              // fl32(x / s) times 16^-(p mod 4), p = awq_nibble_pos(j) (the code's
+              // position in its half-word): exact
+              o[j] = __fmul_rn(x, il[j]) * __uint_as_float((uint32_t)(127 - 4 * (awq_nibble_pos(j) & 3)) << 23);
             }
+            // staged in nibble order: position p of the 8 holds column k with awq_nibble_pos(k) = p
             float4* dst = reinterpret_cast<float4*>(xs + (size_t)i * 8);
-            dst[0] = make_float4(o[0], o[1], o[2], o[3]);
-            dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+            dst[0] = make_float4(o[0], o[2], o[4], o[6]);
+            dst[1] = make_float4(o[1], o[3], o[5], o[7]);
           }
         }
       }

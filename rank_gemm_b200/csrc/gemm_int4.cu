@@ -20,11 +20,12 @@
 //                tiles of qX and qR (128-byte swizzle) into the operand ring
 //                and the k-tile's scale chunks of both (1 KB each) into a
 //                scale ring; then the low-rank chunks (LR and L2, 64 columns).
-//   warp 1       TMEM owner and MMA issuer (per group into one of four TMEM
-//                buffers; the low-rank chunks as kind::f16 into one more
-//                buffer use).
+//   warp 1       TMEM owner and MMA issuer (per 128-wide k-tile, its two
+//                groups into the two halves of one of two TMEM buffers; the
+//                low-rank chunks as kind::f16 into one more buffer use).
 //   warps 2-17   rescale + epilogue: 4 warps per TMEM sub-partition, 32 columns
-//                each; fp32 accumulators in registers; bias, GELU, bf16 store.
+//                each, one barrier round trip per k-tile (two groups); fp32
+//                accumulators in registers; bias, GELU, bf16 store.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -43,14 +44,15 @@ constexpr int W_MMA = 1, W_RESCALE = 2;
 constexpr int RS_WARPS = 16;             // four per TMEM sub-partition, 32 columns each
 constexpr int RS_COLS = BN / (RS_WARPS / 4);
 constexpr int THREADS = (W_RESCALE + RS_WARPS) * 32;
-constexpr int NBUF = 4;                  // TMEM group buffers of BN columns
-constexpr uint32_t TMEM_COLS = NBUF * BN;
+constexpr int NKB = 2;                   // TMEM k-tile buffers, each the two groups' BN columns side by side
+constexpr uint32_t KB_COLS = 2 * BN;
+constexpr uint32_t TMEM_COLS = NKB * KB_COLS;
 // kind::f8f6f4: fp32 D, E4M3 A and B (format code 0), K-major
 constexpr uint32_t IDESC_F8 = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 constexpr uint32_t IDESC_BF = idesc_bf16_f32(BM, BN);
 
 struct Ctl {
-  uint64_t full[MS], empty[MS], cfull[SC], cempty[SC], dfull[NBUF], dempty[NBUF];
+  uint64_t full[MS], empty[MS], cfull[SC], cempty[SC], dfull[NKB], dempty[NKB];
   uint32_t tmem_base;
   int abort;
 };
@@ -120,7 +122,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(smem_u32(&ctl->cfull[c]), 1);
       mbar_init(smem_u32(&ctl->cempty[c]), RS_WARPS);
     }
-    for (int b = 0; b < NBUF; ++b) {
+    for (int b = 0; b < NKB; ++b) {
       mbar_init(smem_u32(&ctl->dfull[b]), 1);
       mbar_init(smem_u32(&ctl->dempty[b]), RS_WARPS);
     }
@@ -195,19 +197,20 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           tc_fence_after();
           const uint32_t a = smem_u32(ring + s * STAGE_BYTES), b = a + OP_BYTES;
-          for (int j = 0; j < 2; ++j, ++uses) {
-            const uint32_t buf = uses % NBUF, dph = (uses / NBUF) & 1;
-            if (!mbar_wait(smem_u32(&ctl->dempty[buf]), dph ^ 1, abort_flag, p.err)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t d = tmem + buf * BN;
+          const uint32_t buf = uses % NKB, dph = (uses / NKB) & 1;
+          if (!mbar_wait(smem_u32(&ctl->dempty[buf]), dph ^ 1, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {   // group j of the k-tile into columns j BN of the buffer
+            const uint32_t d = tmem + buf * KB_COLS + j * BN;
             mma_f8(d, desc_k_sw128(a + 64 * j), desc_k_sw128(b + 64 * j), IDESC_F8, 0);
             mma_f8(d, desc_k_sw128(a + 64 * j + 32), desc_k_sw128(b + 64 * j + 32), IDESC_F8, 1);
-            tc_commit(smem_u32(&ctl->dfull[buf]));
           }
-          if (!ok) break;
+          tc_commit(smem_u32(&ctl->dfull[buf]));
+          ++uses;
           tc_commit(smem_u32(&ctl->empty[s]));
           if (++s == MS) {
             s = 0;
@@ -216,7 +219,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         if (!ok) break;
         if (nl) {
-          const uint32_t buf = uses % NBUF, dph = (uses / NBUF) & 1;
+          const uint32_t buf = uses % NKB, dph = (uses / NKB) & 1;
           if (!mbar_wait(smem_u32(&ctl->dempty[buf]), dph ^ 1, abort_flag, p.err)) break;
           for (int c = 0; c < nl; ++c) {
             if (!mbar_wait(smem_u32(&ctl->full[s]), ph, abort_flag, p.err)) {
@@ -227,7 +230,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint32_t a = smem_u32(ring + s * STAGE_BYTES), b = a + OP_BYTES;
             const int steps = min(4, (p.r_tot - 64 * c) / 16);
             for (int j = 0; j < steps; ++j)
-              mma_bf16(tmem + buf * BN, desc_k_sw128(a + 32 * j), desc_k_sw128(b + 32 * j), IDESC_BF,
+              mma_bf16(tmem + buf * KB_COLS, desc_k_sw128(a + 32 * j), desc_k_sw128(b + 32 * j), IDESC_BF,
                        (c | j) != 0);
             tc_commit(smem_u32(&ctl->empty[s]));
             if (++s == MS) {
@@ -262,22 +265,29 @@ __global__ void __launch_bounds__(THREADS, 1)
           break;
         }
         const float* sc = reinterpret_cast<const float*>(sring + c * SC_BYTES);
-        for (int j = 0; j < 2; ++j, ++uses) {        // the k-tile's two 64-groups
+        const uint32_t buf = uses % NKB, dph = (uses / NKB) & 1;
+        ++uses;
+        if (!mbar_wait(smem_u32(&ctl->dfull[buf]), dph, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // the two groups' sums of this warp's 32 columns; after the second
+        // load the buffer goes back to the MMA warp
+        const uint32_t taddr = tmem + ((uint32_t)(sub * 32) << 16) + buf * KB_COLS + quarter * RS_COLS;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {                // the k-tile's two 64-groups
+          uint32_t r[32];
+          tmem_ld32(taddr + j * BN, r);
+          tmem_wait_ld();
+          if (j == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&ctl->dempty[buf]));
+          }
           const uint32_t sxb = __float_as_uint(sc[j * 128 + row]);
           const uint64_t sx2 = u2(sxb, sxb);
           const uint32_t sra = smem_u32(sc + 256 + j * 128 + quarter * RS_COLS);
-          const uint32_t buf = uses % NBUF, dph = (uses / NBUF) & 1;
-          if (!mbar_wait(smem_u32(&ctl->dfull[buf]), dph, abort_flag, p.err)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          uint32_t r[32];
-          tmem_ld32(tmem + ((uint32_t)(sub * 32) << 16) + buf * BN + quarter * RS_COLS, r);
-          tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&ctl->dempty[buf]));
           // acc += (sx sr) d: the group's exact fp32 sum, rescaled by the
           // product of two binary16 scales (exact in fp32), then one FMA
 #pragma unroll
@@ -297,14 +307,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (ok && nl) {
         // the low-rank branch: LR (L2) accumulated in fp32 by the tensor core
-        const uint32_t buf = uses % NBUF, dph = (uses / NBUF) & 1;
+        const uint32_t buf = uses % NKB, dph = (uses / NKB) & 1;
         ++uses;
         if (!mbar_wait(smem_u32(&ctl->dfull[buf]), dph, abort_flag, p.err)) {
           ok = false;
         } else {
           tc_fence_after();
           uint32_t r[32];
-          tmem_ld32(tmem + ((uint32_t)(sub * 32) << 16) + buf * BN + quarter * RS_COLS, r);
+          tmem_ld32(tmem + ((uint32_t)(sub * 32) << 16) + buf * KB_COLS + quarter * RS_COLS, r);
           tmem_wait_ld();
           tc_fence_before();
           __syncwarp();

@@ -29,9 +29,12 @@
 //               bf16 and the 32-byte stores, which overlap the next tile's MMAs.
 //               In emit mode (cross-layer fusion) the epilogue instead writes
 //               the next layer's kernel-1 outputs: its NVFP4 codes and
-//               replicated scales, and float32 partials of its low-rank down
-//               projection computed with mma.sync from bf16 pairs parked in
-//               free TMEM columns.
+//               replicated scales from bf16 pairs parked in free TMEM
+//               columns, and the float32 partial of its low-rank down
+//               projection, which the MMA warp computes on the tensor core
+//               with those parked pairs as the A operand (A in TMEM) and the
+//               next layer's L1 slice as B, loaded as one extra ring stage a
+//               few k-tiles into the following tile.
 // All waits are bounded (see mbar_wait); TMEM is freed on every exit path.
 #include "common.cuh"
 #include "kernels.h"
@@ -52,6 +55,8 @@ constexpr int EPI_WARPS = 8;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0, SFA_COL = 256, SFB_COL = 272;
 constexpr uint32_t STASH_COL = 320;   // emit mode: bf16 pairs of the row slices, 64 columns per half
+constexpr uint32_t DPART_COL = 448;   // emit mode: the next layer's LR partial, up to 64 float32 columns
+constexpr int EMIT_AT = 3;            // emit mode: the partial's stage follows this FP4 k-tile of the next tile
 constexpr uint32_t IDESC_F4 = idesc_nvf4(BLOCK_M, BLOCK_N);
 constexpr uint32_t IDESC_BF = idesc_bf16_f32(BLOCK_M, BLOCK_N);
 
@@ -59,6 +64,7 @@ struct Ctl {
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
   uint64_t tfull, tempty;
+  uint64_t stash_full, part_full, part_empty;   // emit mode
   uint32_t tmem_base;
   int abort;
 };
@@ -93,6 +99,48 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+// D (TMEM) += A (TMEM: 128 lanes x 16 bf16, two per 32-bit column) B (smem descriptor), kind::f16.
+__device__ __forceinline__ void mma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 32 lanes x 16 consecutive 32-bit columns -> 16 registers per thread.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+// The k-iterations of one tile: the FP4 k-tiles, then the low-rank chunks;
+// in emit mode with a previous tile, that tile's LR-partial stage comes after
+// FP4 k-tile EMIT_AT (or the last one), by when its epilogue has parked its
+// output.  kind 0: FP4 k-tile idx; 1: low-rank chunk idx; 2: the partial.
+struct Iter {
+  int kind, idx;
+};
+__device__ __forceinline__ Iter iter_of(int it, int nk, bool with_part) {
+  if (!with_part) return it < nk ? Iter{0, it} : Iter{1, it - nk};
+  const int at = min(EMIT_AT, nk - 1) + 1;
+  if (it < at) return Iter{0, it};
+  if (it == at) return Iter{2, 0};
+  return it - 1 < nk ? Iter{0, it - 1} : Iter{1, it - 1 - nk};
+}
+
+// Emit mode: the stash holds the tile's 256 bf16 columns in the order the
+// epilogue warps park them (warp column set ch, then the 128-column half),
+// i.e. stash position p holds tile column p with bits 6 and 7 swapped: the
+// 64-wide block q of the stash is column block (q & 1) * 2 + (q >> 1).
+__device__ __forceinline__ uint32_t stash_block(uint32_t q) { return ((q & 1u) << 1) | (q >> 1); }
+
 }  // namespace
 
 // EMIT: instead of Y, write the next layer's kernel-1 outputs from this
@@ -124,6 +172,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     mbar_init(smem_u32(&ctl->tfull), 1);
     mbar_init(smem_u32(&ctl->tempty), EPI_WARPS);
+    mbar_init(smem_u32(&ctl->stash_full), EPI_WARPS);
+    mbar_init(smem_u32(&ctl->part_full), 1);
+    mbar_init(smem_u32(&ctl->part_empty), EPI_WARPS);
     ctl->abort = 0;
     fence_barrier_init();
   }
@@ -149,34 +200,46 @@ __global__ void __launch_bounds__(THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-        int mb, nb;
-        tile_coords(tile, p.num_m_blocks, p.num_n_blocks, mb, nb);
-        for (int it = 0; it < kiters; ++it) {
+      int prev_nb = -1;   // emit mode: the previous tile's column block
+      // one more pass of the loop in emit mode: the last tile's partial stage
+      for (int tile = blockIdx.x; ok && (tile < num_tiles || (EMIT && prev_nb >= 0)); tile += gridDim.x) {
+        const bool last = tile >= num_tiles;
+        int mb = 0, nb = 0;
+        if (!last) tile_coords(tile, p.num_m_blocks, p.num_n_blocks, mb, nb);
+        const bool with_part = EMIT && prev_nb >= 0;
+        const int n_it = last ? 1 : kiters + (with_part ? 1 : 0);
+        for (int it = 0; it < n_it; ++it) {
           if (!mbar_wait(smem_u32(&ctl->empty[stage]), phase ^ 1, abort_flag, p.err)) {
             ok = false;
             break;
           }
           const uint32_t st = smem_u32(base + stage * STAGE_BYTES);
           const uint32_t bar = smem_u32(&ctl->full[stage]);
-          if (it < p.nk) {
+          const Iter I = last ? Iter{2, 0} : iter_of(it, p.nk, with_part);
+          if (I.kind == 0) {
             mbar_arrive_expect_tx(bar, STAGE_BYTES);
-            tma_load_2d(st, &tmA, it * 128, mb * BLOCK_M, bar);
-            tma_load_2d(st + A_BYTES, &tmB, it * 128, nb * BLOCK_N, bar);
-            bulk_load(st + A_BYTES + B_BYTES, p.sX + ((size_t)mb * p.nk + it) * SFA_BYTES, SFA_BYTES, bar);
-            bulk_load(st + A_BYTES + B_BYTES + SFA_BYTES, p.sR + ((size_t)nb * p.nk + it) * SFB_BYTES, SFB_BYTES,
-                      bar);
-          } else {
-            const int c = it - p.nk;
+            tma_load_2d(st, &tmA, I.idx * 128, mb * BLOCK_M, bar);
+            tma_load_2d(st + A_BYTES, &tmB, I.idx * 128, nb * BLOCK_N, bar);
+            bulk_load(st + A_BYTES + B_BYTES, p.sX + ((size_t)mb * p.nk + I.idx) * SFA_BYTES, SFA_BYTES, bar);
+            bulk_load(st + A_BYTES + B_BYTES + SFA_BYTES, p.sR + ((size_t)nb * p.nk + I.idx) * SFB_BYTES,
+                      SFB_BYTES, bar);
+          } else if (I.kind == 1) {
             mbar_arrive_expect_tx(bar, A_BYTES + B_BYTES);
-            tma_load_2d(st, &tmLR, c * 64, mb * BLOCK_M, bar);
-            tma_load_2d(st + A_BYTES, &tmL2, c * 64, nb * BLOCK_N, bar);
+            tma_load_2d(st, &tmLR, I.idx * 64, mb * BLOCK_M, bar);
+            tma_load_2d(st + A_BYTES, &tmL2, I.idx * 64, nb * BLOCK_N, bar);
+          } else {
+            // the next layer's L1 rows of the previous tile's 256 columns:
+            // four staged [r_tot x 64] boxes, contiguous
+            const uint32_t bytes = 4u * (uint32_t)p.next.r_tot * 128u;
+            mbar_arrive_expect_tx(bar, bytes);
+            bulk_load(st, p.next.L1t + (size_t)prev_nb * 4 * p.next.r_tot * 64, bytes, bar);
           }
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
+        prev_nb = last ? -1 : nb;
       }
     }
   } else if (warp == 1) {
@@ -185,10 +248,32 @@ __global__ void __launch_bounds__(THREADS, 1)
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-        if (!mbar_wait(smem_u32(&ctl->tempty), acc_phase ^ 1, abort_flag, p.err)) break;
+      bool prev = false;            // emit mode: a previous tile's partial is still to come
+      uint32_t part_phase = 0;      // emit mode: stash_full / part_full / part_empty uses
+      const uint32_t idesc_p = EMIT ? idesc_bf16_f32(BLOCK_M, p.next.r_tot) : 0u;
+      // the next layer's LR partial of the previous tile: A = the parked bf16
+      // output (TMEM), B = its L1 rows (the stage), D = DPART_COL
+      auto partial = [&](uint32_t a) -> bool {
+        if (!mbar_wait(smem_u32(&ctl->stash_full), part_phase, abort_flag, p.err) ||
+            !mbar_wait(smem_u32(&ctl->part_empty), part_phase ^ 1, abort_flag, p.err))
+          return false;
         tc_fence_after();
-        for (int it = 0; it < kiters; ++it) {
+        const uint32_t box = (uint32_t)p.next.r_tot * 128u;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          mma_bf16_ta(tmem + DPART_COL, tmem + STASH_COL + 8 * j,
+                      desc_k_sw128(a + stash_block((uint32_t)j >> 2) * box + 32 * (j & 3)), idesc_p, j != 0);
+        return true;
+      };
+      for (int tile = blockIdx.x; ok && (tile < num_tiles || (EMIT && prev)); tile += gridDim.x) {
+        const bool last = tile >= num_tiles;
+        const bool with_part = EMIT && prev;
+        if (!last) {
+          if (!mbar_wait(smem_u32(&ctl->tempty), acc_phase ^ 1, abort_flag, p.err)) break;
+          tc_fence_after();
+        }
+        const int n_it = last ? 1 : kiters + (with_part ? 1 : 0);
+        for (int it = 0; it < n_it; ++it) {
           if (!mbar_wait(smem_u32(&ctl->full[stage]), phase, abort_flag, p.err)) {
             ok = false;
             break;
@@ -196,7 +281,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           tc_fence_after();
           const uint32_t a = smem_u32(base + stage * STAGE_BYTES);
           const uint32_t b = a + A_BYTES;
-          if (it < p.nk) {
+          const Iter I = last ? Iter{2, 0} : iter_of(it, p.nk, with_part);
+          if (I.kind == 0) {
             const uint32_t sfa = b + B_BYTES, sfb = sfa + SFA_BYTES;
             // six copies of 8 columns: SFA k-blocks (0,1), (2,3); SFB k-block kb, both row halves
 #pragma unroll
@@ -206,22 +292,31 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int kb = 0; kb < 4; ++kb)
               mma_nvf4(tmem + ACC_COL, desc_k_sw128(a + 32 * kb), desc_k_sw128(b + 32 * kb), IDESC_F4,
-                       tmem + SFA_COL + 4 * kb, tmem + SFB_COL + 8 * kb, (it | kb) != 0);
-          } else {
-            const int c = it - p.nk;
-            const int steps = min(4, (p.r_tot - 64 * c) / 16);
+                       tmem + SFA_COL + 4 * kb, tmem + SFB_COL + 8 * kb, (I.idx | kb) != 0);
+          } else if (I.kind == 1) {
+            const int steps = min(4, (p.r_tot - 64 * I.idx) / 16);
             for (int j = 0; j < steps; ++j)
               mma_bf16(tmem + ACC_COL, desc_k_sw128(a + 32 * j), desc_k_sw128(b + 32 * j), IDESC_BF, 1);
+          } else {
+            if (!partial(a)) {
+              ok = false;
+              break;
+            }
           }
           tc_commit(smem_u32(&ctl->empty[stage]));
+          if (I.kind == 2) {
+            tc_commit(smem_u32(&ctl->part_full));
+            part_phase ^= 1;
+          }
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
-        if (!ok) break;
+        if (!ok || last) break;
         tc_commit(smem_u32(&ctl->tfull));
         acc_phase ^= 1;
+        prev = true;
       }
     }
   } else {
@@ -323,66 +418,11 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_st16(stash + c * 16, pk);
         }
         tmem_wait_st();
-        // phase B1: the LR partial on the tensor cores (mma.m16n8k16 over this
-        // warp's 32 rows x its 128 columns x 32 ranks).  The A fragments come
-        // straight from the stash with tcgen05.ld.16x256b (all sixteen loads
-        // before one wait), whose k order inside a 16-column group the B
-        // fragments' layout matches; B streams from L2 two groups ahead.
-        const int fi = lane >> 2, fq = lane & 3;
-        float acc[2][4][4];
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-          for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-            for (int e2 = 0; e2 < 4; ++e2) acc[h][nt][e2] = 0.f;
-        {
-          uint32_t fr[8][2][4];
-#pragma unroll
-          for (int g = 0; g < 8; ++g) {
-            tmem_ld_16x256b(stash + g * 8, fr[g][0]);                 // rows 0-15 of this warp
-            tmem_ld_16x256b(stash + g * 8 + (16u << 16), fr[g][1]);   // rows 16-31
-          }
-          auto bfrag = [&](int g) {
-            const int nn = n0 + 128 * (g >> 2) + 16 * (g & 3);
-            return reinterpret_cast<const uint4*>(nx.L1frag + ((size_t)(nn >> 4) * 32 + lane) * 8);
-          };
-          uint4 bq[2][2];
-          bq[0][0] = __ldg(bfrag(0));
-          bq[0][1] = __ldg(bfrag(0) + 1);
-          bq[1][0] = __ldg(bfrag(1));
-          bq[1][1] = __ldg(bfrag(1) + 1);
-          tmem_wait_ld();
-#pragma unroll
-          for (int g = 0; g < 8; ++g) {
-            const uint4 b01 = bq[g & 1][0], b23 = bq[g & 1][1];
-            if (g + 2 < 8) {
-              bq[g & 1][0] = __ldg(bfrag(g + 2));
-              bq[g & 1][1] = __ldg(bfrag(g + 2) + 1);
-            }
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const uint32_t* f = fr[g][h];
-              mma_bf16_16816(acc[h][0], f[0], f[2], f[1], f[3], b01.x, b01.y);
-              mma_bf16_16816(acc[h][1], f[0], f[2], f[1], f[3], b01.z, b01.w);
-              mma_bf16_16816(acc[h][2], f[0], f[2], f[1], f[3], b23.x, b23.y);
-              mma_bf16_16816(acc[h][3], f[0], f[2], f[1], f[3], b23.z, b23.w);
-            }
-          }
-        }
-        // this warp's partial over its 128 columns of column block nb: rows
-        // 16 h + fi (+ 8), ranks 8 nt + 2 fq, +1 (zeros past r_tot)
-        float* pbase = nx.part + ((size_t)(2 * nb + ch) * (p.num_m_blocks * BLOCK_M) + mb * BLOCK_M + sub * 32) *
-                                     LR_PART_STRIDE;
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-          for (int nt = 0; nt < 4; ++nt)
-            if (8 * nt < nx.r_tot) {
-              float* pr = pbase + (size_t)(16 * h + fi) * LR_PART_STRIDE + 8 * nt + 2 * fq;
-              *reinterpret_cast<float2*>(pr) = make_float2(acc[h][nt][0], acc[h][nt][1]);
-              *reinterpret_cast<float2*>(pr + 8 * LR_PART_STRIDE) = make_float2(acc[h][nt][2], acc[h][nt][3]);
-            }
+        // the MMA warp may now run the LR partial over the whole tile with the
+        // parked pairs as its A operand
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&ctl->stash_full));
         // phase B2: codes and scales, the whole stash in two loads and one wait
         {
           uint32_t pa[32], pb[32];
@@ -427,6 +467,26 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
           }
         }
+        // the LR partial of this tile (sum over its 256 columns), once the MMA
+        // warp has computed it: the two warps of a sub-partition take half of
+        // the r_tot columns each, then hand the TMEM columns back
+        if (!mbar_wait(smem_u32(&ctl->part_full), acc_phase ^ 1, abort_flag, p.err)) break;
+        tc_fence_after();
+        {
+          const int half = nx.r_tot / 2, c0 = ch * half;   // a multiple of 8
+          float* prow = nx.part + ((size_t)nb * (p.num_m_blocks * BLOCK_M) + m) * LR_PART_STRIDE + c0;
+          const uint32_t dsrc = tmem + ((uint32_t)(sub * 32) << 16) + DPART_COL + (uint32_t)c0;
+          for (int c8 = 0; c8 < half; c8 += 8) {
+            uint32_t d[8];
+            tmem_ld8(dsrc + (uint32_t)c8, d);
+            tmem_wait_ld();
+            reinterpret_cast<uint4*>(prow + c8)[0] = make_uint4(d[0], d[1], d[2], d[3]);
+            reinterpret_cast<uint4*>(prow + c8)[1] = make_uint4(d[4], d[5], d[6], d[7]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&ctl->part_empty));
       }
     }
   }

@@ -28,6 +28,7 @@ struct K1Params {
   int fmt;                 // 0 NVFP4, 1 INT4
   int do_quant, do_lr;     // fused: both; unfused baseline: one of them
   int stages;              // set by the launcher
+  int ksplit;              // CTAs per row block (the cluster with the low-rank branch), set by the launcher
   const float* inv_lambda; // [K_pad], permuted per 64-wide stage (see prepare.cu)
   const __nv_bfloat16* L1t; // L1f^T in the staged layout (one contiguous tile per stage)
   float s_t, six_st;       // NVFP4 activation tensor scale and fl32(6 s_t)
@@ -46,7 +47,7 @@ struct K1Params {
 // Kernel 1 stages X in [K1_BOX_ROWS x 64] bf16 TMA boxes (128-byte swizzle);
 // the host encodes tmX with exactly this box.
 constexpr int K1_BOX_ROWS = 64;
-cudaError_t launch_quant_down(const CUtensorMap& tmX, K1Params p, cudaStream_t stream);
+cudaError_t launch_quant_down(const CUtensorMap& tmX, K1Params p, int num_sms, cudaStream_t stream);
 
 // ---------------------------------------------------------------- kernel 2
 struct K2Params {
@@ -68,26 +69,16 @@ struct K2Params {
   // layer's bf16 output Y is the next layer's activation X2 (its K = N)
   struct Next {
     const float* inv_lambda;   // [N] the next layer's 1/lambda
-    const uint32_t* L1frag;    // its first factor (with any LoRA A) as m16n8k16 B fragments (l1frag_offset)
+    const __nv_bfloat16* L1t;  // its first factor (with any LoRA A) in kernel 1's staged layout: per 64 rows
+                               // of K one [r_tot x 64] bf16 box, 128-byte swizzled (a K-major MMA B operand)
     float s_t, six_st;         // its static NVFP4 activation tensor scale and fl32(6 s_t)
-    int r_tot;                 // <= 32
+    int r_tot;                 // <= 64
     uint8_t* qX;               // [M][N_pad / 2]
     uint8_t* sX;               // replicated layout over N_pad (sfx_rep_offset)
-    float* part;               // [2 num_n_blocks][M_128][LR_PART_STRIDE] partial LR, one per warp column set
+    float* part;               // [num_n_blocks][M_128][LR_PART_STRIDE] partial LR, one per column block
   } next;
 };
-constexpr int LR_PART_STRIDE = 32;   // floats per row of an emit-mode LR partial
-// Emit mode's copy of a first factor L1 ([K][r_tot] bf16, r_tot <= 32, zeros
-// past K and r_tot) in the B-fragment order of mma.m16n8k16 over 16-row k
-// groups: the bf16 offset of element (k, r).  Lane t of a warp holds, for
-// rank 8 nt + t / 4, the four consecutive k = 16 G + 4 (t % 4) .. +3 as two
-// registers (b0, b1) at word 2 nt, 2 nt + 1 of its 8 words per group; the k
-// order this gives inside a group matches the A fragments read from TMEM with
-// tcgen05.ld.16x256b (slot pair s < 4 <- pair 2 s, slot pair s + 4 <- pair 2 s + 1).
-__host__ __device__ __forceinline__ size_t l1frag_offset(int k, int r) {
-  const int G = k >> 4, kk = k & 15, t = 4 * (r & 7) + (kk >> 2);
-  return (((size_t)G * 32 + t) * 8 + 2 * (r >> 3)) * 2 + (kk & 3);
-}
+constexpr int LR_PART_STRIDE = 64;   // floats per row of an emit-mode LR partial
 // TMA box heights the host encodes for kernel 2's operands (rows of a tile):
 // NVFP4 stages 128 rows of qX / LR and 256 rows of qR / L2a per k-tile; INT4
 // stages 128 of each.
@@ -157,7 +148,6 @@ struct PrepParams {
   uint8_t* sR_rep;             // NVFP4: kernel 2's replicated copy (sfw_rep_offset)
   uint8_t* qR8;                // INT4: kernel 2's copy of the codes as E4M3 bytes [N_pad][K_pad]
   __nv_bfloat16* L1t;          // [K_pad/64][r_tot][64], 128-byte swizzled
-  uint32_t* L1frag;            // NVFP4 with r_tot <= 32: [L1f | A] in l1frag_offset order ([K_pad / 16][32][8] words), or null
   __nv_bfloat16* L2a;          // [N_pad][r_pad]
   float* bias_f;               // [N_pad]
   float* lambda_inv;           // [K]
@@ -177,8 +167,12 @@ cudaError_t lowrank_factors(int K, int N, int r, const __nv_bfloat16* Wt, const 
 
 // ---------------------------------------------------------------- AWQ W4A16 layer
 // Codes: uint8 [K/32][N_pad][16] (chunk c holds k in [32c, 32c+32) of feature
-// n, two codes per byte, even k in the low nibble); scale binary16 and zero
-// uint8 [K/64][N_pad]; N_pad = N rounded up to 32.
+// n, 4 bits each; 32-bit word w of a chunk holds k = 32c + 8w + i at bit
+// 4 awq_nibble_pos(i): the even k in the low half-word, the odd in the high,
+// so one shift and mask give the bf16 pair (k, k + 1) and the float32
+// pairs (k, k + 2)); scale binary16 and zero uint8 [K/64][N_pad]; N_pad = N
+// rounded up to 32.
+__host__ __device__ constexpr int awq_nibble_pos(int i) { return (i >> 1) + 4 * (i & 1); }
 constexpr int AWQ_WARPS = 8;      // warps of a CTA, splitting K
 constexpr int AWQ_MB_MAX = 4;     // activation rows per pass over the weights
 constexpr int AWQ_STAGES = 4;     // TMA ring depth (stages of 8 groups x 32 features)
@@ -205,6 +199,21 @@ struct AwqParams {
   __nv_bfloat16* Y;               // [M][N]
   DeviceErr err;
 };
+// The tensor-core form (awq_gemm.cu): 128 x 256 tiles over 64-wide k-tiles.
+struct AwqGemmParams {
+  int M, K, N, N_pad;
+  int num_m_blocks, num_n_blocks;  // ceil(M / 128), ceil(N / 256)
+  const float* inv_s;              // [K] fl32(1/s) (read only when the handle has an AWQ scale)
+  const float* bias;               // [N_pad]
+  __nv_bfloat16* Y;                // [M][N], N % 16 == 0, 32-byte aligned
+  DeviceErr err;
+};
+// tmX: X bf16 [M][K], box {64, 128}, 128-byte swizzle; tmCode: the codes as a
+// 3-D uint8 tensor [K/32][N_pad][16], box {16, 256, 2}; tmScale / tmZero:
+// [K/64][N_pad] binary16 / uint8, box {256, 1}.
+cudaError_t launch_awq_gemm(const CUtensorMap& tmX, const CUtensorMap& tmCode, const CUtensorMap& tmScale,
+                            const CUtensorMap& tmZero, AwqGemmParams p, bool has_s, int num_sms,
+                            cudaStream_t stream);
 cudaError_t launch_awq_quantize(const AwqPrepParams& p, cudaStream_t stream);
 // tmCode: codes as a 3-D uint8 tensor [K/32][N_pad][16], box {16, 32, 16};
 // tmScale / tmZero: [K/64][N_pad] binary16 / uint8, box {32, 8}.

@@ -173,17 +173,6 @@ __global__ void factors_kernel(PrepParams p, float alpha) {
     const size_t off = (size_t)kb * p.r_tot * 64 + (size_t)r * 64 + ((((c >> 3) ^ (r & 7)) << 3) | (c & 7));
     p.L1t[off] = v;
   }
-  // emit mode's fragment-ordered copy: all 32 ranks, zeros past r_tot and K
-  if (p.L1frag) {
-    __nv_bfloat16* f = reinterpret_cast<__nv_bfloat16*>(p.L1frag);
-    for (int i = tid; i < 32 * p.K_pad; i += stride) {
-      const int r = i / p.K_pad, k = i % p.K_pad;
-      __nv_bfloat16 v = __float2bfloat16(0.f);
-      if (k < p.K && r < p.r_tot)
-        v = (r < p.rank) ? p.L1f[(size_t)k * p.rank + r] : p.loraA[(size_t)k * p.lora_rank + (r - p.rank)];
-      f[l1frag_offset(k, r)] = v;
-    }
-  }
   // L2a [N_pad][r_pad] = ([L2 ; B] / alpha)^T, zero padded
   for (int i = tid; i < p.N_pad * p.r_pad; i += stride) {
     const int n = i / p.r_pad, r = i % p.r_pad;

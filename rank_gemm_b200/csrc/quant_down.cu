@@ -3,8 +3,9 @@
 // model card: the Quantize and Down Projection kernels read the same input,
 // so they are fused and X is read from HBM once).
 //
-// A cluster of two CTAs owns 64 rows of X; CTA c of the cluster walks the
-// c-th half of K in 256-column stages.  A producer warp keeps a TMA ring of
+// A cluster of S CTAs (S = 2 at large batches, up to 8 at small ones, so that
+// the grid still fills the SMs) owns 64 rows of X; CTA c of the cluster walks
+// the c-th of S slices of K in 256-column stages.  A producer warp keeps a TMA ring of
 // stages in flight; a stage holds the [64 x 256] bf16 tile of X (four
 // 128-byte-swizzled [64 x 64] boxes: 512 contiguous bytes of every row, which
 // HBM streams faster than 256), the matching [r_tot x 256] tile of L1f^T
@@ -18,17 +19,20 @@
 //     A = the staged X tile (M = 64 rows), B = the L1f^T tile (N = r_tot),
 //     fp32 accumulation in TMEM across the CTA's half of K.
 // At the end four warps move the partial [64 x r_tot] tile from TMEM to
-// shared memory; after a cluster barrier CTA c adds the two partials of rows
-// [32c, 32c + 32) through distributed shared memory, always in the order
-// CTA 0, 1 (so LR is the same on every run), and stores LR in bf16.
-// Why 64 rows and two CTAs: the four-way split of a 128-row tile needs
-// clusters of four, and at one CTA per SM only 33 of those are resident at
-// once on 148 SMs; clusters of two fill every SM.
+// shared memory; after a cluster barrier CTA c adds the S partials of rows
+// [64c/S, 64(c+1)/S) through distributed shared memory, always in the order
+// CTA 0, 1, .., S-1 (so LR is the same on every run), and stores LR in bf16.
+// Why 64 rows: the four-way split of a 128-row tile needs clusters of four,
+// and at one CTA per SM only 33 of those are resident at once on 148 SMs;
+// 64-row clusters of two fill every SM at the FLUX batch sizes, and small
+// batches split K further instead of leaving SMs idle.
 // Stages are released through an mbarrier (the 16 quantizer warps plus the
 // MMA commit) instead of a CTA-wide sync, so warps drift apart and overlap
 // their load, math and store phases.  The kernel is HBM-bound: per row it
 // reads 2K bytes of X and writes about K/2 + K/16 bytes of codes and scales
 // plus 2 r_pad bytes of LR.
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -38,7 +42,6 @@ namespace {
 
 constexpr int BM = K1_BOX_ROWS;              // rows per cluster (= MMA M = TMA box rows)
 constexpr int BK = 256;                      // K columns per stage (four 64-column swizzled boxes)
-constexpr int KSPLIT = 2;                    // CTAs per cluster, each half of K
 constexpr int QWARPS = 16;                   // quantizer warps: 64 rows x 8 groups
 constexpr int THREADS = 32 * (QWARPS + 2);   // + producer warp + MMA warp
 constexpr int X_BOX = BM * 128;              // one [64 x 64] bf16 box, 8 KB
@@ -101,15 +104,16 @@ __global__ void __launch_bounds__(THREADS, 1)
     quant_down_kernel(const __grid_constant__ CUtensorMap tmX, K1Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // half of K; with the low-rank branch the two CTAs of a row block form a
+  // slice of K; with the low-rank branch the S CTAs of a row block form a
   // cluster, and the cluster rank equals this index
-  const int split = blockIdx.x % KSPLIT;
-  const int m0 = (blockIdx.x / KSPLIT) * BM;
-  // stages of 256 columns: the first CTA of the pair takes ceil(nk / 2), the
-  // second the rest (possibly none: then its partial LR is zero)
-  const int nk = p.K_pad / BK, nk0 = (nk + 1) / 2;
-  const int ns = split == 0 ? nk0 : nk - nk0;
-  const int kb0 = split * nk0;                           // first 256-column block of this CTA
+  const int S = p.ksplit;
+  const int split = blockIdx.x % S;
+  const int m0 = (blockIdx.x / S) * BM;
+  // stages of 256 columns: nk / S each, the first nk % S CTAs one more
+  // (possibly none: then the partial LR is zero)
+  const int nk = p.K_pad / BK, nq = nk / S, nr = nk % S;
+  const int ns = nq + (split < nr ? 1 : 0);
+  const int kb0 = split * nq + min(split, nr);           // first 256-column block of this CTA
 
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const Layout L = make_layout(p.stages, p.r_tot, p.do_lr != 0);
@@ -174,15 +178,26 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         tc_fence_after();
         const int kvalid = p.K - (kb0 + it) * BK;      // multiple of 64 (may be <= 0 in the pad)
-        const uint32_t xs = smem_u32(base + L.x_ring + s * X_BYTES);
-        const uint32_t ls = smem_u32(base + L.l_ring + s * L.l_bytes);
+        // descriptors of the stage's first 16 columns; a K16 step adds its byte
+        // offset / 16 to the start-address field (no carry: the shared window
+        // is below 256 KB)
+        const uint64_t dx = desc_k_sw128(smem_u32(base + L.x_ring + s * X_BYTES));
+        const uint64_t dl = desc_k_sw128(smem_u32(base + L.l_ring + s * L.l_bytes));
+        const uint32_t lstep = (uint32_t)p.r_tot * 8;   // (r_tot * 128) >> 4
+        if (kvalid >= BK) {
 #pragma unroll
-        for (int j = 0; j < BK / 16; ++j) {
-          if (j * 16 >= kvalid) break;
-          const int b = j >> 2, koff = (j & 3) * 32;
-          mma_bf16(tmem, desc_k_sw128(xs + b * X_BOX + koff), desc_k_sw128(ls + b * p.r_tot * 128 + koff), idesc,
-                   started);
+          for (int j = 0; j < BK / 16; ++j) {
+            const uint32_t b = j >> 2, ko = (j & 3) * 2;
+            mma_bf16(tmem, dx + (b * (X_BOX >> 4) + ko), dl + (b * lstep + ko), idesc, (j == 0) ? started : 1u);
+          }
           started = 1u;
+        } else {
+          for (int j = 0; j < BK / 16; ++j) {
+            if (j * 16 >= kvalid) break;
+            const uint32_t b = j >> 2, ko = (j & 3) * 2;
+            mma_bf16(tmem, dx + (b * (X_BOX >> 4) + ko), dl + (b * lstep + ko), idesc, started);
+            started = 1u;
+          }
         }
         tc_commit(smem_u32(&empty[s]));
       }
@@ -295,7 +310,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // M = 64 accumulator: row i in TMEM lane 32 (i / 16) + i % 16, column =
       // rank index; lanes 16-31 of each sub-partition are unused
       const int sub = warp & 3, row = 16 * sub + lane;
-      const bool has_mma = kb0 * BK < p.K;               // else this half lies in the K pad: zeros
+      const bool has_mma = ns > 0 && kb0 * BK < p.K;     // else this slice is empty or in the K pad: zeros
       if (mbar_wait(smem_u32(dfull), 0, abort_flag, p.err)) {
         tc_fence_after();
         for (int c0 = 0; c0 < p.r_tot; c0 += 32) {
@@ -315,8 +330,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     cluster_sync_all();
     // ---------------------------------------------------------------- cluster reduction
-    // this CTA's 32 rows; four consecutive columns per task; pad columns -> 0
-    const int rows_per = BM / KSPLIT, quads = p.r_pad / 4;
+    // this CTA's 64 / S rows; four consecutive columns per task; pad columns -> 0
+    const int rows_per = BM / S, quads = p.r_pad / 4;
     // per-call scale: LR carries 2^(k_alpha - j) so that kernel 2's single
     // factor 2^j restores it (a power of two: exact before the bf16 rounding)
     const float lrs = p.amax_parts ? *lr_scale_s : 1.f;
@@ -325,8 +340,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       if (c < p.r_tot) {
         const uint32_t a = part + (uint32_t)(rr * ps + c) * 4;
-#pragma unroll
-        for (int q = 0; q < KSPLIT; ++q) {   // fixed order: CTA 0, 1
+        for (int q = 0; q < S; ++q) {   // fixed order: CTA 0, 1, .., S-1
           const float4 v = dsmem_ld_f32x4(dsmem_map(a, (uint32_t)q));
           acc.x += v.x;
           acc.y += v.y;
@@ -373,24 +387,83 @@ size_t quant_down_smem_bytes(int r_tot, bool do_lr, int* stages_out, int ns) {
   return (size_t)L.bar_off + 1024 /*alignment slack*/ + 8 * (2 * stages + 1) + 16 + 128 * 4 + 64;
 }
 
-cudaError_t launch_quant_down(const CUtensorMap& tmX, K1Params p, cudaStream_t stream) {
-  const int ns = (p.K_pad / BK + 1) / 2;   // the larger of the two CTAs' stage counts
-  const size_t smem = quant_down_smem_bytes(p.r_tot, p.do_lr != 0, &p.stages, ns);
+namespace {
+
+// Clusters of s CTAs (with `smem` bytes each) that the current device runs at
+// once, from the occupancy query, remembered per (device, s, smem).
+int resident_clusters(int s, size_t smem, const cudaLaunchConfig_t& base_cfg) {
+  struct Entry {
+    int dev, s;
+    size_t smem;
+    int n;
+  };
+  static std::mutex mu;
+  static Entry table[64];
+  static int used = 0;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    for (int i = 0; i < used; ++i)
+      if (table[i].dev == dev && table[i].s == s && table[i].smem == smem) return table[i].n;
+  }
+  cudaLaunchConfig_t cfg = base_cfg;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = s;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  cfg.gridDim = dim3((unsigned)s);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, quant_down_kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  if (used < 64) table[used++] = Entry{dev, s, smem, n};
+  return n;
+}
+
+}  // namespace
+
+cudaError_t launch_quant_down(const CUtensorMap& tmX, K1Params p, int num_sms, cudaStream_t stream) {
+  // row blocks up to the next multiple of 128, so that every row of the last
+  // 128-row scale block gets its (zero) scales
+  const int row_blocks = round_up(p.M, 128) / BM, nk = p.K_pad / BK;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(THREADS);
+  cfg.stream = stream;
+  // K split: 2 (the whole grid in one wave at the FLUX batch sizes); 4 or 8
+  // when that still fits in one wave with every cluster resident, so that a
+  // small batch spreads over more SMs (each CTA then walks fewer stages)
+  int S = 2;
+  size_t smem = 0;
+  for (int cand = 8; cand >= 2; cand /= 2) {
+    if (cand > nk || cand * row_blocks > num_sms) continue;
+    smem = quant_down_smem_bytes(p.r_tot, p.do_lr != 0, &p.stages, (nk + cand - 1) / cand);
+    if (smem > 227 * 1024) return cudaErrorInvalidValue;
+    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(quant_down_kernel), smem);
+    if (e != cudaSuccess) return e;
+    cfg.dynamicSmemBytes = smem;
+    if (!p.do_lr || resident_clusters(cand, smem, cfg) >= row_blocks) {
+      S = cand;
+      break;
+    }
+  }
+  p.ksplit = S;
+  smem = quant_down_smem_bytes(p.r_tot, p.do_lr != 0, &p.stages, (nk + S - 1) / S);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;   // never launch past the shared-memory limit
   cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(quant_down_kernel), smem);
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  // row blocks up to the next multiple of 128, so that every row of the last
-  // 128-row scale block gets its (zero) scales
-  cfg.gridDim = dim3((unsigned)(KSPLIT * (round_up(p.M, 128) / BM)));
-  cfg.blockDim = dim3(THREADS);
+  cfg.gridDim = dim3((unsigned)(S * row_blocks));
   cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = KSPLIT;
+  attr[1].val.clusterDim.x = S;
   attr[1].val.clusterDim.y = 1;
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;

@@ -166,8 +166,16 @@ def y_check(Y_gpu: np.ndarray, Y_o: np.ndarray, rel: float = 1e-2, slack=0.0):
 # correctly rounded.  For these the bar is: every element over 1e-2 rms is at
 # most one bf16 ulp (plus the LR slack) from the oracle.
 ULP_EXCEPTIONS = {
-    "qkv_nvfp4_full", "qkv_int4_full", "mlp_fc1_full", "mlp_fc2_full", "lora_sweep_full", "awq_qkv_full",
+    "qkv_nvfp4_full", "qkv_int4_full", "mlp_fc1_full", "mlp_fc2_full", "lora_sweep_full",
     "dynamic_qkv_full",
+    # the plain W4A4 GEMM (no low-rank branch) of the unfused-path tests: its
+    # output is alpha Q(X^) Q(R) + b alone, whose largest elements reach
+    # 2.6 - 4.5 rms(Y) (the low-rank branch carries much of the signal)
+    "plain_w4a4_nvfp4", "plain_w4a4_int4",
+    # the naive four-launch path ("Nunchaku engine design" figure (a)): its
+    # up projection reads the GEMM's bf16 Y back and rounds Y + LR L2 to bf16
+    # again, a second rounding the fused layer does not have
+    "unfused_nvfp4", "unfused_int4",
 }
 
 

@@ -44,8 +44,12 @@ class Awq:
         raw = read_device(i.code, (K // 32) * i.N_pad * 16).reshape(K // 32, i.N_pad, 16)
         code = np.empty((K, i.N_pad), np.uint8)
         for b in range(16):
-            code[2 * b::32, :] = raw[:, :, b] & 0xF
-            code[2 * b + 1::32, :] = raw[:, :, b] >> 4
+            # byte b is byte b % 4 of word b // 4, i.e. nibble positions
+            # p = 2 (b % 4) (low) and p + 1 (high); position p holds
+            # k = 8 (b // 4) + i with p = i // 2 + 4 (i % 2)
+            order = [0, 2, 4, 6, 1, 3, 5, 7]
+            code[8 * (b // 4) + order[2 * (b % 4)]::32, :] = raw[:, :, b] & 0xF
+            code[8 * (b // 4) + order[2 * (b % 4) + 1]::32, :] = raw[:, :, b] >> 4
         scale = read_device(i.scale, (K // 64) * i.N_pad * 2).view(np.float16).reshape(K // 64, i.N_pad)
         zero = read_device(i.zero, (K // 64) * i.N_pad).reshape(K // 64, i.N_pad)
         inv_s = read_device(i.inv_s, K * 4).view(np.float32)

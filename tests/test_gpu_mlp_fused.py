@@ -34,13 +34,17 @@ def B():
     return binding
 
 
-def _pair(M, K1, N1, N2, seed):
+def _pair(M, K1, N1, N2, seed, rank2=32, lora2=0):
     g = torch.Generator("cpu").manual_seed(seed)
     fc1 = workloads.draw_layer("mlp_fc1", "nvfp4", M, K1, N1, 32, seed=seed, gelu=True, gen=g)
     W2, b2, _ = workloads.draw_weight_only(N1, N2, workloads.n_outliers(N1), g)
     g1 = GpuLayer("nvfp4", fc1.X, fc1.W, fc1.bias, 32)
     Y1_o = S.forward(g1.pw, fc1.X, gelu=True)["Y"].astype(np.float32)
-    g2 = GpuLayer("nvfp4", Y1_o, W2, b2, 32)
+    A2 = B2 = None
+    if lora2:   # a LoRA on fc2 (A: N1 x l, B: l x N2, N(0, 0.01)), appended to its factors
+        A2 = (torch.randn(N1, lora2, generator=g) * 0.01).to(torch.bfloat16).float().numpy()
+        B2 = (torch.randn(lora2, N2, generator=g) * 0.01).to(torch.bfloat16).float().numpy()
+    g2 = GpuLayer("nvfp4", Y1_o, W2, b2, rank2, A2, B2)
     return fc1, g1, g2, Y1_o
 
 
@@ -58,8 +62,17 @@ def _chain_check(B, g1, g2, X, Y1_o):
     return rel_rms, rel_max
 
 
-def test_emit_matches_the_unfused_gpu_path(B):
-    fc1, g1, g2, _ = _pair(200, 512, 768, 256, seed=70)
+@pytest.mark.parametrize("M,K1,N1,N2,rank2,lora2", [
+    (200, 512, 768, 256, 32, 0),
+    # fc2 with a LoRA (r_tot 48) and at the largest rank emit mode takes (64)
+    (200, 512, 768, 256, 32, 16),
+    (130, 256, 512, 256, 48, 16),
+    # 160 tiles on 148 SMs: some CTAs take two, so a tile's partial runs inside
+    # the next tile's k-loop; one 256-wide k-tile per tile
+    (1280, 256, 4096, 256, 32, 16),
+])
+def test_emit_matches_the_unfused_gpu_path(B, M, K1, N1, N2, rank2, lora2):
+    fc1, g1, g2, _ = _pair(M, K1, N1, N2, seed=70 + rank2 + lora2, rank2=rank2, lora2=lora2)
     try:
         M = fc1.M
         Xd = dev_bf16(fc1.X)

@@ -38,74 +38,65 @@ def test_atom_layout_of_weight_scales_fills_its_buffer_once():
     assert np.array_equal(np.sort(off.ravel()), np.arange(N_pad * K_pad // 16))
 
 
-# ---------------------------------------------------------------- emit mode's L1 fragments
-def l1frag_offset(k, r):
-    """bf16 offset of L1 element (k, r) in emit mode's fragment-ordered copy,
-    as kernels.h states it."""
-    G, kk = k >> 4, k & 15
-    t = 4 * (r & 7) + (kk >> 2)
-    return ((G * 32 + t) * 8 + 2 * (r >> 3)) * 2 + (kk & 3)
+# ---------------------------------------------------------------- emit mode's LR partial
+def stash_block(q):
+    """64-wide block of tile columns held by 64-wide block q of the emit
+    stash, as gemm_nvfp4.cu states it."""
+    return ((q & 1) << 1) | (q >> 1)
 
 
-def test_l1frag_formula_is_the_one_in_the_kernel_header():
+def test_stash_block_formula_is_the_one_in_the_kernel():
     import os
-    src = open(os.path.join(os.path.dirname(__file__), "..", "rank_gemm_b200", "csrc", "kernels.h")).read()
-    assert "const int G = k >> 4, kk = k & 15, t = 4 * (r & 7) + (kk >> 2);" in src
-    assert "return (((size_t)G * 32 + t) * 8 + 2 * (r >> 3)) * 2 + (kk & 3);" in src
+    src = open(os.path.join(os.path.dirname(__file__), "..", "rank_gemm_b200", "csrc", "gemm_nvfp4.cu")).read()
+    assert "return ((q & 1u) << 1) | (q >> 1);" in src
 
 
-def test_l1frag_fills_its_buffer_once():
-    K_pad = 512
-    k = np.arange(K_pad)[:, None]
-    r = np.arange(32)[None, :]
-    off = l1frag_offset(k, r).ravel()
-    assert np.array_equal(np.sort(off), np.arange(32 * K_pad))
+def test_emit_partial_over_the_stash_is_the_product():
+    """The next layer's LR partial of one tile, simulated step by step: the
+    epilogue warps park the tile's bf16 output in the stash (warp column set
+    ch, 32-column chunk c = tile columns ch 64 + 128 (c / 2) + 32 (c % 2) ..
+    +31, pair j of a chunk at stash column ch 64 + 16 c + j, the even column
+    in the low half); the MMA warp then takes K16 steps j = 0..15 with A =
+    stash columns 8 j .. 8 j + 7 (16 bf16 in order) and B = the L1 box
+    stash_block(j / 4) at k offset 16 (j % 4).  Integer data, so equality is
+    exact."""
+    rng = np.random.default_rng(7)
+    R, r_tot = 128, 32
+    Y = rng.integers(-8, 9, size=(R, 256))            # the tile: rows x its 256 columns
+    L1 = rng.integers(-8, 9, size=(256, r_tot))       # the next layer's L1 rows of those columns
+    stash = np.zeros((R, 256), dtype=np.int64)        # bf16 positions (two per 32-bit column)
+    for ch in range(2):
+        for c in range(4):
+            for j in range(16):
+                for e in range(2):
+                    n = ch * 64 + 128 * (c >> 1) + 32 * (c & 1) + 2 * j + e
+                    t = ch * 64 + 16 * c + j
+                    stash[:, 2 * t + e] = Y[:, n]
+    D = np.zeros((R, r_tot), dtype=np.int64)
+    for j in range(16):
+        blk = stash_block(j >> 2)
+        D += stash[:, 16 * j: 16 * j + 16] @ L1[64 * blk + 16 * (j & 3): 64 * blk + 16 * (j & 3) + 16, :]
+    assert np.array_equal(D, Y @ L1)
 
 
-def test_emit_lr_partial_fragments_multiply_to_the_product():
-    """One warp's LR partial over one 16-column group, simulated lane by lane:
-    A fragments as tcgen05.ld.16x256b returns them from the bf16-pair stash
-    (lane t: rows t/4 and t/4 + 8 of its 16-row half, TMEM columns 2(t%4) and
-    2(t%4)+1, each column one pair of adjacent k), assigned to the mma slots
-    as the kernel does (a0 = r0, a1 = r2, a2 = r1, a3 = r3); B fragments read
-    from the l1frag buffer (words 2 nt, 2 nt + 1 of the lane); the product
-    formed with mma.m16n8k16's fragment semantics (PTX ISA: A a0 (row g,
-    k 2q, 2q+1), a1 (row g+8), a2/a3 the same at k + 8; B b0 (k 2q, 2q+1,
-    col g), b1 at k + 8; D d0 d1 (row g, cols 2q, 2q+1), d2 d3 at row g+8;
-    g = lane / 4, q = lane % 4).  Integer data, so equality is exact."""
-    rng = np.random.default_rng(5)
-    G = 3                                              # the group's index along K
-    A = rng.integers(-8, 9, size=(32, 16))             # this warp's 32 rows x the group's 16 k
-    L1 = rng.integers(-8, 9, size=(16 * (G + 1), 32))  # L1 rows for groups 0..G, 32 ranks
-    buf = np.zeros(32 * 16 * (G + 1), dtype=np.int64)
-    for kk in range(16 * (G + 1)):
-        for rr in range(32):
-            buf[l1frag_offset(kk, rr)] = L1[kk, rr]
-
-    def pair(row, col):                                # TMEM column col of a row: k = 2 col, 2 col + 1
-        return (A[row, 2 * col], A[row, 2 * col + 1])
-
-    D = np.zeros((32, 32), dtype=np.int64)
-    for h in range(2):                                 # the two 16-row halves
-        Aslot = np.zeros((16, 16), dtype=np.int64)     # the A the mma sees (slot k order)
-        for t in range(32):
-            g, q = t >> 2, t & 3
-            r0 = pair(16 * h + g, 2 * q)
-            r1 = pair(16 * h + g, 2 * q + 1)
-            r2 = pair(16 * h + g + 8, 2 * q)
-            r3 = pair(16 * h + g + 8, 2 * q + 1)
-            a = (r0, r2, r1, r3)                       # the kernel's slot assignment
-            Aslot[g, 2 * q: 2 * q + 2] = a[0]
-            Aslot[g + 8, 2 * q: 2 * q + 2] = a[1]
-            Aslot[g, 2 * q + 8: 2 * q + 10] = a[2]
-            Aslot[g + 8, 2 * q + 8: 2 * q + 10] = a[3]
-        for nt in range(4):
-            Bslot = np.zeros((16, 8), dtype=np.int64)
-            for t in range(32):
-                g, q = t >> 2, t & 3
-                w = (G * 32 + t) * 8 + 2 * nt          # the lane's word 2 nt (b0), 2 nt + 1 (b1)
-                Bslot[2 * q: 2 * q + 2, g] = buf[2 * w: 2 * w + 2]
-                Bslot[2 * q + 8: 2 * q + 10, g] = buf[2 * w + 2: 2 * w + 4]
-            Dt = Aslot @ Bslot
-            D[16 * h: 16 * h + 16, 8 * nt: 8 * nt + 8] = Dt
-    assert np.array_equal(D, A @ L1[16 * G: 16 * G + 16, :])
+def test_emit_iteration_schedule_places_one_partial_per_tile():
+    """Kernel 2's k-iteration order in emit mode: per tile the FP4 k-tiles
+    and low-rank chunks in order, with the previous tile's partial stage
+    after FP4 k-tile min(3, nk - 1), none in the first tile, one extra after
+    the last; the producer and the MMA warp use the same order."""
+    def iter_of(it, nk, with_part, emit_at=3):
+        if not with_part:
+            return (0, it) if it < nk else (1, it - nk)
+        at = min(emit_at, nk - 1) + 1
+        if it < at:
+            return (0, it)
+        if it == at:
+            return (2, 0)
+        return (0, it - 1) if it - 1 < nk else (1, it - 1 - nk)
+    for nk in (1, 2, 4, 12, 48):
+        for nl in (0, 1, 2):
+            for with_part in (False, True):
+                seq = [iter_of(it, nk, with_part) for it in range(nk + nl + (1 if with_part else 0))]
+                assert [i for k, i in seq if k == 0] == list(range(nk))
+                assert [i for k, i in seq if k == 1] == list(range(nl))
+                assert sum(k == 2 for k, _ in seq) == (1 if with_part else 0)

@@ -200,3 +200,12 @@ def awq_adaln(M: int = 1) -> AwqLayer:
     if M != 1:
         d["name"] = "awq_w4a16_adaln_M%d_K3072_N18432" % M
     return draw_awq_layer(**d)
+
+
+def awq_qkv() -> AwqLayer:
+    """The QKV workload's activation, weight and bias as an AWQ W4A16 layer
+    (no AWQ scale): the W4A16 side of the W4A4-over-W4A16 comparison on the
+    same shape (M=4608, K=3072, N=9216)."""
+    L = qkv()
+    return AwqLayer(name="awq_w4a16_qkv_M4608_K3072_N9216", M=L.M, K=L.K, N=L.N, X=L.X, W=L.W, bias=L.bias,
+                    s=None, seed=L.seed)
