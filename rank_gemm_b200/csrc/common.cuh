@@ -193,12 +193,6 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads) {
 }
 
 // ----------------------------------------------------------------- thread-block clusters
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
 // Every thread of every CTA in the cluster arrives, then waits for all.
 // Release/acquire order the shared-memory writes before it against the
 // distributed-shared-memory reads after it.
@@ -213,11 +207,6 @@ __device__ __forceinline__ uint32_t dsmem_map(uint32_t smem_addr, uint32_t rank)
   return r;
 }
 
-__device__ __forceinline__ float dsmem_ld_f32(uint32_t cluster_addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
-  return v;
-}
 
 // Shared-memory matrix descriptor (tcgen05 "matrix descriptor"):
 //   bits  0-13 start address >> 4, 16-29 leading byte offset >> 4,
@@ -271,15 +260,6 @@ __device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t a, uint64_t b
       : "memory");
 }
 
-// Copies a 512-byte scale-factor atom (32 rows x 16 bytes, contiguous in smem)
-// to 4 TMEM columns starting at `taddr`, replicated into all four 32-lane
-// sub-partitions.
-__device__ __forceinline__ void tmem_cp_sf_atom(uint32_t taddr, uint32_t smem_addr) {
-  const uint64_t d = smem_desc(smem_addr, 0, 128, 0);
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d)
-               : "memory");
-}
-
 // One 4 KB replicated scale block (see sfx_rep_offset) -> 8 TMEM columns of all 128 lanes.
 __device__ __forceinline__ void tmem_cp_sf_block(uint32_t taddr, uint32_t smem_addr) {
   const uint64_t d = smem_desc(smem_addr, 128, 256, 0);
@@ -320,81 +300,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 }
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
-// Per-warpgroup register budget change (every warp of the warpgroup runs it).
-template <int N>
-__device__ __forceinline__ void regs_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <int N>
-__device__ __forceinline__ void regs_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-
-// ----------------------------------------------------------------- CTA pairs (cta_group::2)
-// Two CTAs of a cluster (ranks 2i, 2i+1) run one MMA over both SMs: A rows
-// and B rows come half from each CTA's shared memory (same offsets), D rows
-// 0-127 land in the even CTA's TMEM and 128-255 in the odd CTA's.  TMA loads
-// of both CTAs complete on the even CTA's mbarrier (`bar` is a
-// shared::cluster address, see dsmem_map).
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* tmap, int x, int y,
-                                                 uint32_t bar_cluster) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(bar_cluster)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
-               "r"(ncols)
-               : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish_pair() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-               : "memory");
-}
-// Arrives once on the barrier at offset `bar` in every CTA of `cta_mask` when
-// the tcgen05 operations this thread issued before have completed.
-__device__ __forceinline__ void tc_commit_pair(uint32_t bar, uint16_t cta_mask) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
-          bar),
-      "h"(cta_mask)
-      : "memory");
-}
-__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                              uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void mma_nvf4_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                              uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], "
-      "p;\n\t}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-      : "memory");
-}
-// tmem_cp_sf_atom for the pair: each CTA's atom at `smem_addr` goes to its own TMEM.
-__device__ __forceinline__ void tmem_cp_sf_atom_pair(uint32_t taddr, uint32_t smem_addr) {
-  const uint64_t d = smem_desc(smem_addr, 0, 128, 0);
-  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d)
-               : "memory");
-}
-// Arrive on an mbarrier of another CTA of the cluster (shared::cluster address).
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
 
 
@@ -439,22 +344,7 @@ __device__ __forceinline__ void mul2_rn(float a0, float a1, float b0, float b1, 
   asm("mov.b64 {%0, %1}, %2;" : "=f"(r0), "=f"(r1) : "l"(r));
 }
 
-// (r0, r1) = fl32(a * b + c) element-wise, one packed instruction.
-__device__ __forceinline__ void fma2_rn(float a0, float a1, float b0, float b1, float& c0, float& c1) {
-  uint64_t a, b, c, r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(b) : "f"(b0), "f"(b1));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(c) : "f"(c0), "f"(c1));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(c0), "=f"(c1) : "l"(r));
-}
 
-// Packed float32 pairs in 64-bit registers (element 0 in the low half): a * b + c.
-__device__ __forceinline__ uint64_t fma2_u64(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
 
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float r;
