@@ -42,7 +42,7 @@ sys.path.insert(0, ROOT)
 WORKLOAD = dict(name="nvfp4_qkv_M4608_K3072_N9216_r32", fmt="nvfp4", M=4608, K=3072, N=9216, rank=32)
 # --workload: the QKV projection is the bench line; the others are the
 # remaining parity configurations, timed the same way for their profiles.
-WORKLOADS = ("qkv", "int4_qkv", "mlp_fc1", "mlp_fc2", "lora", "awq_adaln", "mlp_pair", "small", "lora_sweep", "awq_qkv")
+WORKLOADS = ("qkv", "int4_qkv", "mlp_fc1", "mlp_fc2", "lora", "awq_adaln", "mlp_pair", "small", "lora_sweep", "awq_qkv", "library_fp4")
 INT8_PER_BF16 = 2.0         # nominal dense INT8 : BF16 tensor throughput (4.5 : 2.25)
 METRIC = "SVDQuant W4A4 linear effective TFLOPS & % of FP4 tensor peak; µs/layer"
 UNIT = "TFLOP/s"
@@ -1041,6 +1041,80 @@ def run_awq_qkv(args, world, rank, local):
         print(json.dumps(out), flush=True)
 
 
+def run_library_fp4(args, world, rank, local):
+    """Context, not a product path: library NVFP4 GEMMs (flashinfer's mm_fp4
+    with its cuDNN, CUTLASS and TRT-LLM backends, plain GEMM without the
+    low-rank branch) and torch's bf16 matmul on the QKV shape, beside this
+    library's kernel 2 (plain and with the fused low-rank branch), CUDA
+    events on the same stream, the same box.  Backends that fail to build or
+    run are reported as such."""
+    import numpy as np
+    import torch
+    from rank_gemm_b200 import build as _b
+    _b.build()
+    from rank_gemm_b200 import binding as B
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    M, N, K = WORKLOAD["M"], WORKLOAD["N"], WORKLOAD["K"]
+    flops = 2.0 * M * N * K
+    n = max(10, min(args.steps, 100))
+
+    def timed(fn):
+        for _ in range(5):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n * 1e3
+
+    print("library_fp4: timing this library's kernel 2", file=sys.stderr, flush=True)
+    out = {"metric": "NVFP4 GEMM on the QKV shape, library kernels beside this library's kernel 2 (context)",
+           "unit": "us", "n_gpus": 1, "steps": n, "higher_is_better": False,
+           "config": {"workload": WORKLOAD["name"], "M": M, "K": K, "N": N}, "results": {}}
+    lay = build_layer("qkv", B, torch, dev)
+    h, X0 = lay["h"], lay["X0"]
+    qb, sb, lb = B.svdq_act_buffer_sizes(h, M)
+    qX, sX, LR = (torch.empty(v, dtype=torch.uint8, device=dev) for v in (qb, sb, lb))
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    B.svdq_quantize_act_lowrank_down(h, M, X0, qX, sX, LR, stream)
+    t = timed(lambda: B.svdq_w4a4_gemm(h, M, qX, sX, Y, stream))
+    out["results"]["svdq kernel 2, plain W4A4"] = {"us": round(t, 2), "tflops": round(flops / t / 1e6, 1)}
+    t = timed(lambda: B.svdq_w4a4_gemm_lowrank_up(h, M, qX, sX, LR, B.SVDQ_EPI_NONE, Y, stream))
+    out["results"]["svdq kernel 2, fused low-rank branch"] = {"us": round(t, 2), "tflops": round(flops / t / 1e6, 1)}
+    B.svdq_free_weights(h)
+    g = torch.Generator(device="cpu").manual_seed(0)
+    a = torch.randn(M, K, generator=g).to(torch.bfloat16).to(dev)
+    bm = torch.randn(N, K, generator=g).to(torch.bfloat16).to(dev)
+    t = timed(lambda: a @ bm.T)
+    out["results"]["torch bf16 matmul"] = {"us": round(t, 2), "tflops": round(flops / t / 1e6, 1)}
+    try:
+        import flashinfer
+        from flashinfer import SfLayout, mm_fp4, nvfp4_quantize
+        ag = (448 * 6) / a.float().abs().max()
+        bg = (448 * 6) / bm.float().abs().max()
+        for backend, shuffle in (("cudnn", False), ("cutlass", False), ("trtllm", True)):
+            print("library_fp4: flashinfer backend", backend, file=sys.stderr, flush=True)
+            try:
+                a4, asf = nvfp4_quantize(a, ag, sfLayout=SfLayout.layout_128x4, do_shuffle=False)
+                b4, bsf = nvfp4_quantize(bm, bg, sfLayout=SfLayout.layout_128x4, do_shuffle=shuffle)
+                y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+                alpha = torch.tensor([1.0 / (ag * bg)], dtype=torch.float32, device=dev)
+                t = timed(lambda: mm_fp4(a4, b4.T, asf, bsf.T, alpha, torch.bfloat16, y, backend=backend))
+                out["results"]["flashinfer mm_fp4 " + backend] = {"us": round(t, 2), "tflops": round(flops / t / 1e6, 1)}
+            except Exception as ex:
+                out["results"]["flashinfer mm_fp4 " + backend] = {"unavailable": "%s: %s" % (type(ex).__name__,
+                                                                                           str(ex)[:200])}
+        out["flashinfer"] = getattr(flashinfer, "__version__", "?")
+    except Exception as ex:
+        out["results"]["flashinfer"] = {"unavailable": "%s: %s" % (type(ex).__name__, str(ex)[:200])}
+    print(json.dumps(out), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -1061,6 +1135,9 @@ def main():
         run_mlp_pair(args, world, rank, local)
     elif args.workload == "awq_qkv":
         run_awq_qkv(args, world, rank, local)
+    elif args.workload == "library_fp4":
+        if rank == 0:
+            run_library_fp4(args, world, rank, local)
     elif args.workload in ("small", "lora_sweep"):
         run_points(args, world, rank, local, args.workload)
     else:

@@ -18,13 +18,13 @@
 //               tcgen05.mma.kind::f16 (bf16, K = 16) per k-tile into one of two
 //               128 x 256 float32 accumulators (the epilogue of one tile runs
 //               under the MMAs of the next).
-//   warps 2-9   dequantizers, one thread per output feature of the tile: per
-//               k-tile the feature's 64 codes become 64 bf16 weights written
-//               as one 128-byte row of the K-major, 128-byte-swizzled B tile
-//               (a 3-stage ring of its own), with the exact pair arithmetic
-//               below; with an AWQ scale they also rewrite the X tile as
-//               bf16(x / s) in place.
-//   warps 10-13 epilogue, one per TMEM sub-partition: accumulator + bias ->
+//   warps 2-17  dequantizers, two threads per output feature of the tile
+//               (one per 32-k chunk): per k-tile the feature's 64 codes become
+//               64 bf16 weights written as one 128-byte row of the K-major,
+//               128-byte-swizzled B tile (a 3-stage ring of its own), with the
+//               exact pair arithmetic below; with an AWQ scale they also
+//               rewrite the X tile as bf16(x / s) in place.
+//   warps 18-21 epilogue, one per TMEM sub-partition: accumulator + bias ->
 //               bf16, 32-byte stores.
 // Dequantization, two weights per instruction: the codes of k and k + 1 sit
 // at bits 4j and 16 + 4j of their word (awq_nibble_pos), so one shift and one
@@ -41,9 +41,9 @@ namespace svdq {
 namespace {
 
 constexpr int BM = 128, BN = 256, BK = 64;
-constexpr int DQ_WARPS = 8;                                  // BN features, one per thread
+constexpr int DQ_WARPS = 16;                                 // BN features x two 32-k chunks, one per thread
 constexpr int EPI_WARPS = 4;
-constexpr int THREADS = 32 * (2 + DQ_WARPS + EPI_WARPS);     // 448
+constexpr int THREADS = 32 * (2 + DQ_WARPS + EPI_WARPS);     // 704
 constexpr int W_PROD = 0, W_MMA = 1, W_DQ0 = 2, W_EPI0 = 2 + DQ_WARPS;
 constexpr int NS_A = 4, NS_B = 3;
 constexpr int X_BYTES = BM * BK * 2;                         // 16 KB
@@ -210,7 +210,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp < W_EPI0) {
     // ------------------------------------------------------------ dequantizers
-    const int n = threadIdx.x - 32 * W_DQ0;   // feature of the tile, 0..255
+    const int t = threadIdx.x - 32 * W_DQ0;   // 0..511
+    const int n = t & 255, h = t >> 8;         // feature of the tile, 32-k chunk
     uint32_t it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
@@ -228,25 +229,25 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t DH = bf16_bits(dh) * 0x10001u, DL = bf16_bits(dl) * 0x10001u;
         const uint32_t z = sg[OFF_ZERO + n];
         const uint32_t ZZ = 0x43004300u | (z << 16) | z;                       // (128 + zero, 128 + zero)
-        const uint4 c0 = lds128(smem_u32(sg + OFF_CODE + n * 16));            // k 0..31 of the tile
-        const uint4 c1 = lds128(smem_u32(sg + OFF_CODE + 4096 + n * 16));     // k 32..63
+        const uint4 c0 = lds128(smem_u32(sg + OFF_CODE + h * 4096 + n * 16));   // k 32h .. 32h + 31
         const uint32_t row = smem_u32(ringB + sb * B_BYTES) + (uint32_t)n * 128;
         const uint32_t sw = (uint32_t)(n & 7);
-        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const uint32_t words[4] = {c0.x, c0.y, c0.z, c0.w};
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {   // 16-byte chunk c = k 8c .. 8c + 7
-          const uint4 v = dequant_word(words[c], ZZ, DH, DL);
+        for (int q = 0; q < 4; ++q) {   // 16-byte chunk c = 4h + q = k 8c .. 8c + 7
+          const uint32_t c = 4 * h + q;
+          const uint4 v = dequant_word(words[q], ZZ, DH, DL);
           sts128(row + ((c ^ sw) << 4), v.x, v.y, v.z, v.w);
         }
         if (HAS_S) {
           // X tile in place: x' = bf16(fl32(x * fl32(1/s))); thread t takes
           // row t / 2, chunks 4 (t % 2) .. + 3
-          const int r = n >> 1;
+          const int r = t >> 2;
           const uint32_t xrow = smem_u32(ringA + sa * A_STAGE) + (uint32_t)r * 128;
           const float* invs = reinterpret_cast<const float*>(sg + OFF_INVS);
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            const int c = 4 * (n & 1) + cc;
+          for (int cc = 0; cc < 2; ++cc) {
+            const int c = 2 * (t & 3) + cc;
             const uint32_t addr = xrow + ((uint32_t)(c ^ (r & 7)) << 4);
             const uint4 x = lds128(addr);
             const float4 i0 = *reinterpret_cast<const float4*>(invs + 8 * c);

@@ -143,13 +143,14 @@ __device__ __forceinline__ uint32_t stash_block(uint32_t q) { return ((q & 1u) <
 
 }  // namespace
 
-// EMIT: instead of Y, write the next layer's kernel-1 outputs from this
-// layer's bf16 output (see K2Params::Next).
-template <bool EMIT>
+// MODE 0: the layer.  MODE 1 (emit): instead of Y, write the next layer's
+// kernel-1 outputs from this layer's bf16 output (see K2Params::Next).
+template <int MODE>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const __grid_constant__ CUtensorMap tmLR, const __grid_constant__ CUtensorMap tmL2,
                       K2Params p) {
+  constexpr bool EMIT = MODE == 1;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* bias_s = reinterpret_cast<float*>(base + STAGES * STAGE_BYTES);
@@ -201,6 +202,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t phase = 0;
       bool ok = true;
       int prev_nb = -1;   // emit mode: the previous tile's column block
+      // the weight tiles (codes and scales) stay in L2 ahead of the streamed
+      // activations and outputs: every row block's CTA reads them again
+      const uint64_t keep = l2_policy_evict_last();
       // one more pass of the loop in emit mode: the last tile's partial stage
       for (int tile = blockIdx.x; ok && (tile < num_tiles || (EMIT && prev_nb >= 0)); tile += gridDim.x) {
         const bool last = tile >= num_tiles;
@@ -217,12 +221,13 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t bar = smem_u32(&ctl->full[stage]);
           const Iter I = last ? Iter{2, 0} : iter_of(it, p.nk, with_part);
           if (I.kind == 0) {
+            const int kt = I.idx;
             mbar_arrive_expect_tx(bar, STAGE_BYTES);
-            tma_load_2d(st, &tmA, I.idx * 128, mb * BLOCK_M, bar);
-            tma_load_2d(st + A_BYTES, &tmB, I.idx * 128, nb * BLOCK_N, bar);
-            bulk_load(st + A_BYTES + B_BYTES, p.sX + ((size_t)mb * p.nk + I.idx) * SFA_BYTES, SFA_BYTES, bar);
-            bulk_load(st + A_BYTES + B_BYTES + SFA_BYTES, p.sR + ((size_t)nb * p.nk + I.idx) * SFB_BYTES,
-                      SFB_BYTES, bar);
+            tma_load_2d(st, &tmA, kt * 128, mb * BLOCK_M, bar);
+            tma_load_2d_hint(st + A_BYTES, &tmB, kt * 128, nb * BLOCK_N, bar, keep);
+            bulk_load(st + A_BYTES + B_BYTES, p.sX + ((size_t)mb * p.nk + kt) * SFA_BYTES, SFA_BYTES, bar);
+            bulk_load_hint(st + A_BYTES + B_BYTES + SFA_BYTES, p.sR + ((size_t)nb * p.nk + kt) * SFB_BYTES,
+                           SFB_BYTES, bar, keep);
           } else if (I.kind == 1) {
             mbar_arrive_expect_tx(bar, A_BYTES + B_BYTES);
             tma_load_2d(st, &tmLR, I.idx * 64, mb * BLOCK_M, bar);
@@ -502,7 +507,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 cudaError_t launch_gemm_nvfp4(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmLR,
                               const CUtensorMap& tmL2, K2Params p, int num_sms, cudaStream_t stream, bool emit_next) {
   void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap, K2Params) =
-      emit_next ? gemm_nvfp4_kernel<true> : gemm_nvfp4_kernel<false>;
+      emit_next ? gemm_nvfp4_kernel<1> : gemm_nvfp4_kernel<0>;
   cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), SMEM_BYTES);
   if (e != cudaSuccess) return e;
   const int tiles = p.num_m_blocks * p.num_n_blocks;

@@ -100,3 +100,40 @@ def test_emit_iteration_schedule_places_one_partial_per_tile():
                 assert [i for k, i in seq if k == 0] == list(range(nk))
                 assert [i for k, i in seq if k == 1] == list(range(nl))
                 assert sum(k == 2 for k, _ in seq) == (1 if with_part else 0)
+
+
+# ---------------------------------------------------------------- K splits over a cluster
+def _slices(nk, S):
+    """[k0, k0 + n) of each CTA of a cluster of S: nk / S each, the first nk % S
+    one more (kernel 1's 256-column stages)."""
+    q, r = divmod(nk, S)
+    return [(c * q + min(c, r), q + (1 if c < r else 0)) for c in range(S)]
+
+
+def test_k_slices_cover_every_k_tile_once_in_order():
+    for nk in range(1, 60):
+        for S in (1, 2, 4, 8):
+            if S > nk:
+                continue
+            sl = _slices(nk, S)
+            assert all(n >= 1 for _, n in sl)
+            flat = [k for k0, n in sl for k in range(k0, k0 + n)]
+            assert flat == list(range(nk))
+
+
+def test_split_formulas_are_the_kernels():
+    import os
+    d = os.path.join(os.path.dirname(__file__), "..", "rank_gemm_b200", "csrc")
+    k1 = open(os.path.join(d, "quant_down.cu")).read()
+    assert "const int ns = nq + (split < nr ? 1 : 0);" in k1
+    assert "const int kb0 = split * nq + min(split, nr);" in k1
+
+
+def test_split_rows_cover_the_tile():
+    """Each CTA of kernel 1's cluster finishes 64 / S rows of the 64-row block:
+    disjoint, complete."""
+    for rows in (64,):
+        for S in (1, 2, 4, 8):
+            per = rows // S
+            got = sorted(r for c in range(S) for r in range(c * per, (c + 1) * per))
+            assert got == list(range(rows))
