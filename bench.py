@@ -403,7 +403,12 @@ def run_ours(args, world, rank, local):
     # the contraction's own peak: FP4 (NVFP4) or INT8 (INT4 codes run on the
     # int8 tensor core), each the measured bf16 peak times the nominal ratio
     ratio = FP4_PER_BF16 if nv else INT8_PER_BF16
-    tc_peak = peaks["bf16"] * ratio
+    # a long back-to-back run that met the power cap is held to the measured
+    # sustained peak (the bf16 GEMM looped for seconds under the same cap);
+    # a run that did not is held to the burst figure
+    capped = "sw_power_cap" in clocks.summary().get("reasons", []) and peaks["bf16_sustained"]
+    tc_peak = (peaks["bf16_sustained"] if capped else peaks["bf16"]) * ratio
+    peak_kind = "sustained" if capped else "burst"
     k2_tflops = flops / (k2_ms * 1e-3) / 1e12
     # algorithmic bytes: each operand once, scales counted once (the four
     # replicas kernel 2 reads are an implementation cost and show in traffic)
@@ -496,8 +501,10 @@ def run_ours(args, world, rank, local):
                                 % (sets * (M * K * 2 + M * N * 2 + qb + sb + lb) / 1e6)},
                "roofline": {"kernel": "%s (kernel 2)" % k2_src[:-3], "bound": "tensor", "achieved": round(k2_tflops, 2),
                             "peak": round(tc_peak, 1), "unit": "TFLOP/s", "frac": round(k2_tflops / tc_peak, 4),
-                            "peak_source": "%s bf16 %.1f TFLOP/s x %.0f (nominal %s:BF16)"
-                                           % (peaks["source"], peaks["bf16"], ratio, "FP4" if nv else "INT8"),
+                            "peak_source": "%s %s bf16 %.1f TFLOP/s x %.0f (nominal %s:BF16)%s"
+                                           % (peaks["source"], peak_kind, tc_peak / ratio, ratio,
+                                              "FP4" if nv else "INT8",
+                                              "; the timed region ran under sw_power_cap" if capped else ""),
                             "traffic": traffic, "algorithmic_bytes": bytes_k2, "us": round(k2_ms * 1e3, 2)},
                "roofline_k1": {"kernel": "quant_down (kernel 1)", "bound": "hbm",
                                "achieved": round(bytes_k1 / (k1_ms * 1e-3) / 1e9, 1), "peak": peaks["hbm"],

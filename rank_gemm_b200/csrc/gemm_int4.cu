@@ -10,10 +10,13 @@
 // an E4M3 copy next to the packed codes), so TMA stages them straight into
 // the operand tiles.  Every group runs as two tcgen05.mma.kind::f8f6f4
 // (K = 32) into a fresh fp32 TMEM tile, whose sums (|.| <= 64 * 64) are exact;
-// CUDA cores apply sX sR and accumulate in fp32 registers with packed f32x2
-// multiply and FMA, one instruction per output element per group: the bound
-// of this kernel.  (A first version unpacked packed int4 tiles in shared
-// memory for every output tile; that byte shuffling set its pace.)
+// CUDA cores apply sX sR and accumulate in fp32 registers: a packed f32x2
+// multiply forms two scale products, one scalar FMA per output element per
+// group adds the rescaled sum (scalar FMAs read the TMEM-load registers as
+// they are; packed FMAs needed a register-pair copy per pair).  That
+// arithmetic is the bound of this kernel.  (A first version unpacked packed
+// int4 tiles in shared memory for every output tile; that byte shuffling set
+// its pace.)
 //
 // One 128 x 128 output tile per CTA at a time, persistent over tiles:
 //   warp 0       TMA producer: per 128-wide k-tile the [128 x 128 B] E4M3
@@ -24,8 +27,10 @@
 //                groups into the two halves of one of two TMEM buffers; the
 //                low-rank chunks as kind::f16 into one more buffer use).
 //   warps 2-17   rescale + epilogue: 4 warps per TMEM sub-partition, 32 columns
-//                each, one barrier round trip per k-tile (two groups); fp32
-//                accumulators in registers; bias, GELU, bf16 store.
+//                each, one barrier round trip per k-tile (two groups), read
+//                from TMEM in 16-column chunks with each chunk's load issued
+//                before the previous chunk's arithmetic; fp32 accumulators in
+//                registers; bias, GELU, bf16 store.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -73,19 +78,49 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
 __device__ __forceinline__ uint64_t u2(uint32_t lo, uint32_t hi) { return ((uint64_t)hi << 32) | lo; }
 __device__ __forceinline__ void lds2x64(uint32_t addr, uint64_t& a, uint64_t& b) {
   asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "r"(addr));
+}
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+// 32 lanes x 16 consecutive 32-bit columns -> 16 registers per thread.
+__device__ __forceinline__ void tmem_ld16_i4(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+// Waits for this thread's TMEM loads; r is passed through, so no use of the
+// loaded registers can be scheduled before the wait.
+__device__ __forceinline__ void tmem_wait_ld16(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+               :
+               : "memory");
+}
+// acc[off .. off + 7] += (sx sr) d for 16 columns: d = the group's exact
+// fp32 sums, sx sr the product of two binary16 scales (exact in fp32)
+__device__ __forceinline__ void rescale16(float (&acc)[32], int off, const uint32_t (&r)[16], uint64_t sx2,
+                                          uint32_t sra) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint64_t sr01, sr23;
+    lds2x64(sra + q * 16, sr01, sr23);
+    const uint64_t c01 = f2_mul(sx2, sr01), c23 = f2_mul(sx2, sr23);
+    float* a = acc + 2 * off + 4 * q;
+    a[0] = fmaf(__uint_as_float((uint32_t)c01), __uint_as_float(r[4 * q]), a[0]);
+    a[1] = fmaf(__uint_as_float((uint32_t)(c01 >> 32)), __uint_as_float(r[4 * q + 1]), a[1]);
+    a[2] = fmaf(__uint_as_float((uint32_t)c23), __uint_as_float(r[4 * q + 2]), a[2]);
+    a[3] = fmaf(__uint_as_float((uint32_t)(c23 >> 32)), __uint_as_float(r[4 * q + 3]), a[3]);
+  }
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -255,9 +290,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const int mb = tile % p.num_m_blocks, nb = tile / p.num_m_blocks;
       const int m = mb * BM + row, n0 = nb * BN + quarter * RS_COLS;
-      uint64_t acc[RS_COLS / 2];                   // 32 columns as float32 pairs
+      float acc[RS_COLS];
 #pragma unroll
-      for (int i = 0; i < RS_COLS / 2; ++i) acc[i] = 0ull;
+      for (int i = 0; i < RS_COLS; ++i) acc[i] = 0.f;
       bool ok = true;
       for (int kt = 0; ok && kt < nk; ++kt) {
         if (!mbar_wait(smem_u32(&ctl->cfull[c]), cph, abort_flag, p.err)) {
@@ -272,32 +307,29 @@ __global__ void __launch_bounds__(THREADS, 1)
           break;
         }
         tc_fence_after();
-        // the two groups' sums of this warp's 32 columns; after the second
-        // load the buffer goes back to the MMA warp
+        // the two groups' sums of this warp's 32 columns in four 16-column
+        // chunks, each chunk's TMEM load issued before the previous chunk's
+        // arithmetic; after the last load the buffer goes back to the MMA warp
         const uint32_t taddr = tmem + ((uint32_t)(sub * 32) << 16) + buf * KB_COLS + quarter * RS_COLS;
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {                // the k-tile's two 64-groups
-          uint32_t r[32];
-          tmem_ld32(taddr + j * BN, r);
-          tmem_wait_ld();
-          if (j == 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&ctl->dempty[buf]));
-          }
-          const uint32_t sxb = __float_as_uint(sc[j * 128 + row]);
-          const uint64_t sx2 = u2(sxb, sxb);
-          const uint32_t sra = smem_u32(sc + 256 + j * 128 + quarter * RS_COLS);
-          // acc += (sx sr) d: the group's exact fp32 sum, rescaled by the
-          // product of two binary16 scales (exact in fp32), then one FMA
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            uint64_t sr01, sr23;
-            lds2x64(sra + q * 16, sr01, sr23);
-            acc[2 * q] = f2_fma(f2_mul(sx2, sr01), u2(r[4 * q], r[4 * q + 1]), acc[2 * q]);
-            acc[2 * q + 1] = f2_fma(f2_mul(sx2, sr23), u2(r[4 * q + 2], r[4 * q + 3]), acc[2 * q + 1]);
-          }
-        }
+        const uint32_t scb = smem_u32(sc);
+        const uint32_t sx0 = lds_u32(scb + 4u * row), sx1 = lds_u32(scb + 4u * (128 + row));
+        const uint32_t sra = scb + 4u * (256 + quarter * RS_COLS);
+        uint32_t ra[16], rb[16];
+        tmem_ld16_i4(taddr, ra);
+        tmem_wait_ld16(ra);
+        tmem_ld16_i4(taddr + 16, rb);
+        rescale16(acc, 0, ra, u2(sx0, sx0), sra);
+        tmem_wait_ld16(rb);
+        tmem_ld16_i4(taddr + BN, ra);
+        rescale16(acc, 8, rb, u2(sx0, sx0), sra + 64);
+        tmem_wait_ld16(ra);
+        tmem_ld16_i4(taddr + BN + 16, rb);
+        rescale16(acc, 0, ra, u2(sx1, sx1), sra + 512);
+        tmem_wait_ld16(rb);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&ctl->dempty[buf]));
+        rescale16(acc, 8, rb, u2(sx1, sx1), sra + 512 + 64);
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&ctl->cempty[c]));   // this warp is done with the k-tile's scales
         if (++c == SC) {
@@ -320,7 +352,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&ctl->dempty[buf]));
 #pragma unroll
-          for (int i = 0; i < 16; ++i) acc[i] = f2_add(acc[i], u2(r[2 * i], r[2 * i + 1]));
+          for (int i = 0; i < 32; ++i) acc[i] += __uint_as_float(r[i]);
         }
       }
       if (!ok) break;
@@ -337,8 +369,7 @@ __global__ void __launch_bounds__(THREADS, 1)
               const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
-                const uint64_t a2 = acc[(c16 + 4 * q + e) >> 1];
-                y[4 * q + e] = __uint_as_float((e & 1) ? (uint32_t)(a2 >> 32) : (uint32_t)a2) + bb[e];
+                y[4 * q + e] = acc[c16 + 4 * q + e] + bb[e];
                 if (p.epi == 1) y[4 * q + e] = gelu_tanh(y[4 * q + e]);
               }
             }

@@ -66,6 +66,28 @@ def test_linear_noalloc_matches_linear_on_two_calls(B, fmt, gelu):
         g.close()
 
 
+def test_linear_noalloc_takes_no_device_memory(B):
+    """After a first call (which may load the library's module and with it
+    the scratch array), a call changes neither the device's free memory nor
+    the caching allocator's count: nothing is allocated behind the caller."""
+    L = workloads.draw_layer("noalloc_mem", "nvfp4", 300, 1024, 768, 32, seed=65, n_out=4)
+    g = GpuLayer(L.fmt, L.X, L.W, L.bias, L.rank)
+    try:
+        Xd = dev_bf16(L.X)
+        Y = torch.empty(L.M, L.N, dtype=torch.bfloat16, device="cuda")
+        B.svdq_linear_noalloc(g.h, L.M, Xd, B.SVDQ_EPI_NONE, Y)
+        torch.cuda.synchronize()
+        free0, alloc0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
+        for _ in range(3):
+            B.svdq_linear_noalloc(g.h, L.M, Xd, B.SVDQ_EPI_NONE, Y)
+        torch.cuda.synchronize()
+        assert torch.cuda.mem_get_info()[0] == free0
+        assert torch.cuda.memory_allocated() == alloc0
+        assert B.svdq_poll_device_error() == 0
+    finally:
+        g.close()
+
+
 def test_linear_noalloc_at_the_size_limit_then_smaller(B):
     """The largest M the array takes, then a smaller M: the second call reads
     nothing the first one left behind."""
