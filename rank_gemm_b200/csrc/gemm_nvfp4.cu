@@ -56,7 +56,7 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0, SFA_COL = 256, SFB_COL = 272;
 constexpr uint32_t STASH_COL = 320;   // emit mode: bf16 pairs of the row slices, 64 columns per half
 constexpr uint32_t DPART_COL = 448;   // emit mode: the next layer's LR partial, up to 64 float32 columns
-constexpr int EMIT_AT = 3;            // emit mode: the partial's stage follows this FP4 k-tile of the next tile
+constexpr int EMIT_AT = 6;            // emit mode: the partial's stage follows this FP4 k-tile of the next tile
 constexpr uint32_t IDESC_F4 = idesc_nvf4(BLOCK_M, BLOCK_N);
 constexpr uint32_t IDESC_BF = idesc_bf16_f32(BLOCK_M, BLOCK_N);
 

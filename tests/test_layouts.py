@@ -1,5 +1,7 @@
 """Host checks of the documented byte layouts (no GPU): every formula in the
 public header that places an element must be a bijection onto its buffer."""
+import itertools
+
 import numpy as np
 
 
@@ -82,9 +84,14 @@ def test_emit_partial_over_the_stash_is_the_product():
 def test_emit_iteration_schedule_places_one_partial_per_tile():
     """Kernel 2's k-iteration order in emit mode: per tile the FP4 k-tiles
     and low-rank chunks in order, with the previous tile's partial stage
-    after FP4 k-tile min(3, nk - 1), none in the first tile, one extra after
-    the last; the producer and the MMA warp use the same order."""
-    def iter_of(it, nk, with_part, emit_at=3):
+    after FP4 k-tile min(EMIT_AT, nk - 1), none in the first tile, one extra
+    after the last; the producer and the MMA warp use the same order.  Checked
+    for the kernel's EMIT_AT (read from its source) and other placements."""
+    import os, re
+    src = open(os.path.join(os.path.dirname(__file__), "..", "rank_gemm_b200", "csrc", "gemm_nvfp4.cu")).read()
+    kernel_at = int(re.search(r"constexpr int EMIT_AT = (\d+);", src).group(1))
+
+    def iter_of(it, nk, with_part, emit_at):
         if not with_part:
             return (0, it) if it < nk else (1, it - nk)
         at = min(emit_at, nk - 1) + 1
@@ -93,13 +100,12 @@ def test_emit_iteration_schedule_places_one_partial_per_tile():
         if it == at:
             return (2, 0)
         return (0, it - 1) if it - 1 < nk else (1, it - 1 - nk)
-    for nk in (1, 2, 4, 12, 48):
-        for nl in (0, 1, 2):
-            for with_part in (False, True):
-                seq = [iter_of(it, nk, with_part) for it in range(nk + nl + (1 if with_part else 0))]
-                assert [i for k, i in seq if k == 0] == list(range(nk))
-                assert [i for k, i in seq if k == 1] == list(range(nl))
-                assert sum(k == 2 for k, _ in seq) == (1 if with_part else 0)
+    for emit_at, nk, nl, with_part in itertools.product((kernel_at, 0, 3, 11), (1, 2, 4, 7, 12, 48), (0, 1, 2),
+                                                       (False, True)):
+        seq = [iter_of(it, nk, with_part, emit_at) for it in range(nk + nl + (1 if with_part else 0))]
+        assert [i for k, i in seq if k == 0] == list(range(nk))
+        assert [i for k, i in seq if k == 1] == list(range(nl))
+        assert sum(k == 2 for k, _ in seq) == (1 if with_part else 0)
 
 
 # ---------------------------------------------------------------- K splits over a cluster
