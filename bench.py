@@ -684,8 +684,9 @@ def run_points(args, world, rank, local, which):
     a rank-16 LoRA).  Every timed call is preceded by an untimed write of a
     buffer twice the L2 size and a read of another one, so weights and
     activations come from HBM as they do when a model runs the layer once per
-    block, and the L2 holds no dirty lines to write back; a call is timed with
-    CUDA events on its stream.  Per point: the layer (kernel 1 + kernel 2),
+    block, and the L2 holds no dirty lines to write back; a call's time is the
+    difference of two event-timed loops on its stream (with and without the
+    call).  Per point: the layer (kernel 1 + kernel 2),
     kernel 2 alone (after an untimed kernel 1), the plain W4A4 path
     (quantize + GEMM without the low-rank branch) and their ratio."""
     import numpy as np
@@ -722,23 +723,34 @@ def run_points(args, world, rank, local, which):
         return torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16).to(dev)
 
     def timed(fn, pre=None, n=100):
-        """Median over n calls of fn's device time, L2 flushed before each."""
+        """Mean device time of fn with the L2 flushed (and pre run) before
+        every call: a loop of n x [flush, pre, fn] between two events minus a
+        loop of n x [flush, pre], each loop taken three times (medians).  CUDA
+        event timestamps on this part step by about 1 us, too coarse for one
+        call of a few microseconds, so no single-call interval is used."""
+        def loop(with_fn):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            a.record(stream)
+            for _ in range(n):
+                flush_l2()
+                if pre:
+                    pre()
+                if with_fn:
+                    fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            return a.elapsed_time(b)
         for _ in range(3):
             flush_l2()
             if pre:
                 pre()
             fn()
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
-        torch.cuda.synchronize()
-        for a, b in evs:
-            flush_l2()
-            if pre:
-                pre()
-            a.record(stream)
-            fn()
-            b.record(stream)
-        torch.cuda.synchronize()
-        return statistics.median(a.elapsed_time(b) for a, b in evs) * 1e3
+        t1, t0 = [], []
+        for _ in range(3):
+            t1.append(loop(True))
+            t0.append(loop(False))
+        return (statistics.median(t1) - statistics.median(t0)) / n * 1e3
 
     if which == "small":
         L = workloads.small()
@@ -806,7 +818,8 @@ def run_points(args, world, rank, local, which):
                           "parallelism": "replicas x%d (each rank its own batch)" % world,
                           "l2": "before every timed call a %d MB buffer is written and another read (2 x L2 each): "
                                 "cold L2, no dirty lines" % (2 * l2 // 2 ** 20),
-                          "timing": "median of %d calls per point, CUDA events around each" % n},
+                          "timing": "mean of %d calls per point: a loop of [flush, call] minus a loop of [flush], "
+                                    "CUDA events at the loop ends, median of 3 each" % n},
                "points": points, "device_status": status, "clocks": clocks.summary(),
                "gpu_launches": 2 * n * len(points)}
         if one:
