@@ -188,6 +188,10 @@ def assert_y(Y_gpu, Y_o, rel=1e-2, slack=0.0, exception=None):
         assert r["n_over"] == 0, r
     else:
         assert exception in ULP_EXCEPTIONS, exception
+        # the record of the exception: how many elements are over the bar and
+        # the worst ones (row, column, GPU, oracle, |dY| / rms, |dY| in ulps)
+        print("ulp exception %s: n_over %d of %d, max |dY| / rms %.5f, worst %s"
+              % (exception, r["n_over"], np.asarray(Y_o).size, r["max_rel_rms"], r["over"][:3]))
         assert r["n_bad"] == 0, r
     return r
 
