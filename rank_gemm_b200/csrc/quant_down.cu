@@ -237,6 +237,21 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     // NVFP4: packed codes (K_pad / 2 bytes a row); INT4: one E4M3 byte per code
     const size_t qx_row_bytes = p.fmt == 0 ? (size_t)(p.K_pad / 2) : (size_t)p.K_pad;
+    // this thread's store addresses at its first stage; each further stage
+    // moves them by one 256-column k-tile: codes by 128 (NVFP4) or 256 (INT4)
+    // bytes, replicated NVFP4 scales by two 4 KB blocks, INT4 scales by 512 floats
+    uint8_t* qxp[2];
+    uint8_t* sxp[2];
+    bool in_rows[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int m = m0 + qr + 32 * h, kb = 4 * kb0 + qb;
+      in_rows[h] = m < p.M;
+      qxp[h] = p.qX + (size_t)m * qx_row_bytes + (size_t)kb * (p.fmt == 0 ? 32 : 64) + qg * (p.fmt == 0 ? 8 : 16);
+      sxp[h] = p.fmt == 0 ? p.sX + sfx_rep_offset(m, kb, qg, p.K_pad)
+                          : p.sX + 4 * int4_scale_offset(m, kb, p.K_pad);
+    }
+    const size_t qx_step = p.fmt == 0 ? 128 : 256, sx_step = p.fmt == 0 ? 8192 : 2048;
     for (int it = 0; it < ns; ++it) {
       const int s = it % p.stages;
       if (!mbar_wait(smem_u32(&full[s]), (it / p.stages) & 1, abort_flag, p.err)) break;
@@ -274,8 +289,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (lane == 0) mbar_arrive_relaxed(smem_u32(&empty[s]));
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int kb = 4 * (kb0 + it) + qb;              // 64-column block
-        const int m = m0 + qr + 32 * h;
         uint2 codes;
         if (p.fmt == 0) {
           uint32_t sc;
@@ -285,20 +298,24 @@ __global__ void __launch_bounds__(THREADS, 1)
           uint32_t sw = sc << (8 * qg);
           sw |= __shfl_xor_sync(0xffffffffu, sw, 1);
           sw |= __shfl_xor_sync(0xffffffffu, sw, 2);
-          *reinterpret_cast<uint32_t*>(p.sX + sfx_rep_offset(m, kb, qg, p.K_pad)) = sw;
+          *reinterpret_cast<uint32_t*>(sxp[h]) = sw;
         } else {
           __half sc;
           quant_int4_16of64(v[h], codes, sc);
           // stored widened to float32 (exact): kernel 2 multiplies in float32
-          if (qg == 0) reinterpret_cast<float*>(p.sX)[int4_scale_offset(m, kb, p.K_pad)] = __half2float(sc);
+          if (qg == 0) *reinterpret_cast<float*>(sxp[h]) = __half2float(sc);
         }
-        if (m < p.M) {
+        if (in_rows[h]) {
           if (p.fmt == 0)
-            *reinterpret_cast<uint2*>(p.qX + (size_t)m * qx_row_bytes + (size_t)kb * 32 + qg * 8) = codes;
+            *reinterpret_cast<uint2*>(qxp[h]) = codes;
           else
-            *reinterpret_cast<uint4*>(p.qX + (size_t)m * qx_row_bytes + (size_t)kb * 64 + qg * 16) =
-                int4x16_to_e4m3(codes);
+            *reinterpret_cast<uint4*>(qxp[h]) = int4x16_to_e4m3(codes);
         }
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        qxp[h] += qx_step;
+        sxp[h] += sx_step;
       }
     }
   }
@@ -441,8 +458,11 @@ cudaError_t launch_quant_down(const CUtensorMap& tmX, K1Params p, int num_sms, c
   cfg.stream = stream;
   // K split: 2 (the whole grid in one wave at the FLUX batch sizes); 4 or 8
   // when that still fits in one wave with every cluster resident, so that a
-  // small batch spreads over more SMs (each CTA then walks fewer stages)
-  int S = 2;
+  // small batch spreads over more SMs (each CTA then walks fewer stages);
+  // none when even S = 2 would need more than one wave: each CTA then walks
+  // all of K and skips the cluster reduction, whose tail every wave would pay
+  // (LoRA-sweep layer at M = 16384: 136.0 -> 126.1 us)
+  int S = 2 * row_blocks > num_sms ? 1 : 2;
   size_t smem = 0;
   for (int cand = 8; cand >= 2; cand /= 2) {
     if (cand > nk || cand * row_blocks > num_sms) continue;
