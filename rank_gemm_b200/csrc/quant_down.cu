@@ -4,7 +4,8 @@
 // so they are fused and X is read from HBM once).
 //
 // A cluster of S CTAs (S = 2 at large batches, up to 8 at small ones, so that
-// the grid still fills the SMs) owns 64 rows of X; CTA c of the cluster walks
+// the grid still fills the SMs; 1 when a split grid would need two waves)
+// owns 64 rows of X; CTA c of the cluster walks
 // the c-th of S slices of K in 256-column stages.  A producer warp keeps a TMA ring of
 // stages in flight; a stage holds the [64 x 256] bf16 tile of X (four
 // 128-byte-swizzled [64 x 64] boxes: 512 contiguous bytes of every row, which
@@ -15,11 +16,13 @@
 //   * 16 quantizer warps: every thread two 16-element groups of one row
 //     (x^ = x / lambda, amax, block scale, 4-bit codes), written packed with
 //     scales in the layout kernel 2's tensor-core MMA consumes;
-//   * one thread issues the down projection on the 5th-generation tensor core:
-//     A = the staged X tile (M = 64 rows), B = the L1f^T tile (N = r_tot),
-//     fp32 accumulation in TMEM across the CTA's half of K.
-// At the end four warps move the partial [64 x r_tot] tile from TMEM to
-// shared memory; after a cluster barrier CTA c adds the S partials of rows
+//   * two threads (of two warps) issue the down projection on the
+//     5th-generation tensor core: A = the staged X tile (M = 64 rows), B = the
+//     L1f^T tile (N = r_tot), the lower and the upper 128 columns of every
+//     stage into two fp32 TMEM accumulators across the CTA's slice of K.
+// At the end four warps move the partial [64 x r_tot] tile (the sum of the two
+// accumulators) from TMEM to shared memory; after a cluster barrier CTA c
+// adds the S partials of rows
 // [64c/S, 64(c+1)/S) through distributed shared memory, always in the order
 // CTA 0, 1, .., S-1 (so LR is the same on every run), and stores LR in bf16.
 // Why 64 rows: the four-way split of a 128-row tile needs clusters of four,
@@ -27,7 +30,7 @@
 // 64-row clusters of two fill every SM at the FLUX batch sizes, and small
 // batches split K further instead of leaving SMs idle.
 // Stages are released through an mbarrier (the 16 quantizer warps plus the
-// MMA commit) instead of a CTA-wide sync, so warps drift apart and overlap
+// two MMA commits) instead of a CTA-wide sync, so warps drift apart and overlap
 // their load, math and store phases.  The kernel is HBM-bound: per row it
 // reads 2K bytes of X and writes about K/2 + K/16 bytes of codes and scales
 // plus 2 r_pad bytes of LR.
@@ -43,15 +46,18 @@ namespace {
 constexpr int BM = K1_BOX_ROWS;              // rows per cluster (= MMA M = TMA box rows)
 constexpr int BK = 256;                      // K columns per stage (four 64-column swizzled boxes)
 constexpr int QWARPS = 16;                   // quantizer warps: 64 rows x 8 groups
-constexpr int THREADS = 32 * (QWARPS + 2);   // + producer warp + MMA warp
+constexpr int THREADS = 32 * (QWARPS + 4);   // + producer warp, two MMA warps, one idle warp
 constexpr int X_BOX = BM * 128;              // one [64 x 64] bf16 box, 8 KB
 constexpr int X_BYTES = 4 * X_BOX;           // 32 KB
 constexpr int IL_BYTES = BK * 4;             // 1/lambda for the stage
-// Warp roles.  Warp w runs on SM sub-partition w % 4: the MMA warp (2) and
-// the producer (3) share theirs with three quantizer warps each, so the
-// single MMA-issuing thread competes with fewer busy warps (kernel 1 alone on
-// QKV 14.0 -> 13.3 us); quantizers are warps 0, 1 and 4..17.
-constexpr int W_PROD = 3, W_MMA = 2, W_Q0 = 4;
+// Warp roles.  Warp w runs on SM sub-partition w % 4: the first MMA warp (2)
+// and the producer (3) share theirs with three quantizer warps each, so an
+// MMA-issuing thread competes with fewer busy warps (kernel 1 alone on QKV
+// 14.0 -> 13.3 us); quantizers are warps 0, 1 and 4..17.  A second MMA warp
+// (19, sub-partition 3) issues the upper half of every stage's K16 steps into
+// an accumulator of its own, which halves the issue work per thread (the
+// down projection alone 9.8 -> 8.6 us on QKV); warp 18 has no role.
+constexpr int W_PROD = 3, W_MMA = 2, W_Q0 = 4, W_IDLE = 18, W_MMA2 = 19;
 constexpr int MAX_STAGES = 8;
 
 __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
@@ -133,16 +139,16 @@ __global__ void __launch_bounds__(THREADS, 1)
     tma_prefetch_desc(&tmX);
     for (int s = 0; s < p.stages; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
-      mbar_init(smem_u32(&empty[s]), (p.do_quant ? QWARPS : 0) + (p.do_lr ? 1 : 0));
+      mbar_init(smem_u32(&empty[s]), (p.do_quant ? QWARPS : 0) + (p.do_lr ? 2 : 0));
     }
-    mbar_init(smem_u32(dfull), 1);
+    mbar_init(smem_u32(dfull), 2);
     *abort_flag = 0;
     fence_barrier_init();
   }
   float* lr_scale_s = inv_tab + 128;                                 // per-call scale only
   if (p.fmt == 0 && !p.amax_parts && tid < 128) inv_tab[tid] = nvfp4_inv_entry((uint32_t)tid, p.s_t);
   if (p.do_lr && warp == W_MMA) {
-    tmem_alloc(smem_u32(tmem_slot), tmem_cols);
+    tmem_alloc(smem_u32(tmem_slot), 2 * tmem_cols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -168,9 +174,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         bulk_load(smem_u32(base + L.il_ring + s * IL_BYTES), p.inv_lambda + kb * BK, IL_BYTES, bar);
       }
     }
-  } else if (warp == W_MMA) {
+  } else if (warp == W_MMA || warp == W_MMA2) {
     // ---------------------------------------------------------------- tensor-core down projection
     if (p.do_lr && lane == 0) {
+      const int half = warp == W_MMA2 ? 1 : 0;   // K16 steps 8 half .. 8 half + 7 of every stage
+      const uint32_t acc = tmem + (uint32_t)half * tmem_cols;
       const uint32_t idesc = idesc_bf16_f32(BM, p.r_tot);
       uint32_t started = 0;
       bool ok = true;
@@ -190,16 +198,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t lstep = (uint32_t)p.r_tot * 8;   // (r_tot * 128) >> 4
         if (kvalid >= BK) {
 #pragma unroll
-          for (int j = 0; j < BK / 16; ++j) {
+          for (int jj = 0; jj < BK / 32; ++jj) {
+            const int j = 8 * half + jj;
             const uint32_t b = j >> 2, ko = (j & 3) * 2;
-            mma_bf16(tmem, dx + (b * (X_BOX >> 4) + ko), dl + (b * lstep + ko), idesc, (j == 0) ? started : 1u);
+            mma_bf16(acc, dx + (b * (X_BOX >> 4) + ko), dl + (b * lstep + ko), idesc, (jj == 0) ? started : 1u);
           }
           started = 1u;
         } else {
-          for (int j = 0; j < BK / 16; ++j) {
+          for (int jj = 0; jj < BK / 32; ++jj) {
+            const int j = 8 * half + jj;
             if (j * 16 >= kvalid) break;
             const uint32_t b = j >> 2, ko = (j & 3) * 2;
-            mma_bf16(tmem, dx + (b * (X_BOX >> 4) + ko), dl + (b * lstep + ko), idesc, started);
+            mma_bf16(acc, dx + (b * (X_BOX >> 4) + ko), dl + (b * lstep + ko), idesc, started);
             started = 1u;
           }
         }
@@ -207,7 +217,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (ok) tc_commit(smem_u32(dfull));
     }
-  } else if (p.do_quant) {
+  } else if (p.do_quant && warp != W_IDLE) {
     // ---------------------------------------------------------------- quantizers
     // box qb, rows qr and qr + 32, 16-column group qg of the stage: both of a
     // thread's groups use the same 16 values of 1/lambda (read once); a warp
@@ -332,13 +342,22 @@ __global__ void __launch_bounds__(THREADS, 1)
       // rank index; lanes 16-31 of each sub-partition are unused
       const int sub = warp & 3, row = 16 * sub + lane;
       const bool has_mma = ns > 0 && kb0 * BK < p.K;     // else this slice is empty or in the K pad: zeros
+      const bool has_mma2 = ns > 0 && p.K - kb0 * BK > BK / 2;   // the second accumulator got at least one step
       if (mbar_wait(smem_u32(dfull), 0, abort_flag, p.err)) {
         tc_fence_after();
         for (int c0 = 0; c0 < p.r_tot; c0 += 32) {
           uint32_t d[32];
           if (has_mma) {
             tmem_ld32(tmem + ((uint32_t)(sub * 32) << 16) + (uint32_t)c0, d);
-            tmem_wait_ld();
+            if (has_mma2) {
+              uint32_t e[32];
+              tmem_ld32(tmem + ((uint32_t)(sub * 32) << 16) + tmem_cols + (uint32_t)c0, e);
+              tmem_wait_ld();
+#pragma unroll
+              for (int n = 0; n < 32; ++n) d[n] = __float_as_uint(__uint_as_float(d[n]) + __uint_as_float(e[n]));
+            } else {
+              tmem_wait_ld();
+            }
           } else {
 #pragma unroll
             for (int n = 0; n < 32; ++n) d[n] = 0u;
@@ -393,7 +412,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   if (p.do_lr && warp == W_MMA) {
     tc_fence_after();
-    tmem_dealloc(tmem, tmem_cols);
+    tmem_dealloc(tmem, 2 * tmem_cols);
   }
 }
 
