@@ -161,9 +161,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == W_PROD) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
-      for (int it = 0; it < ns; ++it) {
-        const int s = it % p.stages;
-        if (!mbar_wait(smem_u32(&empty[s]), ((it / p.stages) & 1) ^ 1, abort_flag, p.err)) break;
+      for (int it = 0, s = 0, ph = 0; it < ns; ++it, s = (s + 1 == p.stages) ? 0 : s + 1, ph ^= (s == 0) ? 1 : 0) {
+        if (!mbar_wait(smem_u32(&empty[s]), (uint32_t)ph ^ 1u, abort_flag, p.err)) break;
         const int kb = kb0 + it;
         const uint32_t bar = smem_u32(&full[s]);
         mbar_arrive_expect_tx(bar, X_BYTES + L.l_bytes + IL_BYTES);
@@ -182,9 +181,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t idesc = idesc_bf16_f32(BM, p.r_tot);
       uint32_t started = 0;
       bool ok = true;
-      for (int it = 0; it < ns; ++it) {
-        const int s = it % p.stages;
-        if (!mbar_wait(smem_u32(&full[s]), (it / p.stages) & 1, abort_flag, p.err)) {
+      for (int it = 0, s = 0, ph = 0; it < ns; ++it, s = (s + 1 == p.stages) ? 0 : s + 1, ph ^= (s == 0) ? 1 : 0) {
+        if (!mbar_wait(smem_u32(&full[s]), (uint32_t)ph, abort_flag, p.err)) {
           ok = false;
           break;
         }
@@ -262,9 +260,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                           : p.sX + 4 * int4_scale_offset(m, kb, p.K_pad);
     }
     const size_t qx_step = p.fmt == 0 ? 128 : 256, sx_step = p.fmt == 0 ? 8192 : 2048;
-    for (int it = 0; it < ns; ++it) {
-      const int s = it % p.stages;
-      if (!mbar_wait(smem_u32(&full[s]), (it / p.stages) & 1, abort_flag, p.err)) break;
+    for (int it = 0, s = 0, ph = 0; it < ns; ++it, s = (s + 1 == p.stages) ? 0 : s + 1, ph ^= (s == 0) ? 1 : 0) {
+      if (!mbar_wait(smem_u32(&full[s]), (uint32_t)ph, abort_flag, p.err)) break;
       // this thread's two groups of the stage: rows qr and qr + 32 of box qb;
       // read both and form x^ = x * (1/lambda) in registers, release the
       // stage, then quantize and store
