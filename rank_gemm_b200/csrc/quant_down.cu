@@ -110,6 +110,9 @@ __host__ __device__ constexpr uint32_t tmem_cols_for(int r_tot) {
 
 }  // namespace
 
+// FMT: 0 NVFP4, 1 INT4 (one instantiation per format, so the stage loop has no
+// format branches)
+template <int FMT>
 __global__ void __launch_bounds__(THREADS, 1)
     quant_down_kernel(const __grid_constant__ CUtensorMap tmX, K1Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -146,7 +149,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     fence_barrier_init();
   }
   float* lr_scale_s = inv_tab + 128;                                 // per-call scale only
-  if (p.fmt == 0 && !p.amax_parts && tid < 128) inv_tab[tid] = nvfp4_inv_entry((uint32_t)tid, p.s_t);
+  if ((FMT == 0) && !p.amax_parts && tid < 128) inv_tab[tid] = nvfp4_inv_entry((uint32_t)tid, p.s_t);
   if (p.do_lr && warp == W_MMA) {
     tmem_alloc(smem_u32(tmem_slot), 2 * tmem_cols);
     tmem_relinquish();
@@ -244,7 +247,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       named_bar_sync(1, 32 * QWARPS);
     }
     // NVFP4: packed codes (K_pad / 2 bytes a row); INT4: one E4M3 byte per code
-    const size_t qx_row_bytes = p.fmt == 0 ? (size_t)(p.K_pad / 2) : (size_t)p.K_pad;
+    const size_t qx_row_bytes = (FMT == 0) ? (size_t)(p.K_pad / 2) : (size_t)p.K_pad;
     // this thread's store addresses at its first stage; each further stage
     // moves them by one 256-column k-tile: codes by 128 (NVFP4) or 256 (INT4)
     // bytes, replicated NVFP4 scales by two 4 KB blocks, INT4 scales by 512 floats
@@ -255,11 +258,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int h = 0; h < 2; ++h) {
       const int m = m0 + qr + 32 * h, kb = 4 * kb0 + qb;
       in_rows[h] = m < p.M;
-      qxp[h] = p.qX + (size_t)m * qx_row_bytes + (size_t)kb * (p.fmt == 0 ? 32 : 64) + qg * (p.fmt == 0 ? 8 : 16);
-      sxp[h] = p.fmt == 0 ? p.sX + sfx_rep_offset(m, kb, qg, p.K_pad)
+      qxp[h] = p.qX + (size_t)m * qx_row_bytes + (size_t)kb * ((FMT == 0) ? 32 : 64) + qg * ((FMT == 0) ? 8 : 16);
+      sxp[h] = (FMT == 0) ? p.sX + sfx_rep_offset(m, kb, qg, p.K_pad)
                           : p.sX + 4 * int4_scale_offset(m, kb, p.K_pad);
     }
-    const size_t qx_step = p.fmt == 0 ? 128 : 256, sx_step = p.fmt == 0 ? 8192 : 2048;
+    const size_t qx_step = (FMT == 0) ? 128 : 256, sx_step = (FMT == 0) ? 8192 : 2048;
     for (int it = 0, s = 0, ph = 0; it < ns; ++it, s = (s + 1 == p.stages) ? 0 : s + 1, ph ^= (s == 0) ? 1 : 0) {
       if (!mbar_wait(smem_u32(&full[s]), (uint32_t)ph, abort_flag, p.err)) break;
       // this thread's two groups of the stage: rows qr and qr + 32 of box qb;
@@ -297,7 +300,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint2 codes;
-        if (p.fmt == 0) {
+        if ((FMT == 0)) {
           uint32_t sc;
           quant_nvfp4_16_tab(v[h], six_st, inv_tab, codes, sc);
           // the row's four scale bytes form one word; kernel 2 wants it in four
@@ -313,7 +316,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (qg == 0) *reinterpret_cast<float*>(sxp[h]) = __half2float(sc);
         }
         if (in_rows[h]) {
-          if (p.fmt == 0)
+          if ((FMT == 0))
             *reinterpret_cast<uint2*>(qxp[h]) = codes;
           else
             *reinterpret_cast<uint4*>(qxp[h]) = int4x16_to_e4m3(codes);
@@ -454,7 +457,8 @@ int resident_clusters(int s, size_t smem, const cudaLaunchConfig_t& base_cfg) {
   cfg.numAttrs = 1;
   cfg.gridDim = dim3((unsigned)s);
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, quant_down_kernel, &cfg) != cudaSuccess) {
+  // both instantiations take the same threads and shared memory
+  if (cudaOccupancyMaxActiveClusters(&n, quant_down_kernel<0>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     n = 0;
   }
@@ -484,7 +488,8 @@ cudaError_t launch_quant_down(const CUtensorMap& tmX, K1Params p, int num_sms, c
     if (cand > nk || cand * row_blocks > num_sms) continue;
     smem = quant_down_smem_bytes(p.r_tot, p.do_lr != 0, &p.stages, (nk + cand - 1) / cand);
     if (smem > 227 * 1024) return cudaErrorInvalidValue;
-    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(quant_down_kernel), smem);
+    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(quant_down_kernel<0>), smem);
+    if (e == cudaSuccess) e = ensure_dynamic_smem(reinterpret_cast<const void*>(quant_down_kernel<1>), smem);
     if (e != cudaSuccess) return e;
     cfg.dynamicSmemBytes = smem;
     if (!p.do_lr || resident_clusters(cand, smem, cfg) >= row_blocks) {
@@ -495,7 +500,8 @@ cudaError_t launch_quant_down(const CUtensorMap& tmX, K1Params p, int num_sms, c
   p.ksplit = S;
   smem = quant_down_smem_bytes(p.r_tot, p.do_lr != 0, &p.stages, (nk + S - 1) / S);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;   // never launch past the shared-memory limit
-  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(quant_down_kernel), smem);
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(quant_down_kernel<0>), smem);
+  if (e == cudaSuccess) e = ensure_dynamic_smem(reinterpret_cast<const void*>(quant_down_kernel<1>), smem);
   if (e != cudaSuccess) return e;
   cfg.gridDim = dim3((unsigned)(S * row_blocks));
   cfg.dynamicSmemBytes = smem;
@@ -508,7 +514,8 @@ cudaError_t launch_quant_down(const CUtensorMap& tmX, K1Params p, int num_sms, c
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = p.do_lr ? 2 : 1;   // only the LR reduction needs the cluster
-  return cudaLaunchKernelEx(&cfg, quant_down_kernel, tmX, p);
+  return p.fmt == 0 ? cudaLaunchKernelEx(&cfg, quant_down_kernel<0>, tmX, p)
+                    : cudaLaunchKernelEx(&cfg, quant_down_kernel<1>, tmX, p);
 }
 
 }  // namespace svdq
